@@ -1,0 +1,188 @@
+"""Python wrapper of the CPU oracle (``qattn_oracle.c``) for the smoothed-K INT8 attention forward.
+
+TEST INFRASTRUCTURE ONLY: the test suite, the package smoke check and the benchmark's CPU-baseline
+leg are the only callers.  The product (the CUDA library and its Python binding) never imports
+this module.
+
+The C source states the method and the readings it follows (SageAttention summary page,
+aibr.jp/archives/102657, sec. 2-4).  This wrapper only marshals numpy arrays; every step of the
+arithmetic is in the C file.  fp16 arrays travel as their uint16 bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "qattn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+QBLOCK = 128  # Q quantization block (rows)
+KBLOCK = 64   # K quantization block (rows)
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2 -ffp-contract=off, no fast-math) if it is stale."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+               "-pthread", "-Wall", "-o", tmp, _SRC, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i = ctypes.c_int
+        L.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
+        L.oracle_f16_to_f64.restype = ctypes.c_double
+        L.oracle_f64_to_f16.argtypes = [ctypes.c_double]
+        L.oracle_f64_to_f16.restype = ctypes.c_uint16
+        L.oracle_k_channel_sums.argtypes = [P, i, i, i, i, P]
+        L.oracle_k_channel_sums.restype = None
+        L.oracle_mean_from_sum.argtypes = [ctypes.c_int64, i]
+        L.oracle_mean_from_sum.restype = ctypes.c_float
+        L.oracle_quantize_block.argtypes = [P, i, i, P]
+        L.oracle_quantize_block.restype = ctypes.c_float
+        L.oracle_smooth_quant.argtypes = [P, P, i, i, i, i, i, i, P, P, P, P, P]
+        L.oracle_smooth_quant.restype = None
+        L.oracle_qk_int32.argtypes = [P, P, i, i, i, i, i, i, i, i, i, i, i, P]
+        L.oracle_qk_int32.restype = None
+        L.oracle_attention_quantized.argtypes = [P, P, P, P, P, i, i, i, i, i, i, P, P,
+                                                 ctypes.c_long, P, i]
+        L.oracle_attention_quantized.restype = i
+        L.oracle_attention_fp64.argtypes = [P, P, P, i, i, i, i, i, i, i, P, P, ctypes.c_long, P, i]
+        L.oracle_attention_fp64.restype = i
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _bits16(x) -> np.ndarray:
+    """fp16 input (numpy float16 or uint16 bit patterns) as a contiguous uint16 array."""
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float16:
+        return x.view(np.uint16)
+    assert x.dtype == np.uint16, x.dtype
+    return x
+
+
+def f16_to_f64(bits: int) -> float:
+    return lib().oracle_f16_to_f64(int(bits))
+
+
+def f64_to_f16(x: float) -> int:
+    return int(lib().oracle_f64_to_f16(float(x)))
+
+
+def f64_to_f16_array(x: np.ndarray) -> np.ndarray:
+    f = lib().oracle_f64_to_f16
+    flat = np.asarray(x, dtype=np.float64).ravel()
+    return np.array([f(float(v)) for v in flat], dtype=np.uint16).reshape(np.shape(x))
+
+
+def k_channel_sums(k, B, Hkv, N, d) -> np.ndarray:
+    k = _bits16(k)
+    out = np.zeros((B, Hkv, d), dtype=np.int64)
+    lib().oracle_k_channel_sums(_ptr(k), B, Hkv, N, d, _ptr(out))
+    return out
+
+
+def mean_from_sum(s: int, N: int) -> np.float32:
+    return np.float32(lib().oracle_mean_from_sum(int(s), int(N)))
+
+
+def quantize_block(x: np.ndarray):
+    """x: float32 [rows, d] -> (int8 codes [rows, d], float32 scale)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    rows, d = x.shape
+    codes = np.zeros((rows, d), dtype=np.int8)
+    s = lib().oracle_quantize_block(_ptr(x), rows, d, _ptr(codes))
+    return codes, np.float32(s)
+
+
+def smooth_quant(q, k, B, H, Hkv, N, d, smooth=True):
+    """Returns dict with q_i8 [B,H,N,d], q_scale [B,H,ceil(N/128)], k_i8 [B,Hkv,N,d],
+    k_scale [B,Hkv,ceil(N/64)], k_mean [B,Hkv,d] (float32)."""
+    q = _bits16(q)
+    k = _bits16(k)
+    nqb = (N + QBLOCK - 1) // QBLOCK
+    nkb = (N + KBLOCK - 1) // KBLOCK
+    r = dict(
+        q_i8=np.zeros((B, H, N, d), dtype=np.int8),
+        q_scale=np.zeros((B, H, nqb), dtype=np.float32),
+        k_i8=np.zeros((B, Hkv, N, d), dtype=np.int8),
+        k_scale=np.zeros((B, Hkv, nkb), dtype=np.float32),
+        k_mean=np.zeros((B, Hkv, d), dtype=np.float32),
+    )
+    lib().oracle_smooth_quant(_ptr(q), _ptr(k), B, H, Hkv, N, d, 1 if smooth else 0,
+                              _ptr(r["q_i8"]), _ptr(r["q_scale"]), _ptr(r["k_i8"]),
+                              _ptr(r["k_scale"]), _ptr(r["k_mean"]))
+    return r
+
+
+def qk_int32(q_i8, k_i8, B, H, Hkv, N, d, b, h, i0, ni, j0, nj) -> np.ndarray:
+    q_i8 = np.ascontiguousarray(q_i8, dtype=np.int8)
+    k_i8 = np.ascontiguousarray(k_i8, dtype=np.int8)
+    out = np.zeros((ni, nj), dtype=np.int32)
+    lib().oracle_qk_int32(_ptr(q_i8), _ptr(k_i8), B, H, Hkv, N, d, b, h, i0, ni, j0, nj, _ptr(out))
+    return out
+
+
+def all_rows(B, H, N):
+    bh = np.repeat(np.arange(B * H, dtype=np.int64), N)
+    i = np.tile(np.arange(N, dtype=np.int64), B * H)
+    return bh, i
+
+
+def attention_quantized(q_i8, q_scale, k_i8, k_scale, v, B, H, Hkv, N, d, causal,
+                        rows=None, nthreads=0):
+    """Rows of the quantized attention output (float64 [nrows, d]).  rows = (row_bh, row_i) or
+    None for all rows in (b, h, i) order."""
+    row_bh, row_i = all_rows(B, H, N) if rows is None else rows
+    row_bh = np.ascontiguousarray(row_bh, dtype=np.int64)
+    row_i = np.ascontiguousarray(row_i, dtype=np.int64)
+    out = np.zeros((row_bh.size, d), dtype=np.float64)
+    v = _bits16(v)
+    q_i8 = np.ascontiguousarray(q_i8, dtype=np.int8)
+    k_i8 = np.ascontiguousarray(k_i8, dtype=np.int8)
+    q_scale = np.ascontiguousarray(q_scale, dtype=np.float32)
+    k_scale = np.ascontiguousarray(k_scale, dtype=np.float32)
+    lib().oracle_attention_quantized(_ptr(q_i8), _ptr(q_scale), _ptr(k_i8), _ptr(k_scale), _ptr(v),
+                                     B, H, Hkv, N, d, 1 if causal else 0, _ptr(row_bh),
+                                     _ptr(row_i), row_bh.size, _ptr(out), int(nthreads))
+    return out
+
+
+def attention_fp64(q, k, v, B, H, Hkv, N, d, causal, smooth=False, rows=None, nthreads=0):
+    """Rows of the full-precision attention softmax(Q K'^T/sqrt(d)) V (float64 [nrows, d])."""
+    row_bh, row_i = all_rows(B, H, N) if rows is None else rows
+    row_bh = np.ascontiguousarray(row_bh, dtype=np.int64)
+    row_i = np.ascontiguousarray(row_i, dtype=np.int64)
+    out = np.zeros((row_bh.size, d), dtype=np.float64)
+    lib().oracle_attention_fp64(_ptr(_bits16(q)), _ptr(_bits16(k)), _ptr(_bits16(v)), B, H, Hkv,
+                                N, d, 1 if causal else 0, 1 if smooth else 0, _ptr(row_bh),
+                                _ptr(row_i), row_bh.size, _ptr(out), int(nthreads))
+    return out
+
+
+def forward(q, k, v, B, H, Hkv, N, d, causal, rows=None, nthreads=0, smooth=True):
+    """The whole path: smoothing + quantization, then quantized attention rows (float64)."""
+    sq = smooth_quant(q, k, B, H, Hkv, N, d, smooth=smooth)
+    out = attention_quantized(sq["q_i8"], sq["q_scale"], sq["k_i8"], sq["k_scale"], v,
+                              B, H, Hkv, N, d, causal, rows=rows, nthreads=nthreads)
+    return out, sq

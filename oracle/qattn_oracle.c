@@ -1,0 +1,342 @@
+/*
+ * qattn_oracle.c -- plain, slow, obviously-correct CPU oracle for the smoothed-K INT8 attention
+ * forward (prefill) described on the SageAttention summary page
+ * ("SAGEATTENTION: accurate 8-bit attention for plug-and-play inference acceleration",
+ * aibr.jp/archives/102657).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the package's smoke check and the CPU-baseline leg
+ * of the benchmark may load this library.  The product path (the CUDA library) never calls it and
+ * shares no code, header, table or helper with it.
+ *
+ * What the page fixes, and where (section names of that page):
+ *   - K is smoothed before quantization so that extreme values do not inflate the INT8 scale
+ *     (dialogue answer on accuracy; sec. 2 "differences from prior work"; sec. 3 "core technical
+ *     elements").
+ *   - Q and K are quantized to INT8 and Q K^T runs as an integer product with 32-bit accumulation
+ *     (sec. 3: the Tensor Core instruction mma(u8.u8.s32)).
+ *   - P V runs in FP16 (sec. 2 and 3: FP16 accumulation, mma(f16.f16.f16)).
+ *   - The kernel follows FlashAttention's blockwise softmax (sec. 4); blockwise evaluation is exact
+ *     up to rounding, so the oracle evaluates the plain row softmax.
+ * The page gives no formula, block size, scale rule or rounding mode.  The readings used here:
+ *   - smoothing: K'[n,c] = K[n,c] - mean_n K[n,c], the mean over all N tokens of the sequence, per
+ *     (batch, kv head, channel); the sum is exact in int64 fixed point (every fp16 value is an
+ *     integer multiple of 2^-24), mean = (float)((double)sum / (N * 2^24)), K' = (float)K - mean
+ *     in binary32;
+ *   - quantization: blocks of 128 consecutive Q rows and 64 consecutive K rows (all d channels)
+ *     per (batch, head); scale = amax / 127 (binary32 division), code = clamp(rint(x / scale),
+ *     -127, 127) with binary32 division and round-half-even; amax == 0 gives scale 0, codes 0;
+ *   - dequantization: S = S_int * sQ * sK / sqrt(d) in binary64;
+ *   - causal: key j is visible to query i iff j <= i (square prefill);
+ *   - GQA: query head h reads kv head h / (H / Hkv).
+ * Everything after the int32 product is binary64.  Compile with -O2 -ffp-contract=off and without
+ * -ffast-math, so that every binary32 operation above rounds exactly once to nearest-even.
+ *
+ * Layouts (all row-major, contiguous):
+ *   q, out: [B, H, N, d]; k, v: [B, Hkv, N, d]; fp16 arrays are passed as raw uint16 bit patterns.
+ *   q_scale: [B, H, ceil(N/128)]; k_scale: [B, Hkv, ceil(N/64)]; k_mean: [B, Hkv, d].
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+#define ORACLE_QBLOCK 128
+#define ORACLE_KBLOCK 64
+
+/* ------------------------------------------------------------------------------------------------
+ * IEEE 754 binary16, written from the format's definition: 1 sign bit, 5 exponent bits (bias 15),
+ * 10 fraction bits; exponent 0 encodes subnormals m * 2^-24, exponent 31 encodes inf/NaN.
+ * ---------------------------------------------------------------------------------------------- */
+double oracle_f16_to_f64(uint16_t h) {
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 31;
+    int m = h & 1023;
+    double v;
+    if (e == 0) {
+        v = ldexp((double)m, -24);
+    } else if (e == 31) {
+        v = (m == 0) ? INFINITY : NAN;
+    } else {
+        v = ldexp((double)(1024 + m), e - 25);
+    }
+    return sign ? -v : v;
+}
+
+/* Round a binary64 value to the nearest binary16 (ties to even); overflow gives +-inf. */
+uint16_t oracle_f64_to_f16(double x) {
+    uint16_t sign = 0;
+    if (isnan(x)) return 0x7E00;
+    if (signbit(x)) { sign = 0x8000; x = -x; }
+    if (x == 0.0) return sign;
+    if (x < ldexp(1.0, -14)) {                  /* subnormal range: units of 2^-24 */
+        double q = rint(ldexp(x, 24));          /* exact scaling, then round-half-even */
+        return (uint16_t)(sign | (uint16_t)q);  /* q == 1024 is the smallest normal, still right */
+    }
+    int e;
+    (void)frexp(x, &e);                         /* x = f * 2^e, f in [0.5, 1) */
+    e -= 1;                                     /* x in [2^e, 2^(e+1)) */
+    double q = rint(ldexp(x, 10 - e));          /* 11-bit significand in [1024, 2048] */
+    if (q == 2048.0) { q = 1024.0; e += 1; }
+    if (e + 15 >= 31) return (uint16_t)(sign | 0x7C00);
+    return (uint16_t)(sign | (uint16_t)((e + 15) << 10) | (uint16_t)((int)q - 1024));
+}
+
+/* ------------------------------------------------------------------------------------------------
+ * Smoothing of K (page sec. 3, first technical element).
+ * ---------------------------------------------------------------------------------------------- */
+
+/* K * 2^24 as an exact integer: every binary16 value is an integer multiple of 2^-24 and
+ * |K| <= 65504 < 2^16, so |K * 2^24| < 2^40. */
+static int64_t k_fixed(uint16_t h) {
+    return (int64_t)(oracle_f16_to_f64(h) * 16777216.0);
+}
+
+/* sums[(b*Hkv+g)*d + c] = sum over n of K[b,g,n,c] * 2^24, exact (|sum| < 2^57 for N <= 2^17). */
+void oracle_k_channel_sums(const uint16_t* k, int B, int Hkv, int N, int d, int64_t* sums) {
+    for (long bg = 0; bg < (long)B * Hkv; ++bg) {
+        for (int c = 0; c < d; ++c) sums[bg * d + c] = 0;
+        for (int n = 0; n < N; ++n) {
+            const uint16_t* row = k + (bg * N + n) * (long)d;
+            for (int c = 0; c < d; ++c) sums[bg * d + c] += k_fixed(row[c]);
+        }
+    }
+}
+
+/* mean = (float)((double)sum / (N * 2^24)): one rounding to binary64, one division, one
+ * rounding to binary32. */
+float oracle_mean_from_sum(int64_t sum, int N) {
+    double den = (double)N * 16777216.0;
+    return (float)((double)sum / den);
+}
+
+/* ------------------------------------------------------------------------------------------------
+ * Per-block symmetric INT8 quantization (page sec. 3: INT8 operands; block sizes, scale rule and
+ * rounding per the reading in the file header).
+ * x holds `rows` rows of `d` binary32 values; writes codes and returns the block scale.
+ * ---------------------------------------------------------------------------------------------- */
+float oracle_quantize_block(const float* x, int rows, int d, int8_t* codes) {
+    float amax = 0.0f;
+    for (long i = 0; i < (long)rows * d; ++i) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    if (amax == 0.0f) {
+        memset(codes, 0, (size_t)rows * d);
+        return 0.0f;
+    }
+    float s = amax / 127.0f;
+    for (long i = 0; i < (long)rows * d; ++i) {
+        float t = x[i] / s;
+        float r = rintf(t);          /* default rounding mode: nearest, ties to even */
+        if (r > 127.0f) r = 127.0f;
+        if (r < -127.0f) r = -127.0f;
+        codes[i] = (int8_t)r;
+    }
+    return s;
+}
+
+/* The whole pre-processing: smoothing of K, then per-block quantization of Q and K'.
+ * smooth = 0 skips the smoothing (mean taken as 0); used only for the negative control.
+ * k_mean may be NULL. */
+void oracle_smooth_quant(const uint16_t* q, const uint16_t* k, int B, int H, int Hkv, int N, int d,
+                         int smooth, int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
+                         float* k_mean) {
+    int nqb = (N + ORACLE_QBLOCK - 1) / ORACLE_QBLOCK;
+    int nkb = (N + ORACLE_KBLOCK - 1) / ORACLE_KBLOCK;
+    int64_t* sums = (int64_t*)calloc((size_t)B * Hkv * d, sizeof(int64_t));
+    float* mean = (float*)calloc((size_t)B * Hkv * d, sizeof(float));
+    float* buf = (float*)malloc(sizeof(float) * (size_t)ORACLE_QBLOCK * d);
+    if (smooth) {
+        oracle_k_channel_sums(k, B, Hkv, N, d, sums);
+        for (long i = 0; i < (long)B * Hkv * d; ++i) mean[i] = oracle_mean_from_sum(sums[i], N);
+    }
+    if (k_mean) memcpy(k_mean, mean, sizeof(float) * (size_t)B * Hkv * d);
+    for (long bg = 0; bg < (long)B * Hkv; ++bg) {
+        for (int blk = 0; blk < nkb; ++blk) {
+            int r0 = blk * ORACLE_KBLOCK;
+            int rows = N - r0 < ORACLE_KBLOCK ? N - r0 : ORACLE_KBLOCK;
+            for (int r = 0; r < rows; ++r)
+                for (int c = 0; c < d; ++c) {
+                    float kv = (float)oracle_f16_to_f64(k[(bg * N + r0 + r) * (long)d + c]);
+                    buf[(long)r * d + c] = kv - mean[bg * d + c];
+                }
+            k_scale[bg * nkb + blk] =
+                oracle_quantize_block(buf, rows, d, k_i8 + (bg * N + r0) * (long)d);
+        }
+    }
+    for (long bh = 0; bh < (long)B * H; ++bh) {
+        for (int blk = 0; blk < nqb; ++blk) {
+            int r0 = blk * ORACLE_QBLOCK;
+            int rows = N - r0 < ORACLE_QBLOCK ? N - r0 : ORACLE_QBLOCK;
+            for (int r = 0; r < rows; ++r)
+                for (int c = 0; c < d; ++c)
+                    buf[(long)r * d + c] = (float)oracle_f16_to_f64(q[(bh * N + r0 + r) * (long)d + c]);
+            q_scale[bh * nqb + blk] =
+                oracle_quantize_block(buf, rows, d, q_i8 + (bh * N + r0) * (long)d);
+        }
+    }
+    free(buf);
+    free(mean);
+    free(sums);
+}
+
+/* ------------------------------------------------------------------------------------------------
+ * INT8 Q K^T with exact 32-bit accumulation (page sec. 3, mma(u8.u8.s32); signed codes per the
+ * symmetric quantization).  out[i][j] = sum_c q[b,h,i0+i,c] * k[b,g(h),j0+j,c], no masking.
+ * ---------------------------------------------------------------------------------------------- */
+void oracle_qk_int32(const int8_t* q_i8, const int8_t* k_i8, int B, int H, int Hkv, int N, int d,
+                     int b, int h, int i0, int ni, int j0, int nj, int32_t* out) {
+    (void)B;
+    int g = h / (H / Hkv);
+    const int8_t* qb = q_i8 + ((long)b * H + h) * (long)N * d;
+    const int8_t* kb = k_i8 + ((long)b * Hkv + g) * (long)N * d;
+    for (int i = 0; i < ni; ++i)
+        for (int j = 0; j < nj; ++j) {
+            int32_t acc = 0;
+            for (int c = 0; c < d; ++c)
+                acc += (int32_t)qb[(long)(i0 + i) * d + c] * (int32_t)kb[(long)(j0 + j) * d + c];
+            out[(long)i * nj + j] = acc;
+        }
+}
+
+/* ------------------------------------------------------------------------------------------------
+ * Attention rows, binary64 (page sec. 4: FlashAttention-style blockwise softmax, evaluated here
+ * as the plain two-pass row softmax it is exactly equal to).
+ * ---------------------------------------------------------------------------------------------- */
+
+typedef struct {
+    /* quantized mode */
+    const int8_t* q_i8; const float* q_scale; const int8_t* k_i8; const float* k_scale;
+    /* full-precision mode */
+    const uint16_t* q16; const uint16_t* k16; int smooth;
+    const uint16_t* v16;
+    int B, H, Hkv, N, d, causal, quantized;
+    const int64_t* row_bh; const int64_t* row_i; long nrows;
+    double* out;
+    double* kmean64;   /* full-precision mode: exact per-channel means, [B*Hkv, d] */
+    long next;         /* work counter */
+    pthread_mutex_t lock;
+} attn_job;
+
+static void attn_one_row(attn_job* J, long r, double* s, double* acc) {
+    int H = J->H, Hkv = J->Hkv, N = J->N, d = J->d;
+    long bh = J->row_bh[r];
+    int i = (int)J->row_i[r];
+    int b = (int)(bh / H), h = (int)(bh % H);
+    int g = h / (H / Hkv);
+    long bg = (long)b * Hkv + g;
+    int nvis = J->causal ? i + 1 : N;
+    double inv_sqrt_d = 1.0 / sqrt((double)d);
+    double m = -INFINITY;
+    if (J->quantized) {
+        int nkb = (N + ORACLE_KBLOCK - 1) / ORACLE_KBLOCK;
+        int nqb = (N + ORACLE_QBLOCK - 1) / ORACLE_QBLOCK;
+        const int8_t* qrow = J->q_i8 + (bh * N + i) * (long)d;
+        double sq = (double)J->q_scale[bh * nqb + i / ORACLE_QBLOCK];
+        for (int j = 0; j < nvis; ++j) {
+            const int8_t* krow = J->k_i8 + (bg * N + j) * (long)d;
+            int32_t acc32 = 0;
+            for (int c = 0; c < d; ++c) acc32 += (int32_t)qrow[c] * (int32_t)krow[c];
+            double sk = (double)J->k_scale[bg * nkb + j / ORACLE_KBLOCK];
+            s[j] = (double)acc32 * sq * sk * inv_sqrt_d;
+            if (s[j] > m) m = s[j];
+        }
+    } else {
+        const uint16_t* qrow = J->q16 + (bh * N + i) * (long)d;
+        for (int j = 0; j < nvis; ++j) {
+            const uint16_t* krow = J->k16 + (bg * N + j) * (long)d;
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c) {
+                double kc = oracle_f16_to_f64(krow[c]);
+                if (J->smooth) kc -= J->kmean64[bg * d + c];
+                dot += oracle_f16_to_f64(qrow[c]) * kc;
+            }
+            s[j] = dot * inv_sqrt_d;
+            if (s[j] > m) m = s[j];
+        }
+    }
+    double l = 0.0;
+    for (int j = 0; j < nvis; ++j) { s[j] = exp(s[j] - m); l += s[j]; }
+    for (int c = 0; c < d; ++c) acc[c] = 0.0;
+    for (int j = 0; j < nvis; ++j) {
+        const uint16_t* vrow = J->v16 + (bg * N + j) * (long)d;
+        for (int c = 0; c < d; ++c) acc[c] += s[j] * oracle_f16_to_f64(vrow[c]);
+    }
+    for (int c = 0; c < d; ++c) J->out[r * d + c] = acc[c] / l;
+}
+
+static void* attn_worker(void* arg) {
+    attn_job* J = (attn_job*)arg;
+    double* s = (double*)malloc(sizeof(double) * (size_t)J->N);
+    double* acc = (double*)malloc(sizeof(double) * (size_t)J->d);
+    for (;;) {
+        long r0;
+        pthread_mutex_lock(&J->lock);
+        r0 = J->next;
+        J->next += 16;
+        pthread_mutex_unlock(&J->lock);
+        if (r0 >= J->nrows) break;
+        long r1 = r0 + 16 < J->nrows ? r0 + 16 : J->nrows;
+        for (long r = r0; r < r1; ++r) attn_one_row(J, r, s, acc);
+    }
+    free(acc);
+    free(s);
+    return NULL;
+}
+
+static void run_rows(attn_job* J, int nthreads) {
+    if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    pthread_t th[256];
+    J->next = 0;
+    pthread_mutex_init(&J->lock, NULL);
+    for (int t = 0; t < nthreads; ++t) pthread_create(&th[t], NULL, attn_worker, J);
+    for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
+    pthread_mutex_destroy(&J->lock);
+}
+
+/* Output rows of the quantized attention: out[r, :] for the query row (bh = row_bh[r],
+ * i = row_i[r]), computed from the INT8 codes and block scales, binary64 after the int32 product.
+ * Returns the number of threads used. */
+int oracle_attention_quantized(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                               const float* k_scale, const uint16_t* v, int B, int H, int Hkv,
+                               int N, int d, int causal, const int64_t* row_bh,
+                               const int64_t* row_i, long nrows, double* out, int nthreads) {
+    attn_job J;
+    memset(&J, 0, sizeof(J));
+    J.q_i8 = q_i8; J.q_scale = q_scale; J.k_i8 = k_i8; J.k_scale = k_scale; J.v16 = v;
+    J.B = B; J.H = H; J.Hkv = Hkv; J.N = N; J.d = d; J.causal = causal; J.quantized = 1;
+    J.row_bh = row_bh; J.row_i = row_i; J.nrows = nrows; J.out = out;
+    if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    run_rows(&J, nthreads);
+    return nthreads;
+}
+
+/* Full-precision attention rows, softmax(Q K'^T / sqrt(d)) V in binary64 from the fp16 inputs,
+ * with K' = K - (exact binary64 per-channel mean) when smooth != 0, else K' = K.  This is the
+ * unquantized reference the quantized result is measured against. */
+int oracle_attention_fp64(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H,
+                          int Hkv, int N, int d, int causal, int smooth, const int64_t* row_bh,
+                          const int64_t* row_i, long nrows, double* out, int nthreads) {
+    attn_job J;
+    memset(&J, 0, sizeof(J));
+    J.q16 = q; J.k16 = k; J.v16 = v; J.smooth = smooth;
+    J.B = B; J.H = H; J.Hkv = Hkv; J.N = N; J.d = d; J.causal = causal; J.quantized = 0;
+    J.row_bh = row_bh; J.row_i = row_i; J.nrows = nrows; J.out = out;
+    J.kmean64 = (double*)calloc((size_t)B * Hkv * d, sizeof(double));
+    if (smooth) {
+        for (long bg = 0; bg < (long)B * Hkv; ++bg)
+            for (int c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (int n = 0; n < N; ++n) acc += oracle_f16_to_f64(k[(bg * N + n) * (long)d + c]);
+                J.kmean64[bg * d + c] = acc / (double)N;
+            }
+    }
+    if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    run_rows(&J, nthreads);
+    free(J.kmean64);
+    return nthreads;
+}

@@ -1,0 +1,377 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix (no GPU).
+
+Each test checks the oracle against something other than itself: a library routine (numpy's
+binary16 conversion, numpy integer matmul, torch's float64 scaled-dot-product attention), a
+brute-force loop, an exact rational result within its rounding bound, a closed form, an
+invariant, or the hand-derived worked example in tests/golden/.  The method is the one on the
+SageAttention summary page (aibr.jp/archives/102657): K smoothing and INT8 Q/K (sec. 3), int32
+Q K^T (sec. 3, mma(u8.u8.s32)), FlashAttention-style softmax (sec. 4).
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from bit_quantized_attention_smoothing_b200.workloads import WORKLOADS, make_inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _np16(t):
+    return t.contiguous().numpy().view(np.uint16) if isinstance(t, torch.Tensor) else t
+
+
+def _cos(a, b):
+    a = np.asarray(a, dtype=np.float64).ravel()
+    b = np.asarray(b, dtype=np.float64).ravel()
+    return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b)))
+
+
+# --------------------------------------------------------------------------------------------
+# binary16 conversions against numpy (an independent implementation of IEEE 754)
+# --------------------------------------------------------------------------------------------
+
+def test_f16_decode_all_patterns(oracle):
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([oracle.f16_to_f64(int(b)) for b in bits])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def test_f16_encode_matches_numpy(oracle):
+    rng = np.random.default_rng(0)
+    x = np.concatenate([
+        rng.standard_normal(4000) * 10.0 ** rng.integers(-8, 5, 4000),
+        # exact ties: midpoints between neighbouring binary16 values
+        (np.arange(1, 200, dtype=np.float64) + 0.5) * 2.0 ** -24,
+        1.0 + (np.arange(0, 64) + 0.5) * 2.0 ** -10,
+        np.array([65504.0, 65519.99, 65520.0, 70000.0, -65520.0, 2.0 ** -25, 3 * 2.0 ** -26]),
+    ])
+    got = oracle.f64_to_f16_array(x)
+    with np.errstate(over="ignore"):
+        ref = x.astype(np.float16).view(np.uint16)
+    assert np.array_equal(got, ref)
+
+
+# --------------------------------------------------------------------------------------------
+# quantization of one block (page sec. 3; scale = amax/127, rint half-even)
+# --------------------------------------------------------------------------------------------
+
+def test_quantize_identity_on_integers(oracle):
+    rng = np.random.default_rng(1)
+    x = rng.integers(-127, 128, size=(64, 32)).astype(np.float32)
+    x[3, 5] = 127.0
+    codes, s = oracle.quantize_block(x)
+    assert s == np.float32(1.0)
+    assert np.array_equal(codes.astype(np.float32), x)
+
+
+def test_quantize_ties_to_even(oracle):
+    x = np.zeros((1, 8), dtype=np.float32)
+    x[0] = [127.0, 2.5, 3.5, -2.5, 0.5, 1.5, -126.5, -0.5]
+    codes, s = oracle.quantize_block(x)
+    assert s == 1.0
+    assert codes[0].tolist() == [127, 2, 4, -2, 0, 2, -126, 0]
+
+
+def test_quantize_zero_block(oracle):
+    codes, s = oracle.quantize_block(np.zeros((64, 16), dtype=np.float32))
+    assert s == 0.0 and not codes.any()
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_quantize_invariants(oracle, seed):
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal((128, 64)) * 3.0 ** (seed - 2)).astype(np.float32)
+    codes, s = oracle.quantize_block(x)
+    amax = Fraction(float(np.abs(x).max()))
+    # the scale is amax/127 to within half an ulp of binary32
+    ulp = Fraction(float(np.spacing(np.float32(s))))
+    assert abs(Fraction(float(s)) - amax / 127) <= ulp / 2
+    assert np.abs(codes.astype(int)).max() == 127
+    am = np.unravel_index(np.abs(x).argmax(), x.shape)
+    assert abs(int(codes[am])) == 127
+    # |x - code*s| <= s/2 (plus the scale's own rounding), elementwise
+    err = np.abs(x.astype(np.float64) - codes.astype(np.float64) * float(s))
+    assert err.max() <= float(s) * 0.5 * (1 + 1e-5)
+    # scaling the block by a power of two scales s and leaves the codes unchanged
+    codes2, s2 = oracle.quantize_block(x * np.float32(2.0 ** 7))
+    assert np.array_equal(codes, codes2) and s2 == s * np.float32(128.0)
+
+
+# --------------------------------------------------------------------------------------------
+# smoothing: exact channel sums and the mean (page sec. 3, K smoothing)
+# --------------------------------------------------------------------------------------------
+
+def test_k_channel_sums_exact(oracle):
+    rng = np.random.default_rng(2)
+    B, G, N, d = 2, 3, 300, 16
+    k = (rng.standard_normal((B, G, N, d)) * 10.0 ** rng.integers(-7, 4, (B, G, N, d)))
+    k = np.clip(k, -60000, 60000).astype(np.float16)
+    sums = oracle.k_channel_sums(k, B, G, N, d)
+    ref = (k.astype(np.float64) * 2.0 ** 24).astype(np.int64).sum(axis=2)
+    assert np.array_equal(sums, ref)
+
+
+def test_mean_within_half_ulp(oracle):
+    rng = np.random.default_rng(3)
+    for _ in range(300):
+        N = int(rng.integers(1, 1 << 17))
+        s = int(rng.integers(-(1 << 56), 1 << 56)) >> int(rng.integers(0, 50))
+        m = oracle.mean_from_sum(s, N)
+        exact = Fraction(s, N * (1 << 24))
+        ulp = Fraction(float(np.spacing(np.abs(m)))) if m != 0 else Fraction(1, 1 << 149)
+        assert abs(Fraction(float(m)) - exact) <= ulp / 2 * (1 + Fraction(1, 1 << 20))
+
+
+def test_constant_k_gives_zero_blocks(oracle):
+    N, d = 200, 64
+    rng = np.random.default_rng(4)
+    row = rng.standard_normal(d).astype(np.float16)
+    k = np.tile(row, (1, 1, N, 1))
+    q = rng.standard_normal((1, 1, N, d)).astype(np.float16)
+    r = oracle.smooth_quant(q, k, 1, 1, 1, N, d)
+    assert np.array_equal(r["k_mean"][0, 0], row.astype(np.float32))
+    assert not r["k_i8"].any() and not r["k_scale"].any()
+
+
+def test_smoothing_removes_channel_offset(oracle):
+    w = WORKLOADS["tiny"]
+    q, k, v = make_inputs(w)
+    r = oracle.smooth_quant(_np16(q), _np16(k), w.B, w.H, w.Hkv, w.N, w.d)
+    deq = r["k_i8"][0, 0].astype(np.float64) * np.repeat(r["k_scale"][0, 0], 64)[:, None]
+    # the dequantized smoothed K has (near) zero channel means; the raw K has the N(0,4) offset
+    raw_mean = k[0, 0].double().mean(0).numpy()
+    assert np.abs(raw_mean).max() > 1.0
+    assert np.abs(deq.mean(0)).max() < 0.05
+    np.testing.assert_allclose(r["k_mean"][0, 0], raw_mean, atol=1e-6)
+
+
+def test_ragged_block_boundaries(oracle):
+    B, H, Hkv, N, d = 1, 2, 1, 200, 32
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((B, H, N, d)).astype(np.float16)
+    k = rng.standard_normal((B, Hkv, N, d)).astype(np.float16)
+    r = oracle.smooth_quant(q, k, B, H, Hkv, N, d)
+    assert r["q_scale"].shape == (B, H, 2) and r["k_scale"].shape == (B, Hkv, 4)
+    for h in range(H):
+        for blk, (r0, r1) in enumerate([(0, 128), (128, 200)]):
+            x = q[0, h, r0:r1].astype(np.float32)
+            am = np.unravel_index(np.abs(x).argmax(), x.shape)
+            assert abs(int(r["q_i8"][0, h, r0:r1][am])) == 127
+            assert r["q_scale"][0, h, blk] == np.float32(np.abs(x).max()) / np.float32(127)
+    kp = k[0, 0].astype(np.float32) - r["k_mean"][0, 0]
+    for blk, (r0, r1) in enumerate([(0, 64), (64, 128), (128, 192), (192, 200)]):
+        x = kp[r0:r1]
+        am = np.unravel_index(np.abs(x).argmax(), x.shape)
+        assert abs(int(r["k_i8"][0, 0, r0:r1][am])) == 127
+
+
+# --------------------------------------------------------------------------------------------
+# int32 Q K^T (page sec. 3, mma(u8.u8.s32)) against brute force and numpy
+# --------------------------------------------------------------------------------------------
+
+def test_qk_int32_bruteforce_gqa(oracle):
+    rng = np.random.default_rng(6)
+    B, H, Hkv, N, d = 2, 4, 2, 9, 8
+    qi = rng.integers(-127, 128, (B, H, N, d)).astype(np.int8)
+    ki = rng.integers(-127, 128, (B, Hkv, N, d)).astype(np.int8)
+    for b in range(B):
+        for h in range(H):
+            got = oracle.qk_int32(qi, ki, B, H, Hkv, N, d, b, h, 2, 5, 1, 7)
+            g = h // (H // Hkv)
+            for i in range(5):
+                for j in range(7):
+                    ref = sum(int(qi[b, h, 2 + i, c]) * int(ki[b, g, 1 + j, c]) for c in range(d))
+                    assert got[i, j] == ref
+            full = oracle.qk_int32(qi, ki, B, H, Hkv, N, d, b, h, 0, N, 0, N)
+            assert np.array_equal(full, qi[b, h].astype(np.int64) @ ki[b, g].astype(np.int64).T)
+
+
+def test_qk_int32_extreme_bound(oracle):
+    d = 128
+    qi = np.full((1, 1, 2, d), -127, dtype=np.int8)
+    ki = np.full((1, 1, 2, d), -127, dtype=np.int8)
+    s = oracle.qk_int32(qi, ki, 1, 1, 1, 2, d, 0, 0, 0, 2, 0, 2)
+    assert (s == 127 * 127 * d).all() and 127 * 127 * d == 2064512
+
+
+# --------------------------------------------------------------------------------------------
+# attention (page sec. 4): brute force, torch float64 SDPA, invariants
+# --------------------------------------------------------------------------------------------
+
+def _sdpa64(q, k, v, H, Hkv, causal, kshift=None):
+    G = H // Hkv
+    qd = torch.from_numpy(q.astype(np.float64))
+    kd = torch.from_numpy(k.astype(np.float64))
+    if kshift is not None:
+        kd = kd - torch.from_numpy(kshift)
+    vd = torch.from_numpy(v.astype(np.float64))
+    kd = kd.repeat_interleave(G, dim=1)
+    vd = vd.repeat_interleave(G, dim=1)
+    return torch.nn.functional.scaled_dot_product_attention(qd, kd, vd, is_causal=causal).numpy()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp64_attention_bruteforce(oracle, causal):
+    rng = np.random.default_rng(7)
+    B, H, Hkv, N, d = 1, 2, 1, 5, 3
+    q = rng.standard_normal((B, H, N, d)).astype(np.float16)
+    k = rng.standard_normal((B, Hkv, N, d)).astype(np.float16)
+    v = rng.standard_normal((B, Hkv, N, d)).astype(np.float16)
+    got = oracle.attention_fp64(q, k, v, B, H, Hkv, N, d, causal).reshape(B, H, N, d)
+    for h in range(H):
+        for i in range(N):
+            keys = range(i + 1) if causal else range(N)
+            sc = [sum(float(q[0, h, i, c]) * float(k[0, 0, j, c]) for c in range(d)) / math.sqrt(d)
+                  for j in keys]
+            mx = max(sc)
+            e = [math.exp(s - mx) for s in sc]
+            for c in range(d):
+                ref = sum(e[t] * float(v[0, 0, j, c]) for t, j in enumerate(keys)) / sum(e)
+                assert abs(got[0, h, i, c] - ref) < 1e-13
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp64_attention_vs_torch_sdpa(oracle, causal):
+    rng = np.random.default_rng(8)
+    B, H, Hkv, N, d = 2, 4, 2, 70, 16
+    q = rng.standard_normal((B, H, N, d)).astype(np.float16)
+    k = (rng.standard_normal((B, Hkv, N, d)) + 2).astype(np.float16)
+    v = rng.standard_normal((B, Hkv, N, d)).astype(np.float16)
+    got = oracle.attention_fp64(q, k, v, B, H, Hkv, N, d, causal).reshape(B, H, N, d)
+    np.testing.assert_allclose(got, _sdpa64(q, k, v, H, Hkv, causal), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_smoothing_leaves_softmax_unchanged(oracle, causal):
+    w = WORKLOADS["tiny"].with_(causal=causal)
+    q, k, v = (_np16(t) for t in make_inputs(w))
+    a = oracle.attention_fp64(q, k, v, w.B, w.H, w.Hkv, w.N, w.d, causal, smooth=False)
+    b = oracle.attention_fp64(q, k, v, w.B, w.H, w.Hkv, w.N, w.d, causal, smooth=True)
+    assert np.abs(a - b).max() <= 1e-12 * max(1.0, np.abs(a).max())
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_quantized_attention_exact_on_dyadic_inputs(oracle, causal):
+    """Inputs that quantize without error (each block's amax is 127 * 2^e, every value a multiple of
+    2^e, K channels sum to zero in each block so the smoothing mean is exactly 0), with different
+    power-of-two scales per Q block and per K block: the quantized path must then equal float64
+    softmax(Q K^T / sqrt(d)) V, which pins the block indexing and the dequantization."""
+    rng = np.random.default_rng(9)
+    B, H, Hkv, N, d = 1, 2, 1, 256, 16
+    q = np.zeros((B, H, N, d))
+    for h in range(H):
+        for blk, e in enumerate([-6, -4]):
+            x = rng.integers(-126, 127, (128, d)).astype(np.float64)
+            x[0, 0] = 127
+            q[0, h, blk * 128:(blk + 1) * 128] = x * 2.0 ** (e - h)
+    k = np.zeros((B, Hkv, N, d))
+    for blk, e in enumerate([-7, -5, -6, -8]):
+        x = rng.integers(-126, 127, (32, d)).astype(np.float64)
+        x[0, 0] = 127
+        k[0, 0, blk * 64:(blk + 1) * 64] = np.concatenate([x, -x]) * 2.0 ** e
+    v = rng.standard_normal((B, Hkv, N, d))
+    q, k, v = q.astype(np.float16), k.astype(np.float16), v.astype(np.float16)
+    out, sq = oracle.forward(q, k, v, B, H, Hkv, N, d, causal)
+    assert not sq["k_mean"].any()
+    assert sq["q_scale"][0, 0].tolist() == [2.0 ** -6, 2.0 ** -4]
+    assert sq["k_scale"][0, 0].tolist() == [2.0 ** -7, 2.0 ** -5, 2.0 ** -6, 2.0 ** -8]
+    ref = _sdpa64(q, k, v, H, Hkv, causal)
+    np.testing.assert_allclose(out.reshape(B, H, N, d), ref, rtol=0, atol=1e-12)
+
+
+def test_causal_first_row_is_v0(oracle):
+    w = WORKLOADS["tiny"].with_(causal=True, N=200)
+    q, k, v = (_np16(t) for t in make_inputs(w))
+    out, _ = oracle.forward(q, k, v, w.B, w.H, w.Hkv, w.N, w.d, True,
+                            rows=(np.array([0]), np.array([0])))
+    assert np.array_equal(out[0], v[0, 0, 0].view(np.float16).astype(np.float64))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_identical_keys_average_values(oracle, causal):
+    rng = np.random.default_rng(10)
+    B, H, Hkv, N, d = 1, 1, 1, 150, 64
+    q = rng.standard_normal((B, H, N, d)).astype(np.float16)
+    k = np.tile(rng.standard_normal(d).astype(np.float16), (B, Hkv, N, 1))
+    v = rng.standard_normal((B, Hkv, N, d)).astype(np.float16)
+    out, sq = oracle.forward(q, k, v, B, H, Hkv, N, d, causal)
+    assert not sq["k_scale"].any()          # K' = 0: every K block has zero scale
+    vv = v[0, 0].astype(np.float64)
+    ref = np.cumsum(vv, 0) / np.arange(1, N + 1)[:, None] if causal else np.tile(vv.mean(0), (N, 1))
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-13)
+
+
+def test_gqa_equals_repeated_heads(oracle):
+    rng = np.random.default_rng(11)
+    B, H, Hkv, N, d = 1, 4, 2, 192, 64
+    q = rng.standard_normal((B, H, N, d)).astype(np.float16)
+    k = (rng.standard_normal((B, Hkv, N, d)) + rng.standard_normal((1, Hkv, 1, d)) * 2).astype(np.float16)
+    v = rng.standard_normal((B, Hkv, N, d)).astype(np.float16)
+    out_g, _ = oracle.forward(q, k, v, B, H, Hkv, N, d, True)
+    kr = np.ascontiguousarray(np.repeat(k, H // Hkv, axis=1))
+    vr = np.ascontiguousarray(np.repeat(v, H // Hkv, axis=1))
+    out_r, _ = oracle.forward(q, kr, vr, B, H, H, N, d, True)
+    assert np.array_equal(out_g, out_r)
+    # and the head mapping is contiguous groups: head 1 must differ when kv heads are swapped
+    out_s, _ = oracle.forward(q, np.ascontiguousarray(k[:, ::-1]), np.ascontiguousarray(v[:, ::-1]),
+                              B, H, Hkv, N, d, True)
+    assert not np.array_equal(out_g[: N], out_s[: N])
+
+
+@pytest.mark.parametrize("name,shrink,bound", [
+    ("tiny", {}, 0.999),
+    ("prefill4k", {"N": 256, "B": 1, "H": 4, "Hkv": 4, "k_outlier_channels": 0}, 0.999),
+    ("prefill4k", {"N": 256, "B": 1, "H": 4, "Hkv": 4}, 0.995),
+])
+def test_quantized_close_to_full_precision(oracle, name, shrink, bound):
+    """Accuracy of the 8-bit path (page dialogue and sec. 4: small end-to-end loss): cosine
+    similarity against float64 full-precision attention, and smoothing must help on inputs with a
+    K channel offset (negative control).  The x20 outlier channels of the 4k prefill workload are
+    scaled noise, not an offset, so smoothing cannot remove them; they set the K block scale and
+    cost the other channels precision (measured cosine 0.9973), hence the lower bound there."""
+    w = WORKLOADS[name].with_(**shrink)
+    q, k, v = (_np16(t) for t in make_inputs(w))
+    ref = oracle.attention_fp64(q, k, v, w.B, w.H, w.Hkv, w.N, w.d, w.causal)
+    out, _ = oracle.forward(q, k, v, w.B, w.H, w.Hkv, w.N, w.d, w.causal)
+    out_ns, _ = oracle.forward(q, k, v, w.B, w.H, w.Hkv, w.N, w.d, w.causal, smooth=False)
+    c, c_ns = _cos(out, ref), _cos(out_ns, ref)
+    assert c >= bound
+    assert c_ns < c
+
+
+# --------------------------------------------------------------------------------------------
+# the hand-derived worked example
+# --------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_worked_example(oracle, causal):
+    with open(os.path.join(GOLDEN, "worked_example_n2_d4.json")) as f:
+        g = json.load(f)
+    q = np.array(g["q"], dtype=np.float16)[None, None]
+    k = np.array(g["k"], dtype=np.float16)[None, None]
+    v = np.array(g["v"], dtype=np.float16)[None, None]
+    e = g["expect"]
+    out, sq = oracle.forward(q, k, v, 1, 1, 1, 2, 4, causal)
+    assert sq["k_mean"][0, 0].tolist() == e["k_mean"]
+    assert sq["k_i8"][0, 0].tolist() == e["k_i8"]
+    assert sq["k_scale"][0, 0].tolist() == e["k_scale"]
+    assert sq["q_i8"][0, 0].tolist() == e["q_i8"]
+    assert sq["q_scale"][0, 0].tolist() == e["q_scale"]
+    s = oracle.qk_int32(sq["q_i8"], sq["k_i8"], 1, 1, 1, 2, 4, 0, 0, 0, 2, 0, 2)
+    assert s.tolist() == e["s_int"]
+    v0, v1 = np.array(g["v"][0]), np.array(g["v"][1])
+    for i, gap in enumerate(e["score_half_gap"]):
+        if causal and i == 0:
+            ref = v0
+        else:
+            w1 = 1.0 / (1.0 + math.exp(2.0 * gap))
+            ref = v0 + w1 * (v1 - v0)
+        np.testing.assert_allclose(out[i], ref, rtol=0, atol=1e-14)
