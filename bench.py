@@ -1,0 +1,407 @@
+#!/usr/bin/env python3
+"""Benchmark of the smoothed-K INT8 attention forward (prefill) on B200.
+
+One step = one pass of the whole path over one batch of synthetic input already resident in HBM:
+K channel sums, smoothing + INT8 quantization of Q and K (the pre-processing kernels), then the
+tcgen05 attention kernel, all through the C ABI (qattn_smooth_quant then qattn_attn_quantized,
+the two halves of qattn_forward_ws, timed separately with CUDA events on the launching stream).
+
+Metric: TOPS = 4*B*H*N^2*d / t, halved for causal; also reported as a fraction of the B200 INT8
+tensor peak (the measured bf16 GEMM peak x 2, the nominal INT8:BF16 ratio).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+Multi-GPU (weak scaling, one full workload per rank, no data-path collective):
+  python -m torch.distributed.run --nproc-per-node N --master-addr 127.0.0.1 ... bench.py --gpus N
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized attention fwd TOPS (4·B·H·N²·d/s) and % of B200 INT8 tensor peak"
+DEFAULT_WORKLOAD = "llama8b_32k"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+ATTN_KERNEL_SOURCES = ["attn_sm100.cuh", "sm100_ptx.cuh"]
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_sm100_llama8b_32k.md")
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="target CPU time of the oracle baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args(argv)
+
+
+# ------------------------------------------------------------------------------------------------
+# peaks, clocks, profile summary
+# ------------------------------------------------------------------------------------------------
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for name in ATTN_KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "bit_quantized_attention_smoothing_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was taken on the
+    current kernel source and this workload; else None."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_w = re.search(r"workload:\s*(\S+)", text)
+    if not (m_sha and m_b and m_w):
+        return None
+    if m_sha.group(1) != kernel_source_sha() or m_w.group(1) != workload:
+        return None
+    return float(m_b.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = max(mx, float(parts[1]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[3:]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle baseline (the oracle as it stands, on a bounded sample of the workload)
+# ------------------------------------------------------------------------------------------------
+
+def oracle_sample_run(w, q, k, v, target_s):
+    """Times the oracle's whole path on a sample of the workload: smoothing + quantization of
+    the kv head 0 and its query heads (full N), then attention for query rows spread over the
+    sequence, the count chosen so the run takes about target_s.  Returns a dict."""
+    import numpy as np
+    from oracle import oracle as O
+    O.build()
+    G = w.H // w.Hkv
+    qs = q[0:1, 0:G].contiguous().cpu().numpy().view(np.uint16)
+    ks = k[0:1, 0:1].contiguous().cpu().numpy().view(np.uint16)
+    vs = v[0:1, 0:1].contiguous().cpu().numpy().view(np.uint16)
+    threads = os.cpu_count() or 1
+
+    def rows_for(nrows):
+        i = np.linspace(0, w.N - 1, nrows).astype(np.int64)
+        bh = np.arange(nrows, dtype=np.int64) % G
+        return bh, i
+
+    def pairs(i):
+        return float(np.sum(i + 1)) if w.causal else float(len(i)) * w.N
+
+    t0 = time.perf_counter()
+    sq = O.smooth_quant(qs, ks, 1, G, 1, w.N, w.d)
+    t_quant = time.perf_counter() - t0
+    nrows = 16
+    while True:
+        bh, i = rows_for(nrows)
+        t1 = time.perf_counter()
+        O.attention_quantized(sq["q_i8"], sq["q_scale"], sq["k_i8"], sq["k_scale"], vs, 1, G, 1,
+                              w.N, w.d, w.causal, rows=(bh, i), nthreads=threads)
+        dt = time.perf_counter() - t1
+        if dt >= 0.4 * max(target_s - t_quant, 0.5) or nrows >= w.N * G:
+            break
+        grow = 0.8 * max(target_s - t_quant, 0.5) / max(dt, 1e-3)
+        nrows = int(min(w.N * G, nrows * min(64.0, max(2.0, grow))))
+    # final timed sample: quantization + attention rows
+    t0 = time.perf_counter()
+    sq = O.smooth_quant(qs, ks, 1, G, 1, w.N, w.d)
+    O.attention_quantized(sq["q_i8"], sq["q_scale"], sq["k_i8"], sq["k_scale"], vs, 1, G, 1, w.N,
+                          w.d, w.causal, rows=(bh, i), nthreads=threads)
+    dt = time.perf_counter() - t0
+    ops = 4.0 * w.d * pairs(i)
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
+            "seconds": round(dt, 3),
+            "sample": (f"kv head 0 of batch 0 with its {G} query heads: smoothing + quantization "
+                       f"over all N={w.N} tokens, then {len(i)} query rows spread evenly over the "
+                       f"sequence ({pairs(i):.3g} visible pairs, 4*d ops each)")}
+
+
+# ------------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from bit_quantized_attention_smoothing_b200 import qattn as Q
+    from bit_quantized_attention_smoothing_b200.workloads import WORKLOADS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = WORKLOADS[args.workload]
+    Q.load()
+    q, k, v = make_inputs(w, device="cuda")
+    B, H, Hkv, N, d = w.B, w.H, w.Hkv, w.N, w.d
+    nqb, nkb = -(-N // 128), -(-N // 64)
+    dev = q.device
+    q_i8 = torch.empty(B, H, N, d, dtype=torch.int8, device=dev)
+    k_i8 = torch.empty(B, Hkv, N, d, dtype=torch.int8, device=dev)
+    q_s = torch.empty(B, H, nqb, dtype=torch.float32, device=dev)
+    k_s = torch.empty(B, Hkv, nkb, dtype=torch.float32, device=dev)
+    ws = torch.empty(Q.qattn_smooth_quant_workspace(B, Hkv, d), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    working_set = sum(t.numel() * t.element_size() for t in (q, k, v, q_i8, k_i8, out))
+
+    def step(ev_mid=None):
+        Q.qattn_smooth_quant(q, k, q_i8, q_s, k_i8, k_s, None, ws, stream, want_mean=False)
+        if ev_mid is not None:
+            ev_mid.record(stream)
+        Q.qattn_attn_quantized(q_i8, q_s, k_i8, k_s, v, out, w.causal, stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if Q.qattn_check_device_status(stream) != 0:
+        raise RuntimeError("device status reports a timed-out wait during warm-up")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            ev[i][0].record(stream)
+            step(ev[i][1])
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    quant_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    if Q.qattn_check_device_status(stream) != 0:
+        raise RuntimeError("device status reports a timed-out wait in the timed region")
+
+    t_max = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    total_ms_max = float(t_max.item())
+    ops = w.ops
+    value = world * ops * K / (total_ms_max / 1e3) / 1e12
+
+    # end to end through the C ABI on host buffers (H2D of q, k, v and D2H of out inside)
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    Q.qattn_forward_host(qh, kh, vh, oh, w.causal, stream)  # warm-up (pool, tensor maps)
+    ke = max(1, args.e2e_steps)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(ke):
+        Q.qattn_forward_host(qh, kh, vh, oh, w.causal, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_value = world * ops * ke / (float(e2e_ms.item()) / 1e3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size()
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    peaks, peak_src = load_peaks()
+    bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    int8_peak = 2.0 * bf16                       # nominal INT8:BF16 dense ratio 4.5:2.25
+    mixed_peak = 2.0 / (1.0 / int8_peak + 1.0 / bf16)   # half the ops INT8, half FP16
+    attn_avg_ms = statistics.mean(attn_ms)
+    achieved = ops / (attn_avg_ms / 1e3) / 1e12
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": round(total_ms_max / K, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "s8xs8->s32 (QK^T), f16xf16->f32 (PV)",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": B, "H": H, "Hkv": Hkv, "N": N, "d": d,
+                   "causal": w.causal, "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "l2": f"inputs larger than L2: working set {working_set / 2**20:.0f} MiB "
+                         f"vs 126 MiB L2, no flush"},
+        "value_frac_of_int8_peak": round(value / int8_peak, 4),
+        "attn_ms": round(attn_avg_ms, 4),
+        "quant_ms": round(statistics.mean(quant_ms), 4),
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "attn_fwd_kernel",
+            "achieved": round(achieved, 2),
+            "peak": round(mixed_peak, 1),
+            "unit": "TFLOP/s",
+            "frac": round(achieved / mixed_peak, 4),
+            "traffic": profiled_traffic(w.name),
+            "peak_source": (f"{peak_src} bf16 GEMM burst {bf16:.1f} TF/s; INT8 = 2x; mixed "
+                            f"INT8/FP16 ceiling 2/(1/P8+1/P16) since half the ops run at each "
+                            f"rate ({'of measured' if peak_src == 'measured' else 'of fallback'})"),
+            "frac_of_int8_peak": round(achieved / int8_peak, 4),
+        },
+        "e2e": {"value": round(e2e_value, 2), "unit": "TOPS", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": ke,
+                "api": "qattn_forward_host (host fp16 buffers; copies, workspace and kernels inside)"},
+        "gpu_launches": 3 * K,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_sample_run(w, q, k, v, args.cpu_seconds)
+    return line
+
+
+# ------------------------------------------------------------------------------------------------
+# reference arm: the oracle, timed on the host cores
+# ------------------------------------------------------------------------------------------------
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    import torch
+    from bit_quantized_attention_smoothing_b200.workloads import WORKLOADS, make_inputs
+    w = WORKLOADS[args.workload]
+    # only the kv head 0 slice is needed; draw the workload on the CPU generator at reduced H
+    small = w.with_(B=1, H=w.H // w.Hkv, Hkv=1)
+    q, k, v = make_inputs(small, device="cpu")
+    per_step = max(1.0, min(args.cpu_seconds, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample_run(small, q, k, v, per_step)
+    vals, secs = [], 0.0
+    for _ in range(args.steps):
+        r = oracle_sample_run(small, q, k, v, per_step)
+        vals.append(r["value"])
+        secs += r["seconds"]
+    value = statistics.mean(vals)
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 6),
+        "unit": "TOPS",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * secs / max(1, args.steps), 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "s8xs8->s32, f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                   "causal": w.causal},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": r["cores"],
+                         "kind": "oracle", "sample": r["sample"]},
+        "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,417 @@
+// qattn.cu -- the C ABI declared in include/qattn.h: argument checks, TMA tensor maps, workspace
+// management and kernel launches for the smoothed-K INT8 attention forward on B200 (sm_100a).
+// One translation unit: the kernels live in the included .cuh files.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+
+#include "qattn.h"
+#include "attn_sm100.cuh"
+#include "quant.cuh"
+
+namespace {
+
+using namespace qattn;
+
+constexpr int kMaxN = 1 << 20;
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+qattn_status check_shape(int B, int H, int Hkv, int N, int d) {
+  if (B < 1 || H < 1 || Hkv < 1 || N < 1) return QATTN_ERR_INVALID_ARG;
+  if (H % Hkv != 0) return QATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return QATTN_ERR_UNSUPPORTED;
+  if (N > kMaxN) return QATTN_ERR_UNSUPPORTED;
+  // grid-size and 32-bit index limits of the kernels
+  if (static_cast<long long>(B) * H > (1 << 20)) return QATTN_ERR_UNSUPPORTED;
+  return QATTN_OK;
+}
+
+template <typename... P>
+qattn_status check_ptrs(P... ptrs) {
+  const void* arr[] = {static_cast<const void*>(ptrs)...};
+  for (const void* p : arr)
+    if (p == nullptr) return QATTN_ERR_INVALID_ARG;
+  for (const void* p : arr)
+    if (!aligned16(p)) return QATTN_ERR_MISALIGNED;
+  return QATTN_OK;
+}
+
+qattn_status device_ok() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QATTN_ERR_CUDA;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return QATTN_ERR_CUDA;
+  if (major != 10) return QATTN_ERR_UNSUPPORTED;
+  return QATTN_OK;
+}
+
+qattn_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? QATTN_OK : QATTN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Tensor maps (driver entry point fetched through the runtime, so no link against libcuda)
+// ---------------------------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D map over a contiguous [dim2][dim1][dim0] tensor with a (box0 x box1 x 1) box.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
+              uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box0, uint32_t box1,
+              CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {dim0, dim1, dim2};
+  cuuint64_t strides[2] = {dim0 * elem_bytes, dim0 * dim1 * elem_bytes};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// int8 [rows_outer][N][d] tiles of 128 rows x d bytes, swizzled to match the MMA descriptors.
+bool make_i8_map(CUtensorMap* m, const void* base, int d, int N, long long outer) {
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, outer, d, 128,
+                  d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+// fp16 V [outer][N][d]: boxes of 64 columns (128 bytes) x 128 rows, 128-byte swizzle.
+bool make_v_map(CUtensorMap* m, const void* base, int d, int N, long long outer) {
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, N, outer, 64, 128,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Launchers
+// ---------------------------------------------------------------------------------------------
+
+struct QuantLayout {
+  int nqb, nkb;
+  size_t q_i8, k_i8, q_scale, k_scale, sums, total;
+};
+
+QuantLayout forward_layout(int B, int H, int Hkv, int N, int d) {
+  QuantLayout L;
+  L.nqb = (N + kQBlock - 1) / kQBlock;
+  L.nkb = (N + kKBlock - 1) / kKBlock;
+  size_t off = 0;
+  L.q_i8 = off;
+  off = align_up(off + static_cast<size_t>(B) * H * N * d);
+  L.k_i8 = off;
+  off = align_up(off + static_cast<size_t>(B) * Hkv * N * d);
+  L.q_scale = off;
+  off = align_up(off + sizeof(float) * B * H * L.nqb);
+  L.k_scale = off;
+  off = align_up(off + sizeof(float) * B * Hkv * L.nkb);
+  L.sums = off;
+  off = align_up(off + sizeof(long long) * B * Hkv * d);
+  L.total = off;
+  return L;
+}
+
+template <int D>
+qattn_status run_smooth_quant(const void* q, const void* k, int B, int H, int Hkv, int N,
+                              int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
+                              float* k_mean, long long* sums, cudaStream_t st) {
+  const int nqb = (N + kQBlock - 1) / kQBlock;
+  const int nkb = (N + kKBlock - 1) / kKBlock;
+  if (cudaMemsetAsync(sums, 0, sizeof(long long) * B * Hkv * D, st) != cudaSuccess)
+    return QATTN_ERR_CUDA;
+  dim3 g1(B * Hkv, (N + kSumRowsPerCta - 1) / kSumRowsPerCta);
+  k_channel_sums_kernel<D><<<g1, 256, 0, st>>>(static_cast<const uint16_t*>(k), N, sums);
+  if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
+  const long long nq = static_cast<long long>(B) * H * nqb;
+  const long long nk = static_cast<long long>(B) * Hkv * nkb;
+  if (nq + nk > 0x7FFFFFFFLL) return QATTN_ERR_UNSUPPORTED;
+  quantize_kernel<D><<<static_cast<unsigned>(nq + nk), 256, 0, st>>>(
+      static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), N, nqb, nkb, nq, sums,
+      q_i8, q_scale, k_i8, k_scale, k_mean);
+  return launch_status();
+}
+
+template <int D, bool CAUSAL>
+qattn_status run_attn(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                      const float* k_scale, const void* v, void* out, int B, int H, int Hkv,
+                      int N, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  if (!make_i8_map(&tq, q_i8, D, N, static_cast<long long>(B) * H) ||
+      !make_i8_map(&tk, k_i8, D, N, static_cast<long long>(B) * Hkv) ||
+      !make_v_map(&tv, v, D, N, static_cast<long long>(B) * Hkv))
+    return QATTN_ERR_CUDA;
+  using Cfg = AttnCfg<D>;
+  auto kern = attn_fwd_kernel<D, CAUSAL>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
+      cudaSuccess)
+    return QATTN_ERR_CUDA;
+  const int nqt = (N + kBM - 1) / kBM;
+  const long long grid = static_cast<long long>(B) * H * ((nqt + 1) / 2);
+  if (grid > 0x7FFFFFFFLL) return QATTN_ERR_UNSUPPORTED;
+  const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  kern<<<static_cast<unsigned>(grid), kAttnThreads, Cfg::kSmemBytes, st>>>(
+      tq, tk, tv, q_scale, k_scale, static_cast<__half*>(out), B, H, Hkv, N, scale_log2);
+  return launch_status();
+}
+
+qattn_status dispatch_attn(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                           const float* k_scale, const void* v, void* out, int B, int H, int Hkv,
+                           int N, int d, int causal, cudaStream_t st) {
+  if (d == 128)
+    return causal ? run_attn<128, true>(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st)
+                  : run_attn<128, false>(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st);
+  return causal ? run_attn<64, true>(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st)
+                : run_attn<64, false>(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st);
+}
+
+qattn_status dispatch_smooth_quant(const void* q, const void* k, int B, int H, int Hkv, int N,
+                                   int d, int8_t* q_i8, float* q_scale, int8_t* k_i8,
+                                   float* k_scale, float* k_mean, long long* sums,
+                                   cudaStream_t st) {
+  if (d == 128)
+    return run_smooth_quant<128>(q, k, B, H, Hkv, N, q_i8, q_scale, k_i8, k_scale, k_mean, sums,
+                                 st);
+  return run_smooth_quant<64>(q, k, B, H, Hkv, N, q_i8, q_scale, k_i8, k_scale, k_mean, sums, st);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Per-device memory pools for the allocating entry points
+// ---------------------------------------------------------------------------------------------
+
+std::mutex g_pool_mu;
+std::map<int, cudaMemPool_t> g_pools;
+
+qattn_status get_pool(cudaMemPool_t* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_pool_mu);
+  auto it = g_pools.find(dev);
+  if (it != g_pools.end()) {
+    *out = it->second;
+    return QATTN_OK;
+  }
+  cudaMemPoolProps props;
+  std::memset(&props, 0, sizeof(props));
+  props.allocType = cudaMemAllocationTypePinned;
+  props.handleTypes = cudaMemHandleTypeNone;
+  props.location.type = cudaMemLocationTypeDevice;
+  props.location.id = dev;
+  cudaMemPool_t pool;
+  if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return QATTN_ERR_CUDA;
+  uint64_t keep = UINT64_MAX;  // keep freed blocks cached for reuse
+  cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+  g_pools[dev] = pool;
+  *out = pool;
+  return QATTN_OK;
+}
+
+qattn_status pool_alloc(void** p, size_t bytes, cudaStream_t st) {
+  cudaMemPool_t pool;
+  qattn_status s = get_pool(&pool);
+  if (s != QATTN_OK) return s;
+  return cudaMallocFromPoolAsync(p, bytes, pool, st) == cudaSuccess ? QATTN_OK : QATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+// =============================================================================================
+// C ABI
+// =============================================================================================
+
+extern "C" {
+
+const char* qattn_status_string(int status) {
+  switch (status) {
+    case QATTN_OK: return "ok";
+    case QATTN_ERR_INVALID_ARG: return "invalid argument";
+    case QATTN_ERR_UNSUPPORTED: return "unsupported shape or device";
+    case QATTN_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case QATTN_ERR_CUDA: return "CUDA error";
+    case QATTN_ERR_TIMEOUT: return "bounded wait inside a kernel timed out";
+    case QATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int qattn_version(void) { return 100; }
+
+size_t qattn_smooth_quant_workspace(int B, int Hkv, int d) {
+  if (B < 1 || Hkv < 1 || d < 1) return 0;
+  return align_up(sizeof(long long) * static_cast<size_t>(B) * Hkv * d);
+}
+
+qattn_status qattn_smooth_quant(const void* q, const void* k, int B, int H, int Hkv, int N, int d,
+                                int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
+                                float* k_mean, void* ws, size_t ws_bytes, qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q, k, q_i8, q_scale, k_i8, k_scale);
+  if (s != QATTN_OK) return s;
+  if (k_mean && !aligned16(k_mean)) return QATTN_ERR_MISALIGNED;
+  if (ws == nullptr || ws_bytes < qattn_smooth_quant_workspace(B, Hkv, d))
+    return QATTN_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QATTN_ERR_MISALIGNED;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  return dispatch_smooth_quant(q, k, B, H, Hkv, N, d, q_i8, q_scale, k_i8, k_scale, k_mean,
+                               static_cast<long long*>(ws), reinterpret_cast<cudaStream_t>(stream));
+}
+
+qattn_status qattn_attn_quantized(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                                  const float* k_scale, const void* v, void* out, int B, int H,
+                                  int Hkv, int N, int d, int causal, qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q_i8, q_scale, k_i8, k_scale, v, out);
+  if (s != QATTN_OK) return s;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  return dispatch_attn(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, d, causal,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t qattn_forward_workspace(int B, int H, int Hkv, int N, int d) {
+  if (check_shape(B, H, Hkv, N, d) != QATTN_OK) return 0;
+  return forward_layout(B, H, Hkv, N, d).total;
+}
+
+qattn_status qattn_forward_ws(const void* q, const void* k, const void* v, void* out, int B,
+                              int H, int Hkv, int N, int d, int causal, void* ws, size_t ws_bytes,
+                              qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q, k, v, out);
+  if (s != QATTN_OK) return s;
+  const QuantLayout L = forward_layout(B, H, Hkv, N, d);
+  if (ws == nullptr || ws_bytes < L.total) return QATTN_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QATTN_ERR_MISALIGNED;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int8_t* q_i8 = reinterpret_cast<int8_t*>(w + L.q_i8);
+  int8_t* k_i8 = reinterpret_cast<int8_t*>(w + L.k_i8);
+  float* q_scale = reinterpret_cast<float*>(w + L.q_scale);
+  float* k_scale = reinterpret_cast<float*>(w + L.k_scale);
+  long long* sums = reinterpret_cast<long long*>(w + L.sums);
+  s = dispatch_smooth_quant(q, k, B, H, Hkv, N, d, q_i8, q_scale, k_i8, k_scale, nullptr, sums, st);
+  if (s != QATTN_OK) return s;
+  return dispatch_attn(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, d, causal, st);
+}
+
+qattn_status qattn_forward(const void* q, const void* k, const void* v, void* out, int B, int H,
+                           int Hkv, int N, int d, int causal, qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q, k, v, out);
+  if (s != QATTN_OK) return s;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = forward_layout(B, H, Hkv, N, d).total;
+  void* ws = nullptr;
+  if ((s = pool_alloc(&ws, bytes, st)) != QATTN_OK) return s;
+  s = qattn_forward_ws(q, k, v, out, B, H, Hkv, N, d, causal, ws, bytes, stream);
+  if (cudaFreeAsync(ws, st) != cudaSuccess && s == QATTN_OK) s = QATTN_ERR_CUDA;
+  return s;
+}
+
+qattn_status qattn_forward_host(const void* q_host, const void* k_host, const void* v_host,
+                                void* out_host, int B, int H, int Hkv, int N, int d, int causal,
+                                qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  if (!q_host || !k_host || !v_host || !out_host) return QATTN_ERR_INVALID_ARG;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t qb = sizeof(uint16_t) * static_cast<size_t>(B) * H * N * d;
+  const size_t kb = sizeof(uint16_t) * static_cast<size_t>(B) * Hkv * N * d;
+  const size_t off_k = align_up(qb), off_v = off_k + align_up(kb), off_o = off_v + align_up(kb);
+  const size_t total = off_o + align_up(qb);
+  void* buf = nullptr;
+  if ((s = pool_alloc(&buf, total, st)) != QATTN_OK) return s;
+  uint8_t* b8 = static_cast<uint8_t*>(buf);
+  if (cudaMemcpyAsync(b8, q_host, qb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(b8 + off_k, k_host, kb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(b8 + off_v, v_host, kb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    s = QATTN_ERR_CUDA;
+  if (s == QATTN_OK)
+    s = qattn_forward(b8, b8 + off_k, b8 + off_v, b8 + off_o, B, H, Hkv, N, d, causal, stream);
+  if (s == QATTN_OK &&
+      cudaMemcpyAsync(out_host, b8 + off_o, qb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    s = QATTN_ERR_CUDA;
+  if (cudaFreeAsync(buf, st) != cudaSuccess && s == QATTN_OK) s = QATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess && s == QATTN_OK) s = QATTN_ERR_CUDA;
+  return s;
+}
+
+qattn_status qattn_debug_qk_int32(const int8_t* q_i8, const int8_t* k_i8, int32_t* s_out, int B,
+                                  int H, int Hkv, int N, int d, int b, int h, int qt0, int nqt,
+                                  int kt0, int nkt, qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q_i8, k_i8, s_out);
+  if (s != QATTN_OK) return s;
+  const int ntiles = (N + 127) / 128;
+  if (b < 0 || b >= B || h < 0 || h >= H || qt0 < 0 || nqt < 1 || kt0 < 0 || nkt < 1 ||
+      qt0 + nqt > ntiles || kt0 + nkt > ntiles || nqt > 65535 || nkt > 65535)
+    return QATTN_ERR_INVALID_ARG;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  CUtensorMap tq, tk;
+  if (!make_i8_map(&tq, q_i8, d, N, static_cast<long long>(B) * H) ||
+      !make_i8_map(&tk, k_i8, d, N, static_cast<long long>(B) * Hkv))
+    return QATTN_ERR_CUDA;
+  // 64 KB of shared memory per CTA caps residency at 3 CTAs (384 TMEM columns) per SM.
+  const int smem = 64 * 1024;
+  const int bh = b * H + h;
+  const int bg = b * Hkv + h / (H / Hkv);
+  dim3 grid(nqt, nkt);
+  if (d == 128) {
+    if (cudaFuncSetAttribute(qk_int32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return QATTN_ERR_CUDA;
+    qk_int32_kernel<128><<<grid, 128, smem, st>>>(tq, tk, s_out, bh, bg, qt0, kt0, nkt * 128);
+  } else {
+    if (cudaFuncSetAttribute(qk_int32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return QATTN_ERR_CUDA;
+    qk_int32_kernel<64><<<grid, 128, smem, st>>>(tq, tk, s_out, bh, bg, qt0, kt0, nkt * 128);
+  }
+  return launch_status();
+}
+
+qattn_status qattn_check_device_status(qattn_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return QATTN_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, qattn::g_device_status, sizeof(v)) != cudaSuccess)
+    return QATTN_ERR_CUDA;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    cudaMemcpyToSymbol(qattn::g_device_status, &zero, sizeof(zero));
+    return static_cast<qattn_status>(v);
+  }
+  return QATTN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,189 @@
+// quant.cuh -- smoothing of K and per-block INT8 quantization of Q and K' (SageAttention summary
+// page, aibr.jp/archives/102657, sec. 3: smooth K, quantize to INT8).  Both kernels are bound by
+// HBM bandwidth: 16-byte coalesced loads, warp-shuffle reductions, one pass over the data each.
+//
+// Bit-exactness.  The codes and scales are exact functions of the inputs:
+//  * the channel sums are exact int64 sums of K * 2^24 (every fp16 value is an integer multiple of
+//    2^-24), so the order of the atomic additions does not matter;
+//  * mean = (float)((double)sum / (N * 2^24)) with correctly rounded operations;
+//  * K' = (float)K - mean, amax, scale = amax / 127 are single correctly rounded binary32 ops;
+//  * code = rint(x / scale): computed as rint(x * (1/scale)), which equals rint(x / scale) unless
+//    x / scale lies within 2^-13 of a half-integer (the two quotients differ by less than 2^-16
+//    for |x / scale| <= 128); those rare elements take the correctly rounded division.
+// Build without fast-math so that division, reciprocal and conversions round to nearest-even
+// and subnormals are kept.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cstdint>
+
+namespace qattn {
+
+constexpr int kQBlock = 128;  // Q quantization block: 128 consecutive rows of one head
+constexpr int kKBlock = 64;   // K quantization block: 64 consecutive rows of one kv head
+constexpr int kSumRowsPerCta = 512;
+
+__device__ __forceinline__ float half_bits_to_float(uint32_t bits16) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(bits16)));
+}
+
+// ---------------------------------------------------------------------------------------------
+// K channel sums: sums[bg * D + c] += sum over this CTA's rows of K[bg, n, c] * 2^24 (exact).
+// grid (B*Hkv, ceil(N / kSumRowsPerCta)), 256 threads.  sums must be zeroed beforehand.
+// ---------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) k_channel_sums_kernel(const uint16_t* __restrict__ k, int N,
+                                                             long long* __restrict__ sums) {
+  constexpr int VPR = D / 8;            // 16-byte vectors per row
+  constexpr int RPI = 256 / VPR;        // rows per iteration of the CTA
+  __shared__ long long red[RPI][D];
+  const int bg = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int cg = tid % VPR;
+  const int r_in = tid / VPR;
+  const int n0 = blockIdx.y * kSumRowsPerCta;
+  const int n1 = min(N, n0 + kSumRowsPerCta);
+  const uint4* base = reinterpret_cast<const uint4*>(k + static_cast<size_t>(bg) * N * D);
+  long long acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0;
+  for (int n = n0 + r_in; n < n1; n += RPI) {
+    const uint4 v = __ldg(base + static_cast<size_t>(n) * VPR + cg);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc[2 * e] += __float2ll_rn(half_bits_to_float(w[e] & 0xFFFFu) * 16777216.0f);
+      acc[2 * e + 1] += __float2ll_rn(half_bits_to_float(w[e] >> 16) * 16777216.0f);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[r_in][cg * 8 + e] = acc[e];
+  __syncthreads();
+  for (int c = tid; c < D; c += 256) {
+    long long s = 0;
+#pragma unroll 4
+    for (int r = 0; r < RPI; ++r) s += red[r][c];
+    atomicAdd(reinterpret_cast<unsigned long long*>(sums + static_cast<size_t>(bg) * D + c),
+              static_cast<unsigned long long>(s));
+  }
+}
+
+// rint(x / s) for x, s > 0 as described in the file header.
+__device__ __forceinline__ float quant_code(float x, float s, float rcp) {
+  const float y = x * rcp;
+  const float f = y - floorf(y);
+  float t = y;
+  if (fabsf(f - 0.5f) < 1.220703125e-4f) t = __fdiv_rn(x, s);  // within 2^-13 of a tie
+  float r = rintf(t);
+  r = fminf(fmaxf(r, -127.0f), 127.0f);
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack4_i8(float a, float b, float c, float d) {
+  const uint32_t ua = static_cast<uint32_t>(static_cast<int>(a)) & 0xFFu;
+  const uint32_t ub = static_cast<uint32_t>(static_cast<int>(b)) & 0xFFu;
+  const uint32_t uc = static_cast<uint32_t>(static_cast<int>(c)) & 0xFFu;
+  const uint32_t ud = static_cast<uint32_t>(static_cast<int>(d)) & 0xFFu;
+  return ua | (ub << 8) | (uc << 16) | (ud << 24);
+}
+
+// One quantization block of R rows x D channels, 256 threads.  src: fp16 rows of the block
+// (head base + r0 * D); mean: per-channel smoothing offsets in shared memory (K) or nullptr (Q).
+template <int D, int R>
+__device__ __forceinline__ void quantize_block_cta(const uint16_t* __restrict__ src, int rows,
+                                                   const float* mean_s, int8_t* __restrict__ dst,
+                                                   float* __restrict__ scale_out, float* red) {
+  constexpr int VPR = D / 8;
+  constexpr int VPT = R * VPR / 256;  // vectors per thread
+  const int tid = threadIdx.x;
+  const int cg = tid % VPR;
+  float x[VPT][8];
+  float m[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) m[e] = mean_s ? mean_s[cg * 8 + e] : 0.0f;
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int vi = tid + i * 256;
+    const int r = vi / VPR;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < rows) v = __ldg(reinterpret_cast<const uint4*>(src) + vi);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      x[i][2 * e] = half_bits_to_float(w[e] & 0xFFFFu) - m[2 * e];
+      x[i][2 * e + 1] = half_bits_to_float(w[e] >> 16) - m[2 * e + 1];
+    }
+    if (r >= rows) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[i][e] = 0.0f;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[i][e]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  if ((tid & 31) == 0) red[tid >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
+  const float s = __fdiv_rn(amax, 127.0f);
+  const float rcp = amax > 0.0f ? __frcp_rn(s) : 0.0f;
+  if (tid == 0) *scale_out = amax > 0.0f ? s : 0.0f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int vi = tid + i * 256;
+    const int r = vi / VPR;
+    if (r < rows) {
+      float q[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) q[e] = amax > 0.0f ? quant_code(x[i][e], s, rcp) : 0.0f;
+      uint2 out;
+      out.x = pack4_i8(q[0], q[1], q[2], q[3]);
+      out.y = pack4_i8(q[4], q[5], q[6], q[7]);
+      reinterpret_cast<uint2*>(dst)[vi] = out;
+    }
+  }
+}
+
+// Quantizes every Q block and every K' block in one launch: blocks [0, nq) are Q blocks in
+// (b*H + h, block) order, blocks [nq, nq + nk) are K blocks in (b*Hkv + g, block) order.
+// 256 threads.  For K blocks the CTA first forms the channel means of its kv head from the
+// exact sums; the first K block of each kv head also writes them to k_mean (if not null).
+template <int D>
+__global__ void __launch_bounds__(256) quantize_kernel(
+    const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, int N, int nqb, int nkb,
+    long long nq, const long long* __restrict__ sums, int8_t* __restrict__ q_i8,
+    float* __restrict__ q_scale, int8_t* __restrict__ k_i8, float* __restrict__ k_scale,
+    float* __restrict__ k_mean) {
+  __shared__ float mean_s[D];
+  __shared__ float red[8];
+  const long long blk = blockIdx.x;
+  if (blk < nq) {
+    const long long bh = blk / nqb;
+    const int qb = static_cast<int>(blk % nqb);
+    const int r0 = qb * kQBlock;
+    const int rows = min(kQBlock, N - r0);
+    const size_t off = (static_cast<size_t>(bh) * N + r0) * D;
+    quantize_block_cta<D, kQBlock>(q + off, rows, nullptr, q_i8 + off, q_scale + blk, red);
+  } else {
+    const long long kblk = blk - nq;
+    const long long bg = kblk / nkb;
+    const int kb = static_cast<int>(kblk % nkb);
+    if (threadIdx.x < D) {
+      const long long s = sums[bg * D + threadIdx.x];
+      const double den = static_cast<double>(N) * 16777216.0;
+      const float mu = __double2float_rn(__ddiv_rn(__ll2double_rn(s), den));
+      mean_s[threadIdx.x] = mu;
+      if (kb == 0 && k_mean != nullptr) k_mean[bg * D + threadIdx.x] = mu;
+    }
+    __syncthreads();
+    const int r0 = kb * kKBlock;
+    const int rows = min(kKBlock, N - r0);
+    const size_t off = (static_cast<size_t>(bg) * N + r0) * D;
+    quantize_block_cta<D, kKBlock>(k + off, rows, mean_s, k_i8 + off, k_scale + kblk, red);
+  }
+}
+
+}  // namespace qattn

@@ -1,0 +1,198 @@
+"""ctypes binding of the C ABI in include/qattn.h (argument marshalling only).
+
+Every computation runs in the CUDA library ``libqattn.so``; there is no CPU or PyTorch fallback.
+If the library is missing (or cannot be built) every call raises.  PyTorch supplies device
+memory and streams.  Function names match the C entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+QATTN_OK = 0
+STATUS = {
+    0: "QATTN_OK", 1: "QATTN_ERR_INVALID_ARG", 2: "QATTN_ERR_UNSUPPORTED",
+    3: "QATTN_ERR_MISALIGNED", 4: "QATTN_ERR_CUDA", 5: "QATTN_ERR_TIMEOUT",
+    6: "QATTN_ERR_WORKSPACE",
+}
+QBLOCK = 128
+KBLOCK = 64
+
+# Every symbol include/qattn.h declares.
+EXPORTS = [
+    "qattn_status_string", "qattn_version", "qattn_smooth_quant_workspace", "qattn_smooth_quant",
+    "qattn_attn_quantized", "qattn_forward_workspace", "qattn_forward_ws", "qattn_forward",
+    "qattn_forward_host", "qattn_debug_qk_int32", "qattn_check_device_status",
+]
+
+
+class QattnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} "
+                         f"({_lib().qattn_status_string(status).decode()})")
+
+
+_L = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def _lib():
+    global _L
+    if _L is None:
+        if _build.stale():
+            if not os.path.exists(_build.NVCC):
+                raise RuntimeError("libqattn.so is missing or stale and nvcc is not available")
+            _build.build()
+        L = ctypes.CDLL(_build.LIB)
+        P, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.qattn_status_string.argtypes = [i]
+        L.qattn_status_string.restype = ctypes.c_char_p
+        L.qattn_version.argtypes = []
+        L.qattn_version.restype = i
+        L.qattn_smooth_quant_workspace.argtypes = [i, i, i]
+        L.qattn_smooth_quant_workspace.restype = sz
+        L.qattn_smooth_quant.argtypes = [P, P, i, i, i, i, i, P, P, P, P, P, P, sz, P]
+        L.qattn_smooth_quant.restype = i
+        L.qattn_attn_quantized.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, P]
+        L.qattn_attn_quantized.restype = i
+        L.qattn_forward_workspace.argtypes = [i, i, i, i, i]
+        L.qattn_forward_workspace.restype = sz
+        L.qattn_forward_ws.argtypes = [P, P, P, P, i, i, i, i, i, i, P, sz, P]
+        L.qattn_forward_ws.restype = i
+        L.qattn_forward.argtypes = [P, P, P, P, i, i, i, i, i, i, P]
+        L.qattn_forward.restype = i
+        L.qattn_forward_host.argtypes = [P, P, P, P, i, i, i, i, i, i, P]
+        L.qattn_forward_host.restype = i
+        L.qattn_debug_qk_int32.argtypes = [P, P, P, i, i, i, i, i, i, i, i, i, i, i, P]
+        L.qattn_debug_qk_int32.restype = i
+        L.qattn_check_device_status.argtypes = [P]
+        L.qattn_check_device_status.restype = i
+        _L = L
+    return _L
+
+
+def load():
+    """Loads (building if needed) the CUDA library; returns the ctypes handle."""
+    return _lib()
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    assert t.is_contiguous(), "tensors must be contiguous"
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(fn: str, st: int):
+    if st != QATTN_OK:
+        raise QattnError(fn, st)
+
+
+def _dims(q: torch.Tensor, k: torch.Tensor):
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    return B, H, Hkv, N, d
+
+
+# ------------------------------------------------------------------------------------------------
+
+def qattn_smooth_quant_workspace(B: int, Hkv: int, d: int) -> int:
+    return int(_lib().qattn_smooth_quant_workspace(B, Hkv, d))
+
+
+def qattn_smooth_quant(q, k, q_i8=None, q_scale=None, k_i8=None, k_scale=None, k_mean=None,
+                       ws=None, stream=None, want_mean=True):
+    """Smooths K and quantizes Q, K' on the GPU.  Allocates missing outputs with torch; returns
+    (q_i8, q_scale, k_i8, k_scale, k_mean)."""
+    B, H, Hkv, N, d = _dims(q, k)
+    dev = q.device
+    nqb, nkb = -(-N // QBLOCK), -(-N // KBLOCK)
+    q_i8 = torch.empty(B, H, N, d, dtype=torch.int8, device=dev) if q_i8 is None else q_i8
+    k_i8 = torch.empty(B, Hkv, N, d, dtype=torch.int8, device=dev) if k_i8 is None else k_i8
+    q_scale = torch.empty(B, H, nqb, dtype=torch.float32, device=dev) if q_scale is None else q_scale
+    k_scale = torch.empty(B, Hkv, nkb, dtype=torch.float32, device=dev) if k_scale is None else k_scale
+    if k_mean is None and want_mean:
+        k_mean = torch.empty(B, Hkv, d, dtype=torch.float32, device=dev)
+    wsb = qattn_smooth_quant_workspace(B, Hkv, d)
+    if ws is None:
+        ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    st = _lib().qattn_smooth_quant(_p(q), _p(k), B, H, Hkv, N, d, _p(q_i8), _p(q_scale), _p(k_i8),
+                                   _p(k_scale), _p(k_mean), _p(ws), ws.numel(), _stream(stream))
+    _check("qattn_smooth_quant", st)
+    return q_i8, q_scale, k_i8, k_scale, k_mean
+
+
+def qattn_attn_quantized(q_i8, q_scale, k_i8, k_scale, v, out=None, causal=False, stream=None):
+    B, H, Hkv, N, d = _dims(q_i8, k_i8)
+    out = torch.empty(B, H, N, d, dtype=torch.float16, device=v.device) if out is None else out
+    st = _lib().qattn_attn_quantized(_p(q_i8), _p(q_scale), _p(k_i8), _p(k_scale), _p(v), _p(out),
+                                     B, H, Hkv, N, d, int(bool(causal)), _stream(stream))
+    _check("qattn_attn_quantized", st)
+    return out
+
+
+def qattn_forward_workspace(B: int, H: int, Hkv: int, N: int, d: int) -> int:
+    return int(_lib().qattn_forward_workspace(B, H, Hkv, N, d))
+
+
+def qattn_forward_ws(q, k, v, out=None, causal=False, ws=None, stream=None):
+    B, H, Hkv, N, d = _dims(q, k)
+    out = torch.empty_like(q) if out is None else out
+    if ws is None:
+        ws = torch.empty(qattn_forward_workspace(B, H, Hkv, N, d), dtype=torch.uint8,
+                         device=q.device)
+    st = _lib().qattn_forward_ws(_p(q), _p(k), _p(v), _p(out), B, H, Hkv, N, d,
+                                 int(bool(causal)), _p(ws), ws.numel(), _stream(stream))
+    _check("qattn_forward_ws", st)
+    return out
+
+
+def qattn_forward(q, k, v, out=None, causal=False, stream=None):
+    """The plug-and-play forward: fp16 q [B,H,N,d], k/v [B,Hkv,N,d] on the GPU -> fp16 out."""
+    B, H, Hkv, N, d = _dims(q, k)
+    out = torch.empty_like(q) if out is None else out
+    st = _lib().qattn_forward(_p(q), _p(k), _p(v), _p(out), B, H, Hkv, N, d, int(bool(causal)),
+                              _stream(stream))
+    _check("qattn_forward", st)
+    return out
+
+
+def qattn_forward_host(q, k, v, out=None, causal=False, stream=None):
+    """Forward on host (CPU, preferably pinned) fp16 tensors; returns after out_host is filled."""
+    B, H, Hkv, N, d = _dims(q, k)
+    out = torch.empty_like(q) if out is None else out
+    st = _lib().qattn_forward_host(_p(q), _p(k), _p(v), _p(out), B, H, Hkv, N, d,
+                                   int(bool(causal)), _stream(stream))
+    _check("qattn_forward_host", st)
+    return out
+
+
+def qattn_debug_qk_int32(q_i8, k_i8, b, h, qt0, nqt, kt0, nkt, s_out=None, stream=None):
+    B, H, Hkv, N, d = _dims(q_i8, k_i8)
+    if s_out is None:
+        s_out = torch.empty(nqt * 128, nkt * 128, dtype=torch.int32, device=q_i8.device)
+    st = _lib().qattn_debug_qk_int32(_p(q_i8), _p(k_i8), _p(s_out), B, H, Hkv, N, d, b, h, qt0,
+                                     nqt, kt0, nkt, _stream(stream))
+    _check("qattn_debug_qk_int32", st)
+    return s_out
+
+
+def qattn_check_device_status(stream=None) -> int:
+    return int(_lib().qattn_check_device_status(_stream(stream)))

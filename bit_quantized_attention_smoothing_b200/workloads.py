@@ -119,13 +119,15 @@ def digest(*tensors: torch.Tensor) -> str:
     return h.hexdigest()[:16]
 
 
-def sample_rows(w: Workload, per_head: int, seed: int = 7):
-    """Seeded query rows to compare on large workloads: per (b, h), the first and last 128 rows of
-    the sequence (clipped to N) plus `per_head` uniformly drawn rows.  Returns (row_bh, row_i) as
-    int64 CPU tensors, sorted."""
+def sample_rows(w: Workload, per_head: int, seed: int = 7, edge_first: int = 128,
+                edge_last: int = 128):
+    """Seeded query rows to compare on large workloads: per (b, h), the first `edge_first` and last
+    `edge_last` rows of the sequence (clipped to N) plus `per_head` uniformly drawn rows.  Returns
+    (row_bh, row_i) as int64 CPU tensors, sorted within each head."""
     gen = torch.Generator().manual_seed(seed)
     bh_all, i_all = [], []
-    edge = torch.cat([torch.arange(0, min(128, w.N)), torch.arange(max(0, w.N - 128), w.N)])
+    edge = torch.cat([torch.arange(0, min(edge_first, w.N)),
+                      torch.arange(max(0, w.N - edge_last), w.N)])
     for bh in range(w.B * w.H):
         rnd = torch.randint(0, w.N, (per_head,), generator=gen)
         rows = torch.unique(torch.cat([edge, rnd]))

@@ -1,0 +1,140 @@
+/*
+ * qattn.h -- C ABI of the B200 (sm_100a) smoothed-K INT8 attention forward (prefill).
+ *
+ * The method is the 8-bit attention summarised on the SageAttention page
+ * ("SAGEATTENTION: accurate 8-bit attention for plug-and-play inference acceleration",
+ * aibr.jp/archives/102657):
+ *   - sec. 3: K is smoothed before quantization, Q and K are quantized to INT8, Q K^T runs on the
+ *     tensor cores with 32-bit integer accumulation (mma(u8.u8.s32) on the page's GPU; signed
+ *     s8 x s8 -> s32 here), P V runs with FP16 operands (mma(f16.f16.f16) on the page's GPU);
+ *   - sec. 4: the kernel keeps FlashAttention's blockwise online softmax;
+ *   - dialogue and sec. 2: it is a plug-and-play replacement of the attention call.
+ * Where the page is silent this library takes these readings:
+ *   - smoothing subtracts the per-channel mean of K over all N tokens of each (batch, kv head);
+ *     the channel sum is exact (int64 of K * 2^24), mean = (float)((double)sum / (N * 2^24)),
+ *     K' = (float)K - mean in binary32;
+ *   - Q is quantized in blocks of 128 consecutive rows, K' in blocks of 64 rows (all d channels
+ *     of one head); scale = amax / 127 (binary32 division), code = clamp(rint(x / scale), -127,
+ *     127), ties to even; amax == 0 gives scale 0 and codes 0;
+ *   - scores are S = S_int * sQ * sK / sqrt(d); causal attention keeps key j <= query i;
+ *   - grouped-query attention maps query head h to kv head h / (H / Hkv).
+ *
+ * Conventions for every entry point:
+ *   - All tensors are contiguous row-major device buffers owned by the caller:
+ *       q, out      fp16 [B, H,   N, d]
+ *       k, v        fp16 [B, Hkv, N, d]
+ *       q_i8        int8 [B, H,   N, d]      q_scale float [B, H,   ceil(N/128)]
+ *       k_i8        int8 [B, Hkv, N, d]      k_scale float [B, Hkv, ceil(N/64)]
+ *       k_mean      float [B, Hkv, d]
+ *     The library never frees or retains a caller pointer.
+ *   - Supported: d in {64, 128}; 1 <= N <= 1048576; H % Hkv == 0; every pointer 16-byte aligned.
+ *     Inputs must be finite (NaN/Inf give undefined results).
+ *   - Arguments are checked on the host before anything is launched; a failed check returns an
+ *     error status and launches nothing.  All work is asynchronous on `stream` (0 = legacy default
+ *     stream) unless an entry point says otherwise.  Launch failures return QATTN_ERR_CUDA.
+ *   - Every wait inside a kernel is bounded; a wait that runs out records QATTN_ERR_TIMEOUT in a
+ *     device status word that qattn_check_device_status() reads.
+ */
+#ifndef QATTN_H
+#define QATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared here so that the header needs no CUDA header. */
+typedef struct CUstream_st* qattn_stream_t;
+
+typedef enum {
+    QATTN_OK = 0,
+    QATTN_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, H % Hkv != 0 */
+    QATTN_ERR_UNSUPPORTED = 2,   /* d not in {64, 128}, N out of range, no sm_100 device */
+    QATTN_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
+    QATTN_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    QATTN_ERR_TIMEOUT = 5,       /* a bounded wait inside a kernel ran out (device status) */
+    QATTN_ERR_WORKSPACE = 6      /* workspace missing or smaller than required */
+} qattn_status;
+
+/* Static text for a status code (never NULL). */
+const char* qattn_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int qattn_version(void);
+
+/* ------------------------------------------------------------------------------------------
+ * Pre-processing: smoothing of K and per-block INT8 quantization of Q and K' (page sec. 3).
+ * ------------------------------------------------------------------------------------------ */
+
+/* Bytes of device workspace qattn_smooth_quant needs (the exact int64 channel sums). */
+size_t qattn_smooth_quant_workspace(int B, int Hkv, int d);
+
+/* Smooths K and quantizes Q and K'.  Writes q_i8, q_scale, k_i8, k_scale and, when k_mean is
+ * not NULL, the per-channel means.  ws: caller-owned device buffer of at least
+ * qattn_smooth_quant_workspace() bytes (256-byte alignment recommended), clobbered.  The codes
+ * and scales are bit-exact functions of the inputs (no dependence on launch order). */
+qattn_status qattn_smooth_quant(const void* q, const void* k, int B, int H, int Hkv, int N, int d,
+                                int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
+                                float* k_mean, void* ws, size_t ws_bytes, qattn_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Attention on already-quantized Q and K (page sec. 3 and 4): S_int = Q_i8 K_i8^T exactly in
+ * int32 on the tensor cores (tcgen05 kind::i8, accumulator in tensor memory), dequantized with
+ * the block scales, blockwise online softmax in fp32, P rounded to fp16, O += P V on the tensor
+ * cores (tcgen05 kind::f16, fp32 accumulator), O / l rounded to fp16.
+ * causal != 0 keeps key j <= query i and skips tiles above the diagonal.
+ * ------------------------------------------------------------------------------------------ */
+qattn_status qattn_attn_quantized(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                                  const float* k_scale, const void* v, void* out, int B, int H,
+                                  int Hkv, int N, int d, int causal, qattn_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * The whole forward: fp16 q, k, v in, fp16 out (the plug-and-play call of the page's dialogue
+ * and sec. 2).  Smoothing + quantization, then attention.
+ * ------------------------------------------------------------------------------------------ */
+
+/* Bytes of device workspace qattn_forward_ws needs (int8 Q and K, scales, channel sums). */
+size_t qattn_forward_workspace(int B, int H, int Hkv, int N, int d);
+
+/* Forward with a caller-owned workspace of at least qattn_forward_workspace() bytes. */
+qattn_status qattn_forward_ws(const void* q, const void* k, const void* v, void* out, int B,
+                              int H, int Hkv, int N, int d, int causal, void* ws, size_t ws_bytes,
+                              qattn_stream_t stream);
+
+/* Forward that takes its workspace, stream-ordered, from a memory pool the library keeps per
+ * device (allocated on first use, reused afterwards, released at process exit). */
+qattn_status qattn_forward(const void* q, const void* k, const void* v, void* out, int B, int H,
+                           int Hkv, int N, int d, int causal, qattn_stream_t stream);
+
+/* Forward on HOST buffers: copies q, k, v to the device, runs qattn_forward, copies the result
+ * back to out_host, and returns after the copy has finished (the stream is synchronized).  Device
+ * buffers come from the library's pool.  Page-locked host memory gives asynchronous copies;
+ * pageable memory works but is slower. */
+qattn_status qattn_forward_host(const void* q_host, const void* k_host, const void* v_host,
+                                void* out_host, int B, int H, int Hkv, int N, int d, int causal,
+                                qattn_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Checks.
+ * ------------------------------------------------------------------------------------------ */
+
+/* int32 score tiles S_int = Q_i8 K_i8^T through the same TMA -> tcgen05.mma kind::i8 -> tensor
+ * memory -> tcgen05.ld path the attention kernel uses, without masking: for query tiles
+ * qt0 .. qt0+nqt-1 and key tiles kt0 .. kt0+nkt-1 (128 rows each) of batch b, query head h.
+ * s_out: device int32 [nqt*128, nkt*128], row-major; rows or columns beyond N are written as the
+ * product with zero-filled rows (0). */
+qattn_status qattn_debug_qk_int32(const int8_t* q_i8, const int8_t* k_i8, int32_t* s_out, int B,
+                                  int H, int Hkv, int N, int d, int b, int h, int qt0, int nqt,
+                                  int kt0, int nkt, qattn_stream_t stream);
+
+/* Synchronizes `stream`, then reports and clears the device status word: QATTN_OK, or
+ * QATTN_ERR_TIMEOUT when a bounded wait inside a kernel ran out since the last check. */
+qattn_status qattn_check_device_status(qattn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QATTN_H */

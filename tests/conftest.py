@@ -17,3 +17,38 @@ def oracle():
     from oracle import oracle as O
     O.build()
     return O
+
+
+def has_gpu():
+    import torch
+    return torch.cuda.is_available()
+
+
+@pytest.fixture(scope="session")
+def lib():
+    """The CUDA binding; GPU tests only."""
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from bit_quantized_attention_smoothing_b200 import qattn as Q
+    Q.load()
+    return Q
+
+
+def np16(t):
+    """fp16 torch tensor (any device) -> contiguous numpy uint16 bit patterns."""
+    import numpy as np
+    return t.detach().contiguous().cpu().numpy().view(np.uint16)
+
+
+def out_errors(gpu_out_rows, ref64_rows):
+    """(max-abs, mean-abs) error of fp16 GPU rows against the oracle's unrounded float64 rows."""
+    import numpy as np
+    g = gpu_out_rows.astype(np.float64)
+    e = np.abs(g - ref64_rows)
+    return float(e.max()), float(e.mean())
+
+
+# Output tolerances of the forward against the oracle's unrounded float64 output.
+MAX_ABS_TOL = 2e-3
+MEAN_ABS_TOL = 2e-4

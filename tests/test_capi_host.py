@@ -1,0 +1,99 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds and loads, exports every
+symbol include/qattn.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_quantized_attention_smoothing_b200 import build as B
+from bit_quantized_attention_smoothing_b200 import qattn as Q
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "qattn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qattn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_builds_and_loads():
+    path = B.build()
+    assert os.path.exists(path)
+    Q.load()
+
+
+def test_exports_every_declared_symbol():
+    L = ctypes.CDLL(B.build())
+    names = declared_functions()
+    assert set(names) == set(Q.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_version():
+    L = Q.load()
+    for code in range(7):
+        assert L.qattn_status_string(code)
+    assert L.qattn_status_string(99) == b"unknown status"
+    assert L.qattn_version() >= 100
+
+
+def test_workspace_sizes():
+    L = Q.load()
+    assert L.qattn_smooth_quant_workspace(1, 8, 128) == 8 * 128 * 8
+    assert L.qattn_smooth_quant_workspace(0, 8, 128) == 0
+    ws = L.qattn_forward_workspace(1, 32, 8, 32768, 128)
+    need = 32 * 32768 * 128 + 8 * 32768 * 128 + 4 * 32 * 256 + 4 * 8 * 512 + 8 * 8 * 128
+    assert need <= ws <= need + 5 * 256
+    assert L.qattn_forward_workspace(1, 32, 8, 32768, 96) == 0
+    assert L.qattn_forward_workspace(1, 30, 8, 32768, 128) == 0
+
+
+P = ctypes.c_void_p
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((P(16), P(32), P(48), P(64), 1, 4, 2, 256, 128, 0, None), Q.QATTN_OK - 0 + 4),  # device call
+    ((None, P(32), P(48), P(64), 1, 4, 2, 256, 128, 0, None), 1),
+    ((P(16), P(32), P(48), P(64), 1, 4, 3, 256, 128, 0, None), 1),
+    ((P(16), P(32), P(48), P(64), 0, 4, 2, 256, 128, 0, None), 1),
+    ((P(16), P(32), P(48), P(64), 1, 4, 2, 0, 128, 0, None), 1),
+    ((P(16), P(32), P(48), P(64), 1, 4, 2, 256, 96, 0, None), 2),
+    ((P(16), P(32), P(48), P(64), 1, 4, 2, (1 << 20) + 1, 128, 0, None), 2),
+    ((P(16), P(33), P(48), P(64), 1, 4, 2, 256, 128, 0, None), 3),
+])
+def test_forward_argument_checks(args, expect):
+    L = Q.load()
+    st = L.qattn_forward(*args)
+    if expect == 4:
+        # valid arguments reach the device query; without a GPU that fails as a CUDA error
+        import torch
+        if torch.cuda.is_available():
+            pytest.skip("argument check only; this box has a GPU")
+        assert st == 4
+    else:
+        assert st == expect
+
+
+def test_workspace_and_alignment_checks():
+    L = Q.load()
+    need = L.qattn_forward_workspace(1, 4, 2, 256, 128)
+    st = L.qattn_forward_ws(P(16), P(32), P(48), P(64), 1, 4, 2, 256, 128, 1, P(4096), need - 1, None)
+    assert st == 6
+    st = L.qattn_forward_ws(P(16), P(32), P(48), P(64), 1, 4, 2, 256, 128, 1, None, need, None)
+    assert st == 6
+    st = L.qattn_forward_ws(P(16), P(32), P(48), P(64), 1, 4, 2, 256, 128, 1, P(4100), need, None)
+    assert st == 3
+    st = L.qattn_smooth_quant(P(16), P(32), 1, 4, 2, 256, 128, P(48), P(64), P(80), P(96), None,
+                              P(112), 8, None)
+    assert st == 6
+    st = L.qattn_smooth_quant(P(16), P(32), 1, 4, 2, 256, 128, P(48), P(64), P(80), P(96), P(20),
+                              P(112), 1 << 20, None)
+    assert st == 3
+    st = L.qattn_debug_qk_int32(P(16), P(32), P(48), 1, 4, 2, 256, 128, 0, 0, 1, 2, 0, 1, None)
+    assert st == 1
+    st = L.qattn_debug_qk_int32(P(16), P(32), P(48), 1, 4, 2, 256, 128, 0, 4, 0, 1, 0, 1, None)
+    assert st == 1

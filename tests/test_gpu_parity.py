@@ -1,0 +1,175 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the same seeded inputs.
+
+* smoothing + quantization (int8 codes, block scales, channel means): bit-exact;
+* int32 score tiles from the tcgen05 kind::i8 path: bit-exact;
+* forward output: max-abs <= 2e-3 and mean-abs <= 2e-4 against the oracle's unrounded float64
+  output (the oracle rounds nothing after the int32 product; the GPU rounds P to fp16, accumulates
+  in fp32, uses a hardware exp2 and rounds O to fp16).
+
+Small cases compare every output element and cover ragged N (partial Q tile, partial K block,
+odd tile counts), N=1, GQA, causal and non-causal, d=64 and d=128.  The five named workloads run at
+full size with the bench's launch configuration, comparing every int8 code and scale and a seeded
+sample of output rows (first and last rows of every head plus random rows).
+"""
+import numpy as np
+import pytest
+import torch
+
+from bit_quantized_attention_smoothing_b200.workloads import ORDER, WORKLOADS, make_inputs, sample_rows
+from conftest import MAX_ABS_TOL, MEAN_ABS_TOL, np16, out_errors
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    ("tiny", {}),
+    ("tiny", {"N": 200}),
+    ("tiny", {"N": 1}),
+    ("tiny", {"N": 129, "causal": True}),
+    ("tiny", {"N": 64, "d": 128}),
+    ("prefill4k", {"B": 1, "H": 4, "Hkv": 2, "N": 1000}),
+    ("prefill4k", {"B": 2, "H": 2, "Hkv": 2, "N": 640, "causal": False}),
+    ("wide64", {"B": 1, "H": 2, "Hkv": 1, "N": 1500}),
+    ("long128k", {"H": 4, "Hkv": 1, "N": 2048}),
+    ("llama8b_32k", {"H": 8, "Hkv": 2, "N": 768}),
+    ("llama8b_32k", {"H": 2, "Hkv": 1, "N": 384}),
+    ("wide64", {"B": 1, "H": 3, "Hkv": 3, "N": 300, "causal": True}),
+]
+SMALL_IDS = [f"{n}-" + "-".join(f"{k}{v}" for k, v in o.items()) for n, o in SMALL]
+
+# rows sampled per head at full size (plus the first 128 and last 128 rows of every head)
+FULL_SAMPLES = {"tiny": None, "prefill4k": 32, "llama8b_32k": 32, "long128k": 4, "wide64": 32}
+
+
+def _inputs(w, device="cuda"):
+    q, k, v = make_inputs(w, device=device)
+    return q.cuda(), k.cuda(), v.cuda()
+
+
+def _check_quant(lib, oracle, w, q, k):
+    q_i8, q_scale, k_i8, k_scale, k_mean = lib.qattn_smooth_quant(q, k)
+    torch.cuda.synchronize()
+    ref = oracle.smooth_quant(np16(q), np16(k), w.B, w.H, w.Hkv, w.N, w.d)
+    assert np.array_equal(k_mean.cpu().numpy().view(np.uint32), ref["k_mean"].view(np.uint32))
+    assert np.array_equal(k_scale.cpu().numpy().view(np.uint32), ref["k_scale"].view(np.uint32))
+    assert np.array_equal(q_scale.cpu().numpy().view(np.uint32), ref["q_scale"].view(np.uint32))
+    assert np.array_equal(k_i8.cpu().numpy(), ref["k_i8"])
+    assert np.array_equal(q_i8.cpu().numpy(), ref["q_i8"])
+    return (q_i8, q_scale, k_i8, k_scale), ref
+
+
+def _rows_of(out, w, rows):
+    bh, i = rows
+    flat = out.reshape(w.B * w.H * w.N, w.d)
+    idx = torch.as_tensor(np.asarray(bh) * w.N + np.asarray(i), device=out.device)
+    return flat[idx].float().cpu().numpy()
+
+
+@pytest.mark.parametrize("name,over", SMALL, ids=SMALL_IDS)
+def test_smooth_quant_bit_exact_small(lib, oracle, name, over):
+    w = WORKLOADS[name].with_(**over)
+    q, k, _ = _inputs(w, "cpu")
+    _check_quant(lib, oracle, w, q, k)
+
+
+@pytest.mark.parametrize("name,over", SMALL, ids=SMALL_IDS)
+def test_qk_int32_tiles_bit_exact_small(lib, oracle, name, over):
+    w = WORKLOADS[name].with_(**over)
+    q, k, _ = _inputs(w, "cpu")
+    (q_i8, _, k_i8, _), ref = _check_quant(lib, oracle, w, q, k)
+    nt = -(-w.N // 128)
+    for b, h in {(0, 0), (w.B - 1, w.H - 1)}:
+        s = lib.qattn_debug_qk_int32(q_i8, k_i8, b, h, 0, nt, 0, nt).cpu().numpy()
+        # rows/columns beyond N are products with zero-filled rows
+        full = np.zeros((nt * 128, nt * 128), dtype=np.int32)
+        full[: w.N, : w.N] = oracle.qk_int32(ref["q_i8"], ref["k_i8"], w.B, w.H, w.Hkv, w.N, w.d,
+                                             b, h, 0, w.N, 0, w.N)
+        assert np.array_equal(s, full)
+
+
+@pytest.mark.parametrize("name,over", SMALL, ids=SMALL_IDS)
+def test_forward_small_all_rows(lib, oracle, name, over):
+    w = WORKLOADS[name].with_(**over)
+    q, k, v = _inputs(w, "cpu")
+    out = lib.qattn_forward(q, k, v, causal=w.causal)
+    assert lib.qattn_check_device_status() == 0
+    ref, _ = oracle.forward(np16(q), np16(k), np16(v), w.B, w.H, w.Hkv, w.N, w.d, w.causal)
+    got = out.float().cpu().numpy().reshape(-1, w.d)
+    mx, mean = out_errors(got, ref)
+    assert mx <= MAX_ABS_TOL and mean <= MEAN_ABS_TOL, (mx, mean)
+
+
+@pytest.mark.parametrize("name,over", SMALL[:6], ids=SMALL_IDS[:6])
+def test_attention_on_oracle_codes(lib, oracle, name, over):
+    """The attention kernel alone, fed the oracle's int8 codes and scales."""
+    w = WORKLOADS[name].with_(**over)
+    q, k, v = _inputs(w, "cpu")
+    ref_sq = oracle.smooth_quant(np16(q), np16(k), w.B, w.H, w.Hkv, w.N, w.d)
+    t = {key: torch.from_numpy(val).cuda() for key, val in ref_sq.items()}
+    out = lib.qattn_attn_quantized(t["q_i8"], t["q_scale"], t["k_i8"], t["k_scale"], v,
+                                   causal=w.causal)
+    ref = oracle.attention_quantized(ref_sq["q_i8"], ref_sq["q_scale"], ref_sq["k_i8"],
+                                     ref_sq["k_scale"], np16(v), w.B, w.H, w.Hkv, w.N, w.d, w.causal)
+    mx, mean = out_errors(out.float().cpu().numpy().reshape(-1, w.d), ref)
+    assert mx <= MAX_ABS_TOL and mean <= MEAN_ABS_TOL, (mx, mean)
+
+
+def test_forward_variants_agree(lib):
+    w = WORKLOADS["prefill4k"].with_(B=1, H=4, Hkv=2, N=777)
+    q, k, v = _inputs(w, "cpu")
+    a = lib.qattn_forward(q, k, v, causal=True)
+    b = lib.qattn_forward_ws(q, k, v, causal=True)
+    c = lib.qattn_forward_host(q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory(),
+                               causal=True)
+    d = lib.qattn_forward_host(q.cpu(), k.cpu(), v.cpu(), causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert torch.equal(a.cpu(), c) and torch.equal(a.cpu(), d)
+
+
+def test_repeated_calls_are_deterministic(lib):
+    w = WORKLOADS["wide64"].with_(B=1, H=2, Hkv=2, N=1024)
+    q, k, v = _inputs(w, "cpu")
+    a = lib.qattn_forward(q, k, v, causal=False)
+    for _ in range(3):
+        assert torch.equal(a, lib.qattn_forward(q, k, v, causal=False))
+
+
+def test_gpu_rejects_bad_arguments(lib):
+    q = torch.zeros(1, 2, 64, 96, dtype=torch.float16, device="cuda")
+    with pytest.raises(lib.QattnError) as e:
+        lib.qattn_forward(q, q, q)
+    assert e.value.status == 2
+    q = torch.zeros(1, 3, 64, 64, dtype=torch.float16, device="cuda")
+    k = torch.zeros(1, 2, 64, 64, dtype=torch.float16, device="cuda")
+    with pytest.raises(lib.QattnError) as e:
+        lib.qattn_forward(q, k, k)
+    assert e.value.status == 1
+    assert lib.qattn_check_device_status() == 0
+
+
+@pytest.mark.parametrize("name", ORDER)
+def test_full_size_workload(lib, oracle, name):
+    """Full-size workload, same launch as the benchmark: every code and scale bit-exact, a seeded
+    sample of output rows within tolerance, plus int32 score tiles on the first/last tiles."""
+    w = WORKLOADS[name]
+    q, k, v = make_inputs(w, device="cuda")
+    (q_i8, _, k_i8, _), ref_sq = _check_quant(lib, oracle, w, q, k)
+    nt = -(-w.N // 128)
+    for qt, kt in {(0, 0), (nt - 1, nt - 1), (nt - 1, 0), (nt // 2, nt // 3)}:
+        s = lib.qattn_debug_qk_int32(q_i8, k_i8, w.B - 1, w.H - 1, qt, 1, kt, 1).cpu().numpy()
+        r = oracle.qk_int32(ref_sq["q_i8"], ref_sq["k_i8"], w.B, w.H, w.Hkv, w.N, w.d,
+                            w.B - 1, w.H - 1, qt * 128, 128, kt * 128, 128)
+        assert np.array_equal(s, r)
+    del q_i8, k_i8
+    out = lib.qattn_forward(q, k, v, causal=w.causal)
+    assert lib.qattn_check_device_status() == 0
+    per = FULL_SAMPLES[name]
+    if per is None:
+        rows = oracle.all_rows(w.B, w.H, w.N)
+    else:
+        rows = tuple(t.numpy() for t in sample_rows(w, per, edge_first=128, edge_last=128 if per > 4 else 8))
+    ref = oracle.attention_quantized(ref_sq["q_i8"], ref_sq["q_scale"], ref_sq["k_i8"],
+                                     ref_sq["k_scale"], np16(v), w.B, w.H, w.Hkv, w.N, w.d,
+                                     w.causal, rows=rows)
+    mx, mean = out_errors(_rows_of(out, w, rows), ref)
+    assert mx <= MAX_ABS_TOL and mean <= MEAN_ABS_TOL, (mx, mean)
