@@ -34,7 +34,8 @@ namespace qattn {
 
 constexpr int kBM = 128;     // rows per Q tile
 constexpr int kBN = 128;     // keys per K/V tile
-constexpr int kAttnThreads = 320;
+constexpr int kAttnThreads = 384;     // 3 warpgroups: softmax 0, softmax 1, TMA + MMA
+constexpr int kAttnLaunchRegs = 168;   // 384 threads x 168 = 128 x 56 + 256 x 224 (setmaxnreg)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8 between rescales
 
 template <int D>
@@ -90,38 +91,47 @@ __device__ __forceinline__ float add_half2_f32(float acc, uint32_t h2) {
   return acc;
 }
 
-// Pass 1 over a score row: maximum of the int32 scores in each 64-key half (each half is one K
-// scale block), read from tensor memory 32 columns at a time; keys with offset above kmax are
-// excluded when MASK.  Four independent chains per half keep the ALU pipe busy.
-template <bool MASK>
-__device__ __forceinline__ void row_max(uint32_t s_tm, int kmax, int& mx0, int& mx1) {
-  int m[2][4];
-#pragma unroll
-  for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-    for (int a = 0; a < 4; ++a) m[hf][a] = INT_MIN;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint32_t r[32];
-    tmem_ld32(s_tm + c * 32, r);
-    tmem_ld_wait(r);
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int key = c * 32 + e;
-      if (!MASK || key <= kmax) m[c >> 1][e & 3] = max(m[c >> 1][e & 3], static_cast<int>(r[e]));
-    }
-  }
-  mx0 = max(max(m[0][0], m[0][1]), max(m[0][2], m[0][3]));
-  mx1 = max(max(m[1][0], m[1][1]), max(m[1][2], m[1][3]));
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
-// Pass 2: p = 2^(S_int * c - m) for the 128 keys of the row (c = c0 for keys 0-63, c1 for keys
-// 64-127); masked keys give 0.  P is packed as fp16 pairs (even key in the low half) and written
-// back into the row's first 64 tensor-memory columns, over scores already consumed: keys 0-63
-// go to columns 0-31 after columns 0-63 have been read, keys 64-127 to columns 32-63 after that.
-// Returns the fp32 sum of the fp16-rounded p.
+// One 128-key score row of one thread, held in registers as floats (exact: |S_int| < 2^24).
+// Masked keys (offset > kmax) are set to -inf.  Returns the row maximum of each 64-key half,
+// each half being one K scale block.
 template <bool MASK>
-__device__ __forceinline__ float row_exp(uint32_t s_tm, int kmax, float c0, float c1, float neg_m) {
+__device__ __forceinline__ void row_to_float_max(uint32_t (&s)[4][32], int kmax, float& mx0,
+                                                 float& mx1) {
+  float m[2][2];
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) m[hf][0] = m[hf][1] = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      float x = static_cast<float>(static_cast<int>(s[c][e]));
+      if (MASK && c * 32 + e > kmax) x = -INFINITY;
+      s[c][e] = __float_as_uint(x);
+    }
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+      float& acc = m[c >> 1][(e >> 2) & 1];
+      acc = fmax3(acc, __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
+      acc = fmax3(acc, __uint_as_float(s[c][e + 2]), __uint_as_float(s[c][e + 3]));
+    }
+  }
+  mx0 = fmaxf(m[0][0], m[0][1]);
+  mx1 = fmaxf(m[1][0], m[1][1]);
+}
+
+// p = 2^(x * c - m) for the 128 keys of the row (c = c0 for keys 0-63, c1 for keys 64-127; x
+// the float scores from row_to_float_max), masked keys give 0.  P is packed as fp16 pairs (even
+// key in the low half) and stored into the row's first 64 tensor-memory columns, aliasing the
+// scores, which are all in registers by now.  Returns the fp32 sum of the fp16-rounded p.
+template <bool MASK>
+__device__ __forceinline__ float row_exp_store(const uint32_t (&s)[4][32], float c0, float c1,
+                                               float neg_m, uint32_t s_tm) {
   float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {
@@ -130,17 +140,16 @@ __device__ __forceinline__ float row_exp(uint32_t s_tm, int kmax, float c0, floa
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       const int c = 2 * hf + q;
-      uint32_t r[32];
-      tmem_ld32(s_tm + c * 32, r);
-      tmem_ld_wait(r);
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
-        const int key = c * 32 + e;
-        float p0 = ex2_approx(fmaf(static_cast<float>(static_cast<int>(r[e])), cc, neg_m));
-        float p1 = ex2_approx(fmaf(static_cast<float>(static_cast<int>(r[e + 1])), cc, neg_m));
+        const float x0 = __uint_as_float(s[c][e]);
+        const float x1 = __uint_as_float(s[c][e + 1]);
+        float p0 = ex2_approx(fmaf(x0, cc, neg_m));
+        float p1 = ex2_approx(fmaf(x1, cc, neg_m));
         if (MASK) {
-          if (key > kmax) p0 = 0.0f;
-          if (key + 1 > kmax) p1 = 0.0f;
+          // -inf * 0 would be NaN for a zero-scale block: select instead
+          p0 = x0 == -INFINITY ? 0.0f : p0;
+          p1 = x1 == -INFINITY ? 0.0f : p1;
         }
         const uint32_t h2 = pack_half2(p0, p1);
         pk[q * 16 + (e >> 1)] = h2;
@@ -152,6 +161,13 @@ __device__ __forceinline__ float row_exp(uint32_t s_tm, int kmax, float c0, floa
     tmem_st32(s_tm + hf * 32, pk);
   }
   return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+__device__ __forceinline__ void setmaxnreg_inc224() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
+}
+__device__ __forceinline__ void setmaxnreg_dec56() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
 }
 
 template <int D, bool CAUSAL>
@@ -212,9 +228,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 8) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+  if (warp >= 8) {
+    // warpgroup 2 (TMA warp, MMA warp, two idle warps) hands registers to the softmax groups
+    setmaxnreg_dec56();
+    if (warp == 8 && lane == 0) {
+      // ---------------------------------------------------------------- TMA producer
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -232,43 +250,42 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int x = 0; x < D / 64; ++x)
           tma_load_3d(vdst + x * Cfg::kVBox, &tm_v, &bars->kv_full[s], x * 64, j * kBN, bg);
       }
-    }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 9 && lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      // Order per key tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1).  tcgen05.mma operations
+      // from one thread execute in issue order, so QK_w(j+1) may be issued right behind PV_w(j)
+      // although it overwrites the tensor-memory columns PV_w(j) reads P_w from; each softmax
+      // group then overlaps the other group's PV + QK^T on the tensor pipe.
       constexpr uint32_t idq = idesc_i8_s32(kBM, kBN);
       constexpr uint32_t idv = idesc_f16_f32_bmn(kBM, D);
       const uint32_t q_addr = smem_u32(smem + Cfg::kOffQ);
       const uint32_t k_addr = smem_u32(smem + Cfg::kOffK);
       const uint32_t v_addr = smem_u32(smem + Cfg::kOffV);
-      bool ok = mbar_wait(&bars->q_full, 0, abort);
+      auto issue_qk = [&](int w, int s) {
+        const uint32_t qa = q_addr + w * Cfg::kQTile;
+        const uint32_t ka = k_addr + s * Cfg::kKTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 32; ++kk) {
+          const uint64_t ad = smem_desc(qa + kk * 32, 16, Cfg::kSboQK, Cfg::kSwQK);
+          const uint64_t bd = smem_desc(ka + kk * 32, 16, Cfg::kSboQK, Cfg::kSwQK);
+          mma_i8_ss(tmem + w * 128, ad, bd, idq, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->s_full[w]);
+      };
+      bool ok = mbar_wait(&bars->q_full, 0, abort) && mbar_wait(&bars->kv_full[0], 0, abort);
       tc_fence_after();
+      if (ok) {
+        issue_qk(0, 0);
+        if (nw1 > 0) issue_qk(1, 0);
+      }
       for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j % ST;
-        const uint32_t u = static_cast<uint32_t>(j / ST);
-        if (!mbar_wait(&bars->kv_full[s], u & 1u, abort)) break;
-        tc_fence_after();
+        const int s1 = (j + 1) % ST;
+        bool next_ready = false;
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
-          if (!ok || j >= (w == 0 ? nw0 : nw1)) continue;
-          if (j > 0) {
-            ok = mbar_wait(&bars->pv_done[w], static_cast<uint32_t>(j - 1) & 1u, abort);
-            if (!ok) continue;
-            tc_fence_after();
-          }
-          const uint32_t qa = q_addr + w * Cfg::kQTile;
-          const uint32_t ka = k_addr + s * Cfg::kKTile;
-#pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk) {
-            const uint64_t ad = smem_desc(qa + kk * 32, 16, Cfg::kSboQK, Cfg::kSwQK);
-            const uint64_t bd = smem_desc(ka + kk * 32, 16, Cfg::kSboQK, Cfg::kSwQK);
-            mma_i8_ss(tmem + w * 128, ad, bd, idq, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&bars->s_full[w]);
-        }
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          if (!ok || j >= (w == 0 ? nw0 : nw1)) continue;
+          const int nw = w == 0 ? nw0 : nw1;
+          if (!ok || j >= nw) continue;
           ok = mbar_wait(&bars->p_full[w], static_cast<uint32_t>(j) & 1u, abort);
           if (!ok) continue;
           tc_fence_after();
@@ -280,6 +297,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                        (j > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&bars->pv_done[w]);
+          if (j + 1 < nw) {
+            if (!next_ready) {
+              ok = mbar_wait(&bars->kv_full[s1], static_cast<uint32_t>((j + 1) / ST) & 1u, abort);
+              if (!ok) continue;
+              tc_fence_after();
+              next_ready = true;
+            }
+            issue_qk(w, s1);
+          }
         }
         if (!ok) break;
         mma_commit(&bars->kv_empty[s]);
@@ -287,6 +313,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ softmax warpgroups
+    setmaxnreg_inc224();
     const int wg = warp >> 2;
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
@@ -302,27 +329,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float m_used = -INFINITY;
       float l = 0.0f;
       bool ok = true;
+      float ks0 = __ldg(ksc);
+      float ks1 = nkb > 1 ? __ldg(ksc + 1) : 0.0f;
       for (int j = 0; j < nt; ++j) {
+        // K scales of the next tile, fetched ahead of the wait
+        const float nks0 = (2 * j + 2 < nkb) ? __ldg(ksc + 2 * j + 2) : 0.0f;
+        const float nks1 = (2 * j + 3 < nkb) ? __ldg(ksc + 2 * j + 3) : 0.0f;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full[wg], static_cast<uint32_t>(j) & 1u, abort));
         if (!ok) break;
         tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(s_tm + c * 32, sr[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
         int kmax = N - 1 - j * kBN;
         if (CAUSAL && j == t) kmax = min(kmax, row);
-        const float c0 = sq * __ldg(ksc + 2 * j) * scale_log2;
-        const float c1 = (2 * j + 1 < nkb) ? sq * __ldg(ksc + 2 * j + 1) * scale_log2 : 0.0f;
-        // warp-uniform, so that every lane runs the same tcgen05.ld sequence
+        const float c0 = sq * ks0 * scale_log2;
+        const float c1 = sq * ks1 * scale_log2;
+        ks0 = nks0;
+        ks1 = nks1;
+        // warp-uniform, so that every lane runs the same tensor-memory access sequence
         const bool masked = __any_sync(0xFFFFFFFFu, kmax < kBN - 1);
-        int mx0, mx1;
-        if (masked) row_max<true>(s_tm, kmax, mx0, mx1);
-        else row_max<false>(s_tm, kmax, mx0, mx1);
+        float mx0, mx1;
+        if (masked) row_to_float_max<true>(sr, kmax, mx0, mx1);
+        else row_to_float_max<false>(sr, kmax, mx0, mx1);
         float mt = -INFINITY;
-        if (mx0 != INT_MIN) mt = static_cast<float>(mx0) * c0;
-        if (mx1 != INT_MIN) mt = fmaxf(mt, static_cast<float>(mx1) * c1);
+        if (mx0 != -INFINITY) mt = mx0 * c0;
+        if (mx1 != -INFINITY) mt = fmaxf(mt, mx1 * c1);
         const float m_new = fmaxf(m_used, mt);
         const bool need = m_new > m_used + kRescaleThreshold;
         if (j == 0) {
           m_used = m_new;
         } else if (__any_sync(0xFFFFFFFFu, need)) {
+          // O holds PV up to tile j-1 (complete: QK(j) was issued after PV(j-1)).
           float alpha = 1.0f;
           if (need) {
             alpha = ex2_approx(m_used - m_new);
@@ -340,8 +380,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         float psum;
-        if (masked) psum = row_exp<true>(s_tm, kmax, c0, c1, -m_used);
-        else psum = row_exp<false>(s_tm, kmax, c0, c1, -m_used);
+        if (masked) psum = row_exp_store<true>(sr, c0, c1, -m_used, s_tm);
+        else psum = row_exp_store<false>(sr, c0, c1, -m_used, s_tm);
         l += psum;
         tmem_st_wait();
         tc_fence_before();

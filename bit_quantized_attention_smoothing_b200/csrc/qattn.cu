@@ -165,6 +165,15 @@ qattn_status run_attn(const int8_t* q_i8, const float* q_scale, const int8_t* k_
     return QATTN_ERR_CUDA;
   using Cfg = AttnCfg<D>;
   auto kern = attn_fwd_kernel<D, CAUSAL>;
+  // The kernel moves registers between its warpgroups with setmaxnreg; the split adds up only if
+  // the launch allocates exactly kAttnLaunchRegs per thread, so never launch it otherwise.
+  static int regs_checked = 0;
+  if (regs_checked == 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return QATTN_ERR_CUDA;
+    regs_checked = fa.numRegs == kAttnLaunchRegs ? 1 : -1;
+  }
+  if (regs_checked != 1) return QATTN_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) !=
       cudaSuccess)
     return QATTN_ERR_CUDA;

@@ -2,9 +2,10 @@
 
 * smoothing + quantization (int8 codes, block scales, channel means): bit-exact;
 * int32 score tiles from the tcgen05 kind::i8 path: bit-exact;
-* forward output: max-abs <= 2e-3 and mean-abs <= 2e-4 against the oracle's unrounded float64
+* forward output: mean-abs <= 2e-4 and max-abs <= 2e-3 against the oracle's unrounded float64
   output (the oracle rounds nothing after the int32 product; the GPU rounds P to fp16, accumulates
-  in fp32, uses a hardware exp2 and rounds O to fp16).
+  in fp32, uses a hardware exp2 and rounds O to fp16); where |O| >= 4 the fp16 output grid's own
+  half-spacing (1.95e-3) is added to the 2e-3 budget (tests/conftest.py, check_output).
 
 Small cases compare every output element and cover ragged N (partial Q tile, partial K block,
 odd tile counts), N=1, GQA, causal and non-causal, d=64 and d=128.  The five named workloads run at
@@ -16,7 +17,7 @@ import pytest
 import torch
 
 from bit_quantized_attention_smoothing_b200.workloads import ORDER, WORKLOADS, make_inputs, sample_rows
-from conftest import MAX_ABS_TOL, MEAN_ABS_TOL, np16, out_errors
+from conftest import check_output, np16
 
 pytestmark = pytest.mark.gpu
 
@@ -93,9 +94,8 @@ def test_forward_small_all_rows(lib, oracle, name, over):
     out = lib.qattn_forward(q, k, v, causal=w.causal)
     assert lib.qattn_check_device_status() == 0
     ref, _ = oracle.forward(np16(q), np16(k), np16(v), w.B, w.H, w.Hkv, w.N, w.d, w.causal)
-    got = out.float().cpu().numpy().reshape(-1, w.d)
-    mx, mean = out_errors(got, ref)
-    assert mx <= MAX_ABS_TOL and mean <= MEAN_ABS_TOL, (mx, mean)
+    ok, msg = check_output(out.float().cpu().numpy().reshape(-1, w.d), ref)
+    assert ok, msg
 
 
 @pytest.mark.parametrize("name,over", SMALL[:6], ids=SMALL_IDS[:6])
@@ -109,8 +109,8 @@ def test_attention_on_oracle_codes(lib, oracle, name, over):
                                    causal=w.causal)
     ref = oracle.attention_quantized(ref_sq["q_i8"], ref_sq["q_scale"], ref_sq["k_i8"],
                                      ref_sq["k_scale"], np16(v), w.B, w.H, w.Hkv, w.N, w.d, w.causal)
-    mx, mean = out_errors(out.float().cpu().numpy().reshape(-1, w.d), ref)
-    assert mx <= MAX_ABS_TOL and mean <= MEAN_ABS_TOL, (mx, mean)
+    ok, msg = check_output(out.float().cpu().numpy().reshape(-1, w.d), ref)
+    assert ok, msg
 
 
 def test_forward_variants_agree(lib):
@@ -171,5 +171,6 @@ def test_full_size_workload(lib, oracle, name):
     ref = oracle.attention_quantized(ref_sq["q_i8"], ref_sq["q_scale"], ref_sq["k_i8"],
                                      ref_sq["k_scale"], np16(v), w.B, w.H, w.Hkv, w.N, w.d,
                                      w.causal, rows=rows)
-    mx, mean = out_errors(_rows_of(out, w, rows), ref)
-    assert mx <= MAX_ABS_TOL and mean <= MEAN_ABS_TOL, (mx, mean)
+    ok, msg = check_output(_rows_of(out, w, rows), ref)
+    print(name, msg)
+    assert ok, msg
