@@ -6,15 +6,17 @@
 // warp-level mma on an RTX4090; this one is built for Blackwell instead:
 //
 //  * one CTA owns two 128-row Q tiles of one (batch, head) and streams 128-key K/V tiles;
-//  * warp 8 (TMA): loads both Q tiles once, then K (int8) and V (fp16) tiles into a STAGES-deep
+//  * warp 16 (TMA): loads both Q tiles once, then K (int8) and V (fp16) tiles into a STAGES-deep
 //    shared-memory ring (128-byte / 64-byte swizzled tiles, mbarrier transaction counts);
-//  * warp 9 (MMA, one thread): S_w = Q_w K^T as tcgen05.mma kind::i8 (M=128, N=128, K=32 per
+//  * warp 17 (MMA, one thread): S_w = Q_w K^T as tcgen05.mma kind::i8 (M=128, N=128, K=32 per
 //    instruction) into tensor memory, then O_w += P_w V as tcgen05.mma kind::f16 with P read
 //    from tensor memory (M=128, N=d, K=16), fp32 accumulator in tensor memory;
-//  * warps 0-3 and 4-7 (softmax warpgroups, one per Q tile, thread = row): tcgen05.ld of the int32
-//    scores, dequantization with the two block scales, running max / sum in registers, exp2,
-//    P written back as fp16 into the same tensor-memory columns (aliasing S), lazy rescaling of
-//    O only when the running max grows by more than 2^8;
+//  * warps 0-15 (softmax, four warpgroups, two per Q tile): each score row is shared by two
+//    threads, one per 64-key half (= one K scale block); tcgen05.ld of the int32 scores,
+//    dequantization with the block scales, half-row maxima swapped through shared memory,
+//    running max / sum in registers, exp2, P written back as fp16 into the same tensor-memory
+//    columns (aliasing S), lazy rescaling of O only when the running max grows by more than 2^8,
+//    P scaled into the top of the fp16 range;
 //  * while one warpgroup runs its softmax the tensor cores work on the other Q tile;
 //  * causal: key tiles above the diagonal are never loaded or multiplied; the diagonal tile is
 //    masked in registers; CTAs are launched heaviest-first;
@@ -34,9 +36,15 @@ namespace qattn {
 
 constexpr int kBM = 128;     // rows per Q tile
 constexpr int kBN = 128;     // keys per K/V tile
-constexpr int kAttnThreads = 384;     // 3 warpgroups: softmax 0, softmax 1, TMA + MMA
-constexpr int kAttnLaunchRegs = 168;   // 384 threads x 168 = 128 x 56 + 256 x 224 (setmaxnreg)
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8 between rescales
+constexpr int kAttnThreads = 640;     // 5 warpgroups: 4 softmax (2 per Q tile), TMA + MMA
+constexpr int kAttnLaunchRegs = 96;    // 640 x 96 = 512 x 104 (softmax) + 128 x 64 (setmaxnreg)
+constexpr int kSoftmaxThreads = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only when the max grows more
+// P = 2^(x - m + kPOffset): with the lazy max above, P <= 2^15 < 65504 (fp16 max), and keys down to
+// about 2^-(24 + kPOffset) of the row maximum still reach the fp16 P instead of underflowing.  At
+// 131072 keys per row, P normalised to 1 loses enough weight in fp16 subnormals to cost ~4e-3 of
+// output accuracy; the offset cancels in O / l.
+constexpr float kPOffset = 7.0f;
 
 template <int D>
 struct AttnCfg {
@@ -48,7 +56,7 @@ struct AttnCfg {
   static constexpr int kOffK = 2 * kQTile;
   static constexpr int kOffV = kOffK + kStages * kKTile;
   static constexpr int kOffBar = kOffV + kStages * kVTile;
-  static constexpr int kBarBytes = 256;
+  static constexpr int kBarBytes = 256 + 4096;  // barriers + half-row max / sum exchange
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
   // K-major int8 operands: rows of D bytes, 8-row swizzle atoms.
   static constexpr uint32_t kSwQK = D == 128 ? kSwizzle128B : kSwizzle64B;
@@ -57,7 +65,7 @@ struct AttnCfg {
   static constexpr uint32_t kVBox = kBN * 128;  // bytes of one 64-column box
 };
 
-struct __align__(8) AttnBars {
+struct __align__(16) AttnBars {
   uint64_t q_full;
   uint64_t kv_full[6];
   uint64_t kv_empty[6];
@@ -66,7 +74,12 @@ struct __align__(8) AttnBars {
   uint64_t pv_done[2];
   uint32_t tmem_base;
   int abort;
+  uint8_t pad[256 - 8 * 19 - 8];
+  // [step parity][Q tile][key half][row]: the two threads of a score row swap half-row maxima
+  // (and, at the end, half-row sums) here
+  float xch[2][2][2][128];
 };
+static_assert(sizeof(AttnBars) <= 256 + 4096, "barrier block");
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -97,77 +110,81 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// One 128-key score row of one thread, held in registers as floats (exact: |S_int| < 2^24).
-// Masked keys (offset > kmax) are set to -inf.  Returns the row maximum of each 64-key half,
-// each half being one K scale block.
+// (d0, d1) = (a0 * b + c, a1 * b + c) as one packed sm_100 fp32x2 FMA (each lane rounds once).
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\tmov.b64 rc, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// One thread's 64 scores of a row (one K scale block), in registers as floats (exact:
+// |S_int| < 2^24); keys with offset above lim are set to -inf.  Returns their maximum.
 template <bool MASK>
-__device__ __forceinline__ void row_to_float_max(uint32_t (&s)[4][32], int kmax, float& mx0,
-                                                 float& mx1) {
-  float m[2][2];
+__device__ __forceinline__ float half_row_to_float_max(uint32_t (&s)[2][32], int lim) {
+  float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-  for (int hf = 0; hf < 2; ++hf) m[hf][0] = m[hf][1] = -INFINITY;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int c = 0; c < 2; ++c) {
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       float x = static_cast<float>(static_cast<int>(s[c][e]));
-      if (MASK && c * 32 + e > kmax) x = -INFINITY;
+      if (MASK && c * 32 + e > lim) x = -INFINITY;
       s[c][e] = __float_as_uint(x);
     }
 #pragma unroll
     for (int e = 0; e < 32; e += 4) {
-      float& acc = m[c >> 1][(e >> 2) & 1];
-      acc = fmax3(acc, __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
-      acc = fmax3(acc, __uint_as_float(s[c][e + 2]), __uint_as_float(s[c][e + 3]));
+      m0 = fmax3(m0, __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
+      m1 = fmax3(m1, __uint_as_float(s[c][e + 2]), __uint_as_float(s[c][e + 3]));
     }
   }
-  mx0 = fmaxf(m[0][0], m[0][1]);
-  mx1 = fmaxf(m[1][0], m[1][1]);
+  return fmaxf(m0, m1);
 }
 
-// p = 2^(x * c - m) for the 128 keys of the row (c = c0 for keys 0-63, c1 for keys 64-127; x
-// the float scores from row_to_float_max), masked keys give 0.  P is packed as fp16 pairs (even
-// key in the low half) and stored into the row's first 64 tensor-memory columns, aliasing the
-// scores, which are all in registers by now.  Returns the fp32 sum of the fp16-rounded p.
+// p = 2^(x * c - m) for the thread's 64 keys, masked keys (x = -inf) give 0.  P is packed as
+// fp16 pairs (even key in the low half) and stored into 32 tensor-memory columns at p_tm.
+// Returns the fp32 sum of the fp16-rounded p.
 template <bool MASK>
-__device__ __forceinline__ float row_exp_store(const uint32_t (&s)[4][32], float c0, float c1,
-                                               float neg_m, uint32_t s_tm) {
-  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+__device__ __forceinline__ float half_row_exp_store(const uint32_t (&s)[2][32], float c,
+                                                    float neg_m, uint32_t p_tm) {
+  float acc0 = 0.0f, acc1 = 0.0f;
 #pragma unroll
-  for (int hf = 0; hf < 2; ++hf) {
-    const float cc = hf == 0 ? c0 : c1;
-    uint32_t pk[32];
+  for (int k = 0; k < 2; ++k) {
+    uint32_t pk[16];
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int c = 2 * hf + q;
-#pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        const float x0 = __uint_as_float(s[c][e]);
-        const float x1 = __uint_as_float(s[c][e + 1]);
-        float p0 = ex2_approx(fmaf(x0, cc, neg_m));
-        float p1 = ex2_approx(fmaf(x1, cc, neg_m));
-        if (MASK) {
-          // -inf * 0 would be NaN for a zero-scale block: select instead
-          p0 = x0 == -INFINITY ? 0.0f : p0;
-          p1 = x1 == -INFINITY ? 0.0f : p1;
-        }
-        const uint32_t h2 = pack_half2(p0, p1);
-        pk[q * 16 + (e >> 1)] = h2;
-        // the row sum takes the fp16-rounded P that the P V product uses, so that O / l is a
-        // weighted mean of V with exactly those weights
-        acc[(e >> 1) & 3] = add_half2_f32(acc[(e >> 1) & 3], h2);
+    for (int e = 0; e < 32; e += 2) {
+      const float x0 = __uint_as_float(s[k][e]);
+      const float x1 = __uint_as_float(s[k][e + 1]);
+      float y0, y1;
+      ffma2(y0, y1, x0, x1, c, neg_m);
+      float p0 = ex2_approx(y0);
+      float p1 = ex2_approx(y1);
+      if (MASK) {
+        // -inf * 0 would be NaN for a zero-scale block: select instead
+        p0 = x0 == -INFINITY ? 0.0f : p0;
+        p1 = x1 == -INFINITY ? 0.0f : p1;
       }
+      const uint32_t h2 = pack_half2(p0, p1);
+      pk[e >> 1] = h2;
+      // the row sum takes the fp16-rounded P that the P V product uses, so that O / l is a
+      // weighted mean of V with exactly those weights
+      if ((e >> 1) & 1) acc1 = add_half2_f32(acc1, h2);
+      else acc0 = add_half2_f32(acc0, h2);
     }
-    tmem_st32(s_tm + hf * 32, pk);
+    tmem_st16(p_tm + k * 16, pk);
   }
-  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  return acc0 + acc1;
 }
 
-__device__ __forceinline__ void setmaxnreg_inc224() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
+__device__ __forceinline__ void setmaxnreg_inc104() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 104;" ::: "memory");
 }
-__device__ __forceinline__ void setmaxnreg_dec56() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+__device__ __forceinline__ void setmaxnreg_dec64() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
 }
 
 template <int D, bool CAUSAL>
@@ -178,6 +195,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     int Hkv, int N, float scale_log2) {
   using Cfg = AttnCfg<D>;
   constexpr int ST = Cfg::kStages;
+  constexpr int kTmaWarp = kSoftmaxThreads / 32;  // warp 16
+  constexpr int kMmaWarp = kTmaWarp + 1;          // warp 17
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -213,13 +232,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&bars->s_full[w], 1);
-      mbar_init(&bars->p_full[w], 128);
+      mbar_init(&bars->p_full[w], 256);
       mbar_init(&bars->pv_done[w], 1);
     }
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
@@ -228,10 +247,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp >= 8) {
-    // warpgroup 2 (TMA warp, MMA warp, two idle warps) hands registers to the softmax groups
-    setmaxnreg_dec56();
-    if (warp == 8 && lane == 0) {
+  if (warp >= kTmaWarp) {
+    // warpgroup 4 (TMA warp, MMA warp, two idle warps) hands registers to the softmax groups
+    setmaxnreg_dec64();
+    if (warp == kTmaWarp && lane == 0) {
       // ---------------------------------------------------------------- TMA producer
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -250,12 +269,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int x = 0; x < D / 64; ++x)
           tma_load_3d(vdst + x * Cfg::kVBox, &tm_v, &bars->kv_full[s], x * 64, j * kBN, bg);
       }
-    } else if (warp == 9 && lane == 0) {
+    } else if (warp == kMmaWarp && lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
       // Order per key tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1).  tcgen05.mma operations
       // from one thread execute in issue order, so QK_w(j+1) may be issued right behind PV_w(j)
-      // although it overwrites the tensor-memory columns PV_w(j) reads P_w from; each softmax
-      // group then overlaps the other group's PV + QK^T on the tensor pipe.
+      // although it overwrites the tensor-memory columns PV_w(j) reads P_w from; the softmax of
+      // one Q tile then overlaps the other tile's PV + QK^T on the tensor pipe.
       constexpr uint32_t idq = idesc_i8_s32(kBM, kBN);
       constexpr uint32_t idv = idesc_f16_f32_bmn(kBM, D);
       const uint32_t q_addr = smem_u32(smem + Cfg::kOffQ);
@@ -313,93 +332,101 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ softmax warpgroups
-    setmaxnreg_inc224();
-    const int wg = warp >> 2;
-    const int wq = warp & 3;
-    const int row = wq * 32 + lane;
-    const int nt = wg == 0 ? nw0 : nw1;
+    // warp = 8 * tile + 4 * half + lane group: two threads share each score row, one per
+    // 64-key half (= one K scale block); they swap half-row maxima through shared memory.
+    setmaxnreg_inc104();
+    const int wt = warp >> 3;
+    const int half = (warp >> 2) & 1;
+    const int lg = warp & 3;
+    const int row = lg * 32 + lane;
+    const int pair_bar = 1 + wt * 4 + lg;  // named barrier of the two warps sharing these rows
+    const int nt = wt == 0 ? nw0 : nw1;
     if (nt > 0) {
-      const int t = wg == 0 ? tq0 : tq1;
+      const int t = wt == 0 ? tq0 : tq1;
       const int qrow = t * kBM + row;
       const float sq = __ldg(q_scale + static_cast<size_t>(bh) * nqt + t);
       const float* ksc = k_scale + static_cast<size_t>(bg) * nkb;
-      const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-      const uint32_t s_tm = tmem + lane_off + wg * 128;
-      const uint32_t o_tm = tmem + lane_off + 256 + wg * D;
+      const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
+      const uint32_t s_tm = tmem + lane_off + wt * 128 + half * 64;
+      const uint32_t p_tm = tmem + lane_off + wt * 128 + half * 32;
+      const uint32_t o_tm = tmem + lane_off + 256 + wt * D + half * (D / 2);
       float m_used = -INFINITY;
       float l = 0.0f;
       bool ok = true;
-      float ks0 = __ldg(ksc);
-      float ks1 = nkb > 1 ? __ldg(ksc + 1) : 0.0f;
+      float ks = (half < nkb) ? __ldg(ksc + half) : 0.0f;
       for (int j = 0; j < nt; ++j) {
-        // K scales of the next tile, fetched ahead of the wait
-        const float nks0 = (2 * j + 2 < nkb) ? __ldg(ksc + 2 * j + 2) : 0.0f;
-        const float nks1 = (2 * j + 3 < nkb) ? __ldg(ksc + 2 * j + 3) : 0.0f;
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full[wg], static_cast<uint32_t>(j) & 1u, abort));
+        const int kb_next = 2 * j + 2 + half;
+        const float ks_next = kb_next < nkb ? __ldg(ksc + kb_next) : 0.0f;
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full[wt], static_cast<uint32_t>(j) & 1u, abort));
         if (!ok) break;
         tc_fence_after();
-        uint32_t sr[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(s_tm + c * 32, sr[c]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
-        int kmax = N - 1 - j * kBN;
-        if (CAUSAL && j == t) kmax = min(kmax, row);
-        const float c0 = sq * ks0 * scale_log2;
-        const float c1 = sq * ks1 * scale_log2;
-        ks0 = nks0;
-        ks1 = nks1;
+        uint32_t sr[2][32];
+        tmem_ld32(s_tm, sr[0]);
+        tmem_ld32(s_tm + 32, sr[1]);
+        tmem_ld_wait(sr[0]);
+        tmem_ld_wait(sr[1]);
+        int lim = N - 1 - j * kBN - half * 64;
+        if (CAUSAL && j == t) lim = min(lim, row - half * 64);
+        const float c = sq * ks * scale_log2;
+        ks = ks_next;
         // warp-uniform, so that every lane runs the same tensor-memory access sequence
-        const bool masked = __any_sync(0xFFFFFFFFu, kmax < kBN - 1);
-        float mx0, mx1;
-        if (masked) row_to_float_max<true>(sr, kmax, mx0, mx1);
-        else row_to_float_max<false>(sr, kmax, mx0, mx1);
-        float mt = -INFINITY;
-        if (mx0 != -INFINITY) mt = mx0 * c0;
-        if (mx1 != -INFINITY) mt = fmaxf(mt, mx1 * c1);
+        const bool masked = __any_sync(0xFFFFFFFFu, lim < 63);
+        float hm = masked ? half_row_to_float_max<true>(sr, lim) : half_row_to_float_max<false>(sr, lim);
+        hm = hm == -INFINITY ? -INFINITY : hm * c;
+        // swap half-row maxima; the barrier also orders this thread's score reads before the
+        // partner's P writes, which land on columns 32-63 of the row
+        bars->xch[j & 1][wt][half][row] = hm;
+        tc_fence_before();
+        named_bar_sync(pair_bar, 64);
+        tc_fence_after();
+        const float mt = fmaxf(hm, bars->xch[j & 1][wt][half ^ 1][row]);
         const float m_new = fmaxf(m_used, mt);
         const bool need = m_new > m_used + kRescaleThreshold;
-        if (j == 0) {
+        float alpha = 1.0f;
+        if (need) {
+          alpha = j == 0 ? 0.0f : ex2_approx(m_used - m_new);
           m_used = m_new;
-        } else if (__any_sync(0xFFFFFFFFu, need)) {
-          // O holds PV up to tile j-1 (complete: QK(j) was issued after PV(j-1)).
-          float alpha = 1.0f;
-          if (need) {
-            alpha = ex2_approx(m_used - m_new);
-            m_used = m_new;
-            l *= alpha;
-          }
+          l *= alpha;
+        }
+        const float neg_m = kPOffset - m_used;
+        const float psum = masked ? half_row_exp_store<true>(sr, c, neg_m, p_tm)
+                                  : half_row_exp_store<false>(sr, c, neg_m, p_tm);
+        l += psum;
+        if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
+          // O holds PV up to tile j-1 (complete: QK(j) was issued after PV(j-1)), and PV(j)
+          // waits for this group's arrive below.  Both threads of a row take the same decision;
+          // each rescales its half of the O row.
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(o_tm + c * 32, o);
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[16];
+            tmem_ld16(o_tm + cc * 16, o);
             tmem_ld_wait(o);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(o_tm + c * 32, o);
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st16(o_tm + cc * 16, o);
           }
         }
-        float psum;
-        if (masked) psum = row_exp_store<true>(sr, c0, c1, -m_used, s_tm);
-        else psum = row_exp_store<false>(sr, c0, c1, -m_used, s_tm);
-        l += psum;
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bars->p_full[wg]);
+        mbar_arrive(&bars->p_full[wt]);
       }
-      if (ok) ok = mbar_wait(&bars->pv_done[wg], static_cast<uint32_t>(nt - 1) & 1u, abort);
+      if (ok) ok = mbar_wait(&bars->pv_done[wt], static_cast<uint32_t>(nt - 1) & 1u, abort);
       ok = __all_sync(0xFFFFFFFFu, ok);
+      // total row sum from the two halves (parity slot nt&1 is free: last used at step nt-2)
+      bars->xch[nt & 1][wt][half][row] = l;
+      named_bar_sync(pair_bar, 64);
+      l += bars->xch[nt & 1][wt][half ^ 1][row];
       tc_fence_after();
       if (ok) {
         const float inv_l = 1.0f / l;
-        __half* orow = out + (static_cast<size_t>(bh) * N + qrow) * D;
+        __half* orow = out + (static_cast<size_t>(bh) * N + qrow) * D + half * (D / 2);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int cc = 0; cc < D / 64; ++cc) {
           uint32_t o[32];
-          tmem_ld32(o_tm + c * 32, o);
+          tmem_ld32(o_tm + cc * 32, o);
           tmem_ld_wait(o);
           if (qrow < N) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+            uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               uint4 pkt;
@@ -417,7 +444,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
