@@ -6,20 +6,20 @@
 // warp-level mma on an RTX4090; this one is built for Blackwell instead:
 //
 //  * one CTA owns two 128-row Q tiles of one (batch, head) and streams 128-key K/V tiles;
-//  * warp 16 (TMA): loads both Q tiles once, then K (int8) and V (fp16) tiles into a STAGES-deep
+//  * warp 8 (TMA): loads both Q tiles once, then K (int8) and V (fp16) tiles into a STAGES-deep
 //    shared-memory ring (128-byte / 64-byte swizzled tiles, mbarrier transaction counts);
-//  * warp 17 (MMA, one thread): S_w = Q_w K^T as tcgen05.mma kind::i8 (M=128, N=128, K=32 per
+//  * warp 9 (MMA, one thread): S_w = Q_w K^T as tcgen05.mma kind::i8 (M=128, N=128, K=32 per
 //    instruction) into tensor memory, then O_w += P_w V as tcgen05.mma kind::f16 with P read
-//    from tensor memory (M=128, N=d, K=16), fp32 accumulator in tensor memory;
-//  * warps 0-15 (softmax, four warpgroups, two per Q tile): each score row is shared by two
-//    threads, one per 64-key half (= one K scale block); tcgen05.ld of the int32 scores,
-//    dequantization with the block scales, half-row maxima swapped through shared memory,
-//    running max / sum in registers, exp2, P written back as fp16 into the same tensor-memory
-//    columns (aliasing S), lazy rescaling of O only when the running max grows by more than 2^8,
-//    P scaled into the top of the fp16 range;
-//  * while one warpgroup runs its softmax the tensor cores work on the other Q tile;
+//    from tensor memory (M=128, N=d, K=16), fp32 accumulator in tensor memory; issue order
+//    PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1) so that one Q tile's softmax overlaps the other's MMAs;
+//  * warps 0-3 and 4-7 (softmax, one warpgroup per Q tile, thread = score row, setmaxnreg 224):
+//    one tcgen05.ld of the row's 128 int32 scores, exact int->float, row maximum per 64-key K
+//    scale block (3-input max), dequantization and exp2 argument with packed fp32x2 FMAs, MUFU
+//    ex2, P packed to fp16 and written back over the scores' tensor-memory columns, row sum of the
+//    fp16-rounded P; lazy rescaling of O only when the running max grows by more than 2^8; P
+//    scaled into the top of the fp16 range;
 //  * causal: key tiles above the diagonal are never loaded or multiplied; the diagonal tile is
-//    masked in registers; CTAs are launched heaviest-first;
+//    masked in registers (a compile-time-specialised path); CTAs are launched heaviest-first;
 //  * grouped-query attention: query head h reads kv head h / (H / Hkv); CTAs of the heads that
 //    share a kv head are adjacent in launch order so their K/V tiles are reused from L2.
 //
@@ -36,9 +36,9 @@ namespace qattn {
 
 constexpr int kBM = 128;     // rows per Q tile
 constexpr int kBN = 128;     // keys per K/V tile
-constexpr int kAttnThreads = 640;     // 5 warpgroups: 4 softmax (2 per Q tile), TMA + MMA
-constexpr int kAttnLaunchRegs = 96;    // 640 x 96 = 512 x 104 (softmax) + 128 x 64 (setmaxnreg)
-constexpr int kSoftmaxThreads = 512;
+constexpr int kAttnThreads = 384;     // 3 warpgroups: softmax Q tile 0, softmax Q tile 1, TMA + MMA
+constexpr int kAttnLaunchRegs = 168;   // 384 x 168 = 256 x 224 (softmax) + 128 x 56 (setmaxnreg)
+constexpr int kSoftmaxThreads = 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only when the max grows more
 // P = 2^(x - m + kPOffset): with the lazy max above, P <= 2^15 < 65504 (fp16 max), and keys down to
 // about 2^-(24 + kPOffset) of the row maximum still reach the fp16 P instead of underflowing.  At
@@ -56,7 +56,7 @@ struct AttnCfg {
   static constexpr int kOffK = 2 * kQTile;
   static constexpr int kOffV = kOffK + kStages * kKTile;
   static constexpr int kOffBar = kOffV + kStages * kVTile;
-  static constexpr int kBarBytes = 256 + 4096;  // barriers + half-row max / sum exchange
+  static constexpr int kBarBytes = 256;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
   // K-major int8 operands: rows of D bytes, 8-row swizzle atoms.
   static constexpr uint32_t kSwQK = D == 128 ? kSwizzle128B : kSwizzle64B;
@@ -74,12 +74,8 @@ struct __align__(16) AttnBars {
   uint64_t pv_done[2];
   uint32_t tmem_base;
   int abort;
-  uint8_t pad[256 - 8 * 19 - 8];
-  // [step parity][Q tile][key half][row]: the two threads of a score row swap half-row maxima
-  // (and, at the end, half-row sums) here
-  float xch[2][2][2][128];
 };
-static_assert(sizeof(AttnBars) <= 256 + 4096, "barrier block");
+static_assert(sizeof(AttnBars) <= 256, "barrier block");
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -119,72 +115,143 @@ __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, 
       : "f"(a0), "f"(a1), "f"(b), "f"(c));
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+// (d0, d1) = (a0 + b0, a1 + b1) and (a0 * b0 + c0, a1 * b1 + c1) as packed sm_100 fp32x2 ops.
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void ffma2v(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                       float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
 
-// One thread's 64 scores of a row (one K scale block), in registers as floats (exact:
-// |S_int| < 2^24); keys with offset above lim are set to -inf.  Returns their maximum.
+// 2^f on [-1/2, 1/2]: degree-4 minimax polynomial (relative error 2.6e-6), coefficients from
+// gen_exp2_poly.py (Chebyshev start, Remez exchange).
+constexpr float kExpC0 = 0.9999992847442627f;
+constexpr float kExpC1 = 0.6931217908859253f;
+constexpr float kExpC2 = 0.240247443318367f;
+constexpr float kExpC3 = 0.05591785907745361f;
+constexpr float kExpC4 = 0.009570102207362652f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + M rounds x to an integer
+
+// 2^y for two values on the FMA pipe instead of MUFU: n = round(y) through the 1.5 * 2^23 add,
+// f = y - n (exact), 2^y = p(f) * 2^n with the power of two added to the exponent bits.  y is
+// clamped at -125 so the exponent stays normal; the results only feed fp16 P, where anything
+// below 2^-24 is zero anyway.
+__device__ __forceinline__ void exp2_poly2(float y0, float y1, float& r0, float& r1) {
+  y0 = fmaxf(y0, -125.0f);
+  y1 = fmaxf(y1, -125.0f);
+  float t0, t1, n0, n1, f0, f1, p0, p1;
+  fadd2(t0, t1, y0, y1, kRoundMagic, kRoundMagic);
+  fadd2(n0, n1, t0, t1, -kRoundMagic, -kRoundMagic);
+  ffma2v(f0, f1, n0, n1, -1.0f, -1.0f, y0, y1);
+  ffma2v(p0, p1, f0, f1, kExpC4, kExpC4, kExpC3, kExpC3);
+  ffma2v(p0, p1, p0, p1, f0, f1, kExpC2, kExpC2);
+  ffma2v(p0, p1, p0, p1, f0, f1, kExpC1, kExpC1);
+  ffma2v(p0, p1, p0, p1, f0, f1, kExpC0, kExpC0);
+  // the low 9 bits of t's pattern hold n (two's complement), so t << 23 is n << 23
+  r0 = __uint_as_float((__float_as_uint(t0) << 23) + __float_as_uint(p0));
+  r1 = __uint_as_float((__float_as_uint(t1) << 23) + __float_as_uint(p1));
+}
+
+__device__ __forceinline__ float scaled_max(float m, float c) {
+  return m == -INFINITY ? -INFINITY : m * c;
+}
+
+// Score-register groups i (0-15) for which kExp2EmulateMask has bit i set go through exp2_poly2
+// on the FMA pipe; the rest use MUFU ex2.  Measured on B200 (llama8b_32k): moving 1/8, 1/4 or 3/8
+// of the exponentials to the FMA pipe made the kernel 3 %, 7 % and 13 % slower, so none is moved.
+constexpr uint32_t kExp2EmulateMask = 0x0000;
+__device__ __forceinline__ constexpr bool emulated_pair(int i) { return (kExp2EmulateMask >> i) & 1; }
+
+// One 128-key step of the softmax for the thread's score row: int32 -> float (exact, |S| < 2^24),
+// masked keys (MASK; key offset above lim) -> -inf, row maximum per 64-key K scale block, lazy
+// update of the running max m (alpha = rescale factor, need = O must be rescaled), then
+// P = 2^(x * c - m + offset) packed as fp16 pairs (even key in the low half) and stored over the
+// row's first 64 TMEM columns, and the row sum of the fp16-rounded P.  MASK is a compile-time
+// switch so the unmasked steps carry no per-element tests.
 template <bool MASK>
-__device__ __forceinline__ float half_row_to_float_max(uint32_t (&s)[2][32], int lim) {
-  float m0 = -INFINITY, m1 = -INFINITY;
+__device__ __forceinline__ void softmax_row(uint32_t (&sr)[4][32], int lim, float c0, float c1,
+                                            bool first, float& m, float& l, float& alpha,
+                                            bool& need, uint32_t s_tm) {
+  float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
+  for (int c = 0; c < 4; ++c) {
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
-      float x = static_cast<float>(static_cast<int>(s[c][e]));
+      float x = static_cast<float>(static_cast<int>(sr[c][e]));
       if (MASK && c * 32 + e > lim) x = -INFINITY;
-      s[c][e] = __float_as_uint(x);
+      sr[c][e] = __float_as_uint(x);
     }
 #pragma unroll
     for (int e = 0; e < 32; e += 4) {
-      m0 = fmax3(m0, __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
-      m1 = fmax3(m1, __uint_as_float(s[c][e + 2]), __uint_as_float(s[c][e + 3]));
+      float& a = (c < 2) ? ((e & 4) ? mx1 : mx0) : ((e & 4) ? mx3 : mx2);
+      a = fmax3(a, __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+      a = fmax3(a, __uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3]));
     }
   }
-  return fmaxf(m0, m1);
-}
-
-// p = 2^(x * c - m) for the thread's 64 keys, masked keys (x = -inf) give 0.  P is packed as
-// fp16 pairs (even key in the low half) and stored into 32 tensor-memory columns at p_tm.
-// Returns the fp32 sum of the fp16-rounded p.
-template <bool MASK>
-__device__ __forceinline__ float half_row_exp_store(const uint32_t (&s)[2][32], float c,
-                                                    float neg_m, uint32_t p_tm) {
+  const float t = fmaxf(scaled_max(fmaxf(mx0, mx1), c0), scaled_max(fmaxf(mx2, mx3), c1));
+  const float mn = fmaxf(m, t);
+  need = mn > m + kRescaleThreshold;
+  alpha = 1.0f;
+  if (need) {
+    alpha = first ? 0.0f : ex2_approx(m - mn);
+    m = mn;
+    l *= alpha;
+  }
+  const float g = kPOffset - m;
   float acc0 = 0.0f, acc1 = 0.0f;
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    uint32_t pk[16];
+  for (int hf = 0; hf < 2; ++hf) {
+    const float c = hf == 0 ? c0 : c1;
+    uint32_t pk[32];
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-      const float x0 = __uint_as_float(s[k][e]);
-      const float x1 = __uint_as_float(s[k][e + 1]);
-      float y0, y1;
-      ffma2(y0, y1, x0, x1, c, neg_m);
-      float p0 = ex2_approx(y0);
-      float p1 = ex2_approx(y1);
-      if (MASK) {
-        // -inf * 0 would be NaN for a zero-scale block: select instead
-        p0 = x0 == -INFINITY ? 0.0f : p0;
-        p1 = x1 == -INFINITY ? 0.0f : p1;
+    for (int q = 0; q < 2; ++q) {
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        const int i = (2 * hf + q) * 16 + (e >> 1);  // pair index 0..63
+        const float x0 = __uint_as_float(sr[2 * hf + q][e]);
+        const float x1 = __uint_as_float(sr[2 * hf + q][e + 1]);
+        float y0, y1, p0, p1;
+        ffma2(y0, y1, x0, x1, c, g);
+        if (emulated_pair(i & 15)) {
+          exp2_poly2(y0, y1, p0, p1);
+        } else {
+          p0 = ex2_approx(y0);
+          p1 = ex2_approx(y1);
+        }
+        if (MASK) {
+          // -inf * 0 would be NaN for a zero-scale block: select instead
+          if (x0 == -INFINITY) p0 = 0.0f;
+          if (x1 == -INFINITY) p1 = 0.0f;
+        }
+        const uint32_t h2 = pack_half2(p0, p1);
+        pk[q * 16 + (e >> 1)] = h2;
+        // the row sum takes the fp16-rounded P that the P V product uses, so that O / l is a
+        // weighted mean of V with exactly those weights
+        if (e & 2) acc1 = add_half2_f32(acc1, h2);
+        else acc0 = add_half2_f32(acc0, h2);
       }
-      const uint32_t h2 = pack_half2(p0, p1);
-      pk[e >> 1] = h2;
-      // the row sum takes the fp16-rounded P that the P V product uses, so that O / l is a
-      // weighted mean of V with exactly those weights
-      if ((e >> 1) & 1) acc1 = add_half2_f32(acc1, h2);
-      else acc0 = add_half2_f32(acc0, h2);
     }
-    tmem_st16(p_tm + k * 16, pk);
+    // keys 64 * hf .. 64 * hf + 63 -> P columns 32 * hf .. 32 * hf + 31; all scores are in
+    // registers by now, so these columns are free
+    tmem_st32(s_tm + hf * 32, pk);
   }
-  return acc0 + acc1;
+  l += acc0 + acc1;
 }
 
-__device__ __forceinline__ void setmaxnreg_inc104() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 104;" ::: "memory");
+__device__ __forceinline__ void setmaxnreg_inc224() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
 }
-__device__ __forceinline__ void setmaxnreg_dec64() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
+__device__ __forceinline__ void setmaxnreg_dec56() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
 }
 
 template <int D, bool CAUSAL>
@@ -195,8 +262,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     int Hkv, int N, float scale_log2) {
   using Cfg = AttnCfg<D>;
   constexpr int ST = Cfg::kStages;
-  constexpr int kTmaWarp = kSoftmaxThreads / 32;  // warp 16
-  constexpr int kMmaWarp = kTmaWarp + 1;          // warp 17
+  constexpr int kTmaWarp = kSoftmaxThreads / 32;  // warp 8
+  constexpr int kMmaWarp = kTmaWarp + 1;          // warp 9: MMA issue
+  constexpr int kAllocWarp = kTmaWarp + 2;        // warp 10: tensor-memory allocation
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -232,13 +300,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&bars->s_full[w], 1);
-      mbar_init(&bars->p_full[w], 256);
+      mbar_init(&bars->p_full[w], 4);  // one arrive per softmax warp of the Q tile
       mbar_init(&bars->pv_done[w], 1);
     }
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kAllocWarp) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
@@ -248,8 +316,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = bars->tmem_base;
 
   if (warp >= kTmaWarp) {
-    // warpgroup 4 (TMA warp, MMA warp, two idle warps) hands registers to the softmax groups
-    setmaxnreg_dec64();
+    // warpgroup 2 (TMA, MMA and allocator warps, one idle) hands registers to the softmax groups
+    setmaxnreg_dec56();
     if (warp == kTmaWarp && lane == 0) {
       // ---------------------------------------------------------------- TMA producer
       tma_prefetch_desc(&tm_q);
@@ -274,32 +342,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // Order per key tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1).  tcgen05.mma operations
       // from one thread execute in issue order, so QK_w(j+1) may be issued right behind PV_w(j)
       // although it overwrites the tensor-memory columns PV_w(j) reads P_w from; the softmax of
-      // one Q tile then overlaps the other tile's PV + QK^T on the tensor pipe.
+      // one Q tile then overlaps the other tile's PV + QK^T on the tensor pipe.  Descriptors are
+      // computed once and advanced by constants (start-address field, 16-byte units), keeping
+      // the instructions per MMA few.
       constexpr uint32_t idq = idesc_i8_s32(kBM, kBN);
       constexpr uint32_t idv = idesc_f16_f32_bmn(kBM, D);
-      const uint32_t q_addr = smem_u32(smem + Cfg::kOffQ);
-      const uint32_t k_addr = smem_u32(smem + Cfg::kOffK);
-      const uint32_t v_addr = smem_u32(smem + Cfg::kOffV);
-      auto issue_qk = [&](int w, int s) {
-        const uint32_t qa = q_addr + w * Cfg::kQTile;
-        const uint32_t ka = k_addr + s * Cfg::kKTile;
-#pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk) {
-          const uint64_t ad = smem_desc(qa + kk * 32, 16, Cfg::kSboQK, Cfg::kSwQK);
-          const uint64_t bd = smem_desc(ka + kk * 32, 16, Cfg::kSboQK, Cfg::kSwQK);
-          mma_i8_ss(tmem + w * 128, ad, bd, idq, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars->s_full[w]);
-      };
+      const uint64_t dq0 = smem_desc(smem_u32(smem + Cfg::kOffQ), 16, Cfg::kSboQK, Cfg::kSwQK);
+      const uint64_t dk0 = smem_desc(smem_u32(smem + Cfg::kOffK), 16, Cfg::kSboQK, Cfg::kSwQK);
+      const uint64_t dv0 = smem_desc(smem_u32(smem + Cfg::kOffV), Cfg::kVBox, 1024, kSwizzle128B);
       bool ok = mbar_wait(&bars->q_full, 0, abort) && mbar_wait(&bars->kv_full[0], 0, abort);
       tc_fence_after();
       if (ok) {
-        issue_qk(0, 0);
-        if (nw1 > 0) issue_qk(1, 0);
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          if (w == 1 && nw1 == 0) break;
+          const uint64_t da = dq0 + static_cast<uint64_t>((w * Cfg::kQTile) >> 4);
+          mma_i8_ss(tmem + w * 128, da, dk0, idq, 0u);
+#pragma unroll
+          for (int kk = 1; kk < D / 32; ++kk) mma_i8_ss(tmem + w * 128, da + 2 * kk, dk0 + 2 * kk, idq, 1u);
+          mma_commit(&bars->s_full[w]);
+        }
       }
+      int s = 0;
       for (int j = 0; ok && j < n_kv; ++j) {
-        const int s = j % ST;
-        const int s1 = (j + 1) % ST;
+        const int s1 = s + 1 == ST ? 0 : s + 1;
+        const uint64_t dk1 = dk0 + static_cast<uint64_t>((s1 * Cfg::kKTile) >> 4);
+        const uint64_t dv = dv0 + static_cast<uint64_t>((s * Cfg::kVTile) >> 4);
         bool next_ready = false;
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
@@ -308,13 +376,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           ok = mbar_wait(&bars->p_full[w], static_cast<uint32_t>(j) & 1u, abort);
           if (!ok) continue;
           tc_fence_after();
-          const uint32_t va = v_addr + s * Cfg::kVTile;
+          const uint32_t ts = tmem + w * 128, to = tmem + 256 + w * D;
+          if (j == 0) mma_f16_ts(to, ts, dv, idv, 0u);
+          else mma_f16_ts(to, ts, dv, idv, 1u);
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint64_t bd = smem_desc(va + kk * 2048, Cfg::kVBox, 1024, kSwizzle128B);
-            mma_f16_ts(tmem + 256 + w * D, tmem + w * 128 + kk * 8, bd, idv,
-                       (j > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 1; kk < kBN / 16; ++kk) mma_f16_ts(to, ts + kk * 8, dv + kk * 128, idv, 1u);
           mma_commit(&bars->pv_done[w]);
           if (j + 1 < nw) {
             if (!next_ready) {
@@ -323,105 +389,87 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               tc_fence_after();
               next_ready = true;
             }
-            issue_qk(w, s1);
+            const uint64_t da = dq0 + static_cast<uint64_t>((w * Cfg::kQTile) >> 4);
+            mma_i8_ss(ts, da, dk1, idq, 0u);
+#pragma unroll
+            for (int kk = 1; kk < D / 32; ++kk) mma_i8_ss(ts, da + 2 * kk, dk1 + 2 * kk, idq, 1u);
+            mma_commit(&bars->s_full[w]);
           }
         }
         if (!ok) break;
         mma_commit(&bars->kv_empty[s]);
+        s = s1;
       }
     }
   } else {
     // ------------------------------------------------------------------ softmax warpgroups
-    // warp = 8 * tile + 4 * half + lane group: two threads share each score row, one per
-    // 64-key half (= one K scale block); they swap half-row maxima through shared memory.
-    setmaxnreg_inc104();
-    const int wt = warp >> 3;
-    const int half = (warp >> 2) & 1;
-    const int lg = warp & 3;
-    const int row = lg * 32 + lane;
-    const int pair_bar = 1 + wt * 4 + lg;  // named barrier of the two warps sharing these rows
+    // Warps 0-3: Q tile 0, warps 4-7: Q tile 1; thread = score row (TMEM lane 32 * (warp % 4)
+    // + lane), read with the 32x32b shape.
+    setmaxnreg_inc224();
+    const int wt = warp >> 2;
+    const int row = (warp & 3) * 32 + lane;
     const int nt = wt == 0 ? nw0 : nw1;
     if (nt > 0) {
       const int t = wt == 0 ? tq0 : tq1;
       const int qrow = t * kBM + row;
       const float sq = __ldg(q_scale + static_cast<size_t>(bh) * nqt + t);
       const float* ksc = k_scale + static_cast<size_t>(bg) * nkb;
-      const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
-      const uint32_t s_tm = tmem + lane_off + wt * 128 + half * 64;
-      const uint32_t p_tm = tmem + lane_off + wt * 128 + half * 32;
-      const uint32_t o_tm = tmem + lane_off + 256 + wt * D + half * (D / 2);
-      float m_used = -INFINITY;
-      float l = 0.0f;
+      const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+      const uint32_t s_tm = tmem + lane_off + wt * 128;
+      const uint32_t o_tm = tmem + lane_off + 256 + wt * D;
+      float m = -INFINITY, l = 0.0f;
       bool ok = true;
-      float ks = (half < nkb) ? __ldg(ksc + half) : 0.0f;
+      float ks0 = __ldg(ksc);
+      float ks1 = nkb > 1 ? __ldg(ksc + 1) : 0.0f;
       for (int j = 0; j < nt; ++j) {
-        const int kb_next = 2 * j + 2 + half;
-        const float ks_next = kb_next < nkb ? __ldg(ksc + kb_next) : 0.0f;
+        const float nks0 = (2 * j + 2 < nkb) ? __ldg(ksc + 2 * j + 2) : 0.0f;
+        const float nks1 = (2 * j + 3 < nkb) ? __ldg(ksc + 2 * j + 3) : 0.0f;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full[wt], static_cast<uint32_t>(j) & 1u, abort));
         if (!ok) break;
         tc_fence_after();
-        uint32_t sr[2][32];
-        tmem_ld32(s_tm, sr[0]);
-        tmem_ld32(s_tm + 32, sr[1]);
-        tmem_ld_wait(sr[0]);
-        tmem_ld_wait(sr[1]);
-        int lim = N - 1 - j * kBN - half * 64;
-        if (CAUSAL && j == t) lim = min(lim, row - half * 64);
-        const float c = sq * ks * scale_log2;
-        ks = ks_next;
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(s_tm + c * 32, sr[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+        int lim = N - 1 - j * kBN;
+        if (CAUSAL && j == t) lim = min(lim, row);
+        const float c0 = sq * ks0 * scale_log2;
+        const float c1 = sq * ks1 * scale_log2;
+        ks0 = nks0;
+        ks1 = nks1;
         // warp-uniform, so that every lane runs the same tensor-memory access sequence
-        const bool masked = __any_sync(0xFFFFFFFFu, lim < 63);
-        float hm = masked ? half_row_to_float_max<true>(sr, lim) : half_row_to_float_max<false>(sr, lim);
-        hm = hm == -INFINITY ? -INFINITY : hm * c;
-        // swap half-row maxima; the barrier also orders this thread's score reads before the
-        // partner's P writes, which land on columns 32-63 of the row
-        bars->xch[j & 1][wt][half][row] = hm;
-        tc_fence_before();
-        named_bar_sync(pair_bar, 64);
-        tc_fence_after();
-        const float mt = fmaxf(hm, bars->xch[j & 1][wt][half ^ 1][row]);
-        const float m_new = fmaxf(m_used, mt);
-        const bool need = m_new > m_used + kRescaleThreshold;
-        float alpha = 1.0f;
-        if (need) {
-          alpha = j == 0 ? 0.0f : ex2_approx(m_used - m_new);
-          m_used = m_new;
-          l *= alpha;
-        }
-        const float neg_m = kPOffset - m_used;
-        const float psum = masked ? half_row_exp_store<true>(sr, c, neg_m, p_tm)
-                                  : half_row_exp_store<false>(sr, c, neg_m, p_tm);
-        l += psum;
+        const bool masked = __any_sync(0xFFFFFFFFu, lim < kBN - 1);
+        float alpha;
+        bool need;
+        if (masked) softmax_row<true>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm);
+        else softmax_row<false>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm);
         if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
           // O holds PV up to tile j-1 (complete: QK(j) was issued after PV(j-1)), and PV(j)
-          // waits for this group's arrive below.  Both threads of a row take the same decision;
-          // each rescales its half of the O row.
+          // waits for this warp's arrive below.
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[16];
-            tmem_ld16(o_tm + cc * 16, o);
+            uint32_t o[32];
+            tmem_ld32(o_tm + cc * 32, o);
             tmem_ld_wait(o);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st16(o_tm + cc * 16, o);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(o_tm + cc * 32, o);
           }
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bars->p_full[wt]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[wt]);
       }
       if (ok) ok = mbar_wait(&bars->pv_done[wt], static_cast<uint32_t>(nt - 1) & 1u, abort);
       ok = __all_sync(0xFFFFFFFFu, ok);
-      // total row sum from the two halves (parity slot nt&1 is free: last used at step nt-2)
-      bars->xch[nt & 1][wt][half][row] = l;
-      named_bar_sync(pair_bar, 64);
-      l += bars->xch[nt & 1][wt][half ^ 1][row];
       tc_fence_after();
       if (ok) {
         const float inv_l = 1.0f / l;
-        __half* orow = out + (static_cast<size_t>(bh) * N + qrow) * D + half * (D / 2);
+        __half* orow = out + (static_cast<size_t>(bh) * N + qrow) * D;
 #pragma unroll
-        for (int cc = 0; cc < D / 64; ++cc) {
+        for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
           tmem_ld32(o_tm + cc * 32, o);
           tmem_ld_wait(o);
@@ -444,7 +492,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kAllocWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -507,16 +555,21 @@ __global__ void __launch_bounds__(128, 1)
   const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar_mma, 0, abort));
   tc_fence_after();
   if (ok) {
-    const int row = warp * 32 + lane;
-    int32_t* orow = s_out + static_cast<size_t>(blockIdx.x * kBM + row) * ldo + blockIdx.y * kBN;
+    // the 16x256b load shape the attention softmax uses: two loads per warp (lanes +0, +16)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t r[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c * 32, r);
+    for (int hh = 0; hh < 2; ++hh) {
+      const int lane_base = warp * 32 + hh * 16;
+      uint32_t r[64];
+      tmem_ld16x256b_x16(tmem + (static_cast<uint32_t>(lane_base) << 16), r);
       tmem_ld_wait(r);
+      const int rA = lane_base + (lane >> 2);
+      int32_t* oA = s_out + static_cast<size_t>(blockIdx.x * kBM + rA) * ldo + blockIdx.y * kBN + 2 * (lane & 3);
+      int32_t* oB = oA + static_cast<size_t>(8) * ldo;
 #pragma unroll
-      for (int v = 0; v < 8; ++v)
-        reinterpret_cast<uint4*>(orow + c * 32)[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+      for (int i = 0; i < 16; ++i) {
+        *reinterpret_cast<uint2*>(oA + 8 * i) = make_uint2(r[4 * i + 0], r[4 * i + 1]);
+        *reinterpret_cast<uint2*>(oB + 8 * i) = make_uint2(r[4 * i + 2], r[4 * i + 3]);
+      }
     }
   }
   tc_fence_before();

@@ -409,6 +409,17 @@ qattn_status qattn_debug_qk_int32(const int8_t* q_i8, const int8_t* k_i8, int32_
   return launch_status();
 }
 
+qattn_status qattn_debug_wait_timeout(long long limit_cycles, int* gave_up,
+                                      qattn_stream_t stream) {
+  if (gave_up == nullptr || limit_cycles < 0 || limit_cycles > kWaitLimitCycles)
+    return QATTN_ERR_INVALID_ARG;
+  qattn_status s = device_ok();
+  if (s != QATTN_OK) return s;
+  wait_timeout_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_cycles,
+                                                                                  gave_up);
+  return launch_status();
+}
+
 qattn_status qattn_check_device_status(qattn_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return QATTN_ERR_CUDA;

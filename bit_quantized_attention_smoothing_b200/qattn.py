@@ -27,7 +27,8 @@ KBLOCK = 64
 EXPORTS = [
     "qattn_status_string", "qattn_version", "qattn_smooth_quant_workspace", "qattn_smooth_quant",
     "qattn_attn_quantized", "qattn_forward_workspace", "qattn_forward_ws", "qattn_forward",
-    "qattn_forward_host", "qattn_debug_qk_int32", "qattn_check_device_status",
+    "qattn_forward_host", "qattn_debug_qk_int32", "qattn_debug_wait_timeout",
+    "qattn_check_device_status",
 ]
 
 
@@ -74,6 +75,8 @@ def _lib():
         L.qattn_forward_host.restype = i
         L.qattn_debug_qk_int32.argtypes = [P, P, P, i, i, i, i, i, i, i, i, i, i, i, P]
         L.qattn_debug_qk_int32.restype = i
+        L.qattn_debug_wait_timeout.argtypes = [ctypes.c_longlong, P, P]
+        L.qattn_debug_wait_timeout.restype = i
         L.qattn_check_device_status.argtypes = [P]
         L.qattn_check_device_status.restype = i
         _L = L
@@ -192,6 +195,14 @@ def qattn_debug_qk_int32(q_i8, k_i8, b, h, qt0, nqt, kt0, nkt, s_out=None, strea
                                      nqt, kt0, nkt, _stream(stream))
     _check("qattn_debug_qk_int32", st)
     return s_out
+
+
+def qattn_debug_wait_timeout(limit_cycles: int, stream=None) -> int:
+    """Runs the deliberately unsatisfied bounded wait; returns 1 if the kernel gave up."""
+    flag = torch.full((4,), -1, dtype=torch.int32, device="cuda")
+    _check("qattn_debug_wait_timeout",
+           _lib().qattn_debug_wait_timeout(int(limit_cycles), _p(flag), _stream(stream)))
+    return int(flag[0].item())
 
 
 def qattn_check_device_status(stream=None) -> int:

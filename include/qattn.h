@@ -129,6 +129,14 @@ qattn_status qattn_debug_qk_int32(const int8_t* q_i8, const int8_t* k_i8, int32_
                                   int H, int Hkv, int N, int d, int b, int h, int qt0, int nqt,
                                   int kt0, int nkt, qattn_stream_t stream);
 
+/* Failure-detection check: launches one block that waits on an mbarrier nothing arrives on,
+ * with a wait limit of limit_cycles SM clock cycles (0 .. the kernels' own limit of 2e9), so the
+ * bounded-wait path runs out on purpose.  The kernel then records QATTN_ERR_TIMEOUT in the device
+ * status word (read by qattn_check_device_status) and exits normally, leaving the context usable;
+ * *gave_up (device int) is set to 1.  No page counterpart: this tests the library's own waits. */
+qattn_status qattn_debug_wait_timeout(long long limit_cycles, int* gave_up,
+                                      qattn_stream_t stream);
+
 /* Synchronizes `stream`, then reports and clears the device status word: QATTN_OK, or
  * QATTN_ERR_TIMEOUT when a bounded wait inside a kernel ran out since the last check. */
 qattn_status qattn_check_device_status(qattn_stream_t stream);

@@ -97,3 +97,6 @@ def test_workspace_and_alignment_checks():
     assert st == 1
     st = L.qattn_debug_qk_int32(P(16), P(32), P(48), 1, 4, 2, 256, 128, 0, 4, 0, 1, 0, 1, None)
     assert st == 1
+    assert L.qattn_debug_wait_timeout(1000, None, None) == 1
+    assert L.qattn_debug_wait_timeout(-1, P(16), None) == 1
+    assert L.qattn_debug_wait_timeout(3_000_000_000, P(16), None) == 1

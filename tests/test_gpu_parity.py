@@ -174,3 +174,17 @@ def test_full_size_workload(lib, oracle, name):
     ok, msg = check_output(_rows_of(out, w, rows), ref)
     print(name, msg)
     assert ok, msg
+
+
+def test_bounded_wait_times_out_and_context_survives(lib):
+    """An mbarrier wait that nothing satisfies gives up after its limit (about 1 ms here), records
+    QATTN_ERR_TIMEOUT in the device status word and returns; the context stays usable."""
+    assert lib.qattn_check_device_status() == 0
+    assert lib.qattn_debug_wait_timeout(2_000_000) == 1
+    assert lib.qattn_check_device_status() == 5
+    assert lib.qattn_check_device_status() == 0      # reading clears it
+    w = WORKLOADS["tiny"]
+    q, k, v = _inputs(w, "cpu")
+    a = lib.qattn_forward(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.isfinite(a.float()).all() and lib.qattn_check_device_status() == 0
