@@ -244,6 +244,37 @@ qattn_status pool_alloc(void** p, size_t bytes, cudaStream_t st) {
   return cudaMallocFromPoolAsync(p, bytes, pool, st) == cudaSuccess ? QATTN_OK : QATTN_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------------------------
+// Fixed scratch for the allocation-free smoothing + quantization entry point
+// ---------------------------------------------------------------------------------------------
+
+// Exact int64 channel sums of K for qattn_smooth_quant_noalloc: room for B * Hkv * d <= 65536
+// (512 KiB), held by every GPU that loads the library until the process exits.
+constexpr size_t kNoAllocMaxSums = 65536;
+static __device__ __align__(256) long long g_noalloc_sums[kNoAllocMaxSums];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+long long* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_sums on the current device.  Host code cannot pass the symbol itself
+// (on the host it names a stand-in, not device memory), so the address is looked up once per
+// device with that device current and cached.
+qattn_status noalloc_scratch(long long** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return QATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_sums) != cudaSuccess || p == nullptr)
+      return QATTN_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<long long*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return QATTN_OK;
+}
+
 }  // namespace
 
 // =============================================================================================
@@ -286,6 +317,25 @@ qattn_status qattn_smooth_quant(const void* q, const void* k, int B, int H, int 
   if ((s = device_ok()) != QATTN_OK) return s;
   return dispatch_smooth_quant(q, k, B, H, Hkv, N, d, q_i8, q_scale, k_i8, k_scale, k_mean,
                                static_cast<long long*>(ws), reinterpret_cast<cudaStream_t>(stream));
+}
+
+// qattn_smooth_quant for callers that cannot allocate device memory: the channel-sum scratch is
+// the library's static g_noalloc_sums instead of a caller workspace.  Same kernels and results.
+qattn_status qattn_smooth_quant_noalloc(const void* q, const void* k, int B, int H, int Hkv, int N,
+                                        int d, int8_t* q_i8, float* q_scale, int8_t* k_i8,
+                                        float* k_scale, float* k_mean, qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q, k, q_i8, q_scale, k_i8, k_scale);
+  if (s != QATTN_OK) return s;
+  if (k_mean && !aligned16(k_mean)) return QATTN_ERR_MISALIGNED;
+  if (static_cast<size_t>(B) * Hkv * d > kNoAllocMaxSums) return QATTN_ERR_WORKSPACE;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  long long* sums = nullptr;
+  if ((s = noalloc_scratch(&sums)) != QATTN_OK) return s;
+  // the shared scratch keeps the previous call's sums: the dispatch zeroes it on `stream` first
+  return dispatch_smooth_quant(q, k, B, H, Hkv, N, d, q_i8, q_scale, k_i8, k_scale, k_mean, sums,
+                               reinterpret_cast<cudaStream_t>(stream));
 }
 
 qattn_status qattn_attn_quantized(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,

@@ -26,6 +26,7 @@ KBLOCK = 64
 # Every symbol include/qattn.h declares.
 EXPORTS = [
     "qattn_status_string", "qattn_version", "qattn_smooth_quant_workspace", "qattn_smooth_quant",
+    "qattn_smooth_quant_noalloc",
     "qattn_attn_quantized", "qattn_forward_workspace", "qattn_forward_ws", "qattn_forward",
     "qattn_forward_host", "qattn_debug_qk_int32", "qattn_debug_wait_timeout",
     "qattn_check_device_status",
@@ -63,6 +64,8 @@ def _lib():
         L.qattn_smooth_quant_workspace.restype = sz
         L.qattn_smooth_quant.argtypes = [P, P, i, i, i, i, i, P, P, P, P, P, P, sz, P]
         L.qattn_smooth_quant.restype = i
+        L.qattn_smooth_quant_noalloc.argtypes = [P, P, i, i, i, i, i, P, P, P, P, P, P]
+        L.qattn_smooth_quant_noalloc.restype = i
         L.qattn_attn_quantized.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, P]
         L.qattn_attn_quantized.restype = i
         L.qattn_forward_workspace.argtypes = [i, i, i, i, i]
@@ -139,6 +142,17 @@ def qattn_smooth_quant(q, k, q_i8=None, q_scale=None, k_i8=None, k_scale=None, k
     st = _lib().qattn_smooth_quant(_p(q), _p(k), B, H, Hkv, N, d, _p(q_i8), _p(q_scale), _p(k_i8),
                                    _p(k_scale), _p(k_mean), _p(ws), ws.numel(), _stream(stream))
     _check("qattn_smooth_quant", st)
+    return q_i8, q_scale, k_i8, k_scale, k_mean
+
+
+def qattn_smooth_quant_noalloc(q, k, q_i8, q_scale, k_i8, k_scale, k_mean=None, stream=None):
+    """qattn_smooth_quant without a workspace or any allocation: the caller passes every output
+    buffer, and the library's fixed device scratch (B*Hkv*d <= 65536) holds the channel sums.
+    For callers that cannot allocate device memory at call time."""
+    B, H, Hkv, N, d = _dims(q, k)
+    st = _lib().qattn_smooth_quant_noalloc(_p(q), _p(k), B, H, Hkv, N, d, _p(q_i8), _p(q_scale),
+                                           _p(k_i8), _p(k_scale), _p(k_mean), _stream(stream))
+    _check("qattn_smooth_quant_noalloc", st)
     return q_i8, q_scale, k_i8, k_scale, k_mean
 
 

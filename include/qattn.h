@@ -79,6 +79,25 @@ qattn_status qattn_smooth_quant(const void* q, const void* k, int B, int H, int 
                                 int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
                                 float* k_mean, void* ws, size_t ws_bytes, qattn_stream_t stream);
 
+/* Same as qattn_smooth_quant, but it allocates nothing and takes no workspace: for callers that
+ * cannot allocate device memory at call time, e.g. runtimes whose device memory is entirely
+ * reserved and sub-allocated by their own allocator, or code that must not add an allocation (and
+ * the synchronization it may bring) to the stream.  The pages have no counterpart: this is an
+ * interface convenience of this library.
+ *  - Scratch: the exact int64 channel sums live in a fixed device array inside the library,
+ *    65536 entries (512 KiB) on every GPU that loads it, held until the process exits.  Calls
+ *    with B * Hkv * d > 65536 return QATTN_ERR_WORKSPACE and launch nothing.
+ *  - The first call on a device looks up that array's device address (cudaGetSymbolAddress, with
+ *    that device current) and caches it; make that first call before any stream capture.
+ *  - All calls on a device share the array, which keeps the last call's contents; each call
+ *    clears it on `stream` before use.  Calls that overlap on the GPU (different streams, no
+ *    ordering between them) race on it and give wrong results: serialize them.
+ *  - No cudaMalloc, cudaFree or other allocating call is made.  Results are bit-identical to
+ *    qattn_smooth_quant's. */
+qattn_status qattn_smooth_quant_noalloc(const void* q, const void* k, int B, int H, int Hkv, int N,
+                                        int d, int8_t* q_i8, float* q_scale, int8_t* k_i8,
+                                        float* k_scale, float* k_mean, qattn_stream_t stream);
+
 /* ------------------------------------------------------------------------------------------
  * Attention on already-quantized Q and K (page sec. 3 and 4): S_int = Q_i8 K_i8^T exactly in
  * int32 on the tensor cores (tcgen05 kind::i8, accumulator in tensor memory), dequantized with
