@@ -165,13 +165,20 @@ __device__ __forceinline__ float scaled_max(float m, float c) {
   return m == -INFINITY ? -INFINITY : m * c;
 }
 
+// The int32 score s as the float 1.5 * 2^23 + s, by one integer add on the bit pattern (exact and
+// order-preserving for |s| < 2^22; an int8 dot product of length <= 128 stays below 2^21).  The
+// float s itself is that value minus kRoundMagic, also exact.
+__device__ __forceinline__ float score_biased(uint32_t s) { return __uint_as_float(s + 0x4B400000u); }
+static_assert(127 * 127 * 128 < (1 << 22), "biased score conversion range");
+
 // Score-register groups i (0-15) for which kExp2EmulateMask has bit i set go through exp2_poly2
 // on the FMA pipe; the rest use MUFU ex2.  Measured on B200 (llama8b_32k): moving 1/8, 1/4 or 3/8
 // of the exponentials to the FMA pipe made the kernel 3 %, 7 % and 13 % slower, so none is moved.
 constexpr uint32_t kExp2EmulateMask = 0x0000;
 __device__ __forceinline__ constexpr bool emulated_pair(int i) { return (kExp2EmulateMask >> i) & 1; }
 
-// One 128-key step of the softmax for the thread's score row: int32 -> float (exact, |S| < 2^24),
+// One 128-key step of the softmax for the thread's score row: int32 -> float (exact, see
+// score_biased),
 // masked keys (MASK; key offset above lim) -> -inf, row maximum per 64-key K scale block, lazy
 // update of the running max m (alpha = rescale factor, need = O must be rescaled), then
 // P = 2^(x * c - m + offset) packed as fp16 pairs (even key in the low half) and stored over the
@@ -186,7 +193,7 @@ __device__ __forceinline__ void softmax_row(uint32_t (&sr)[4][32], int lim, floa
   for (int c = 0; c < 4; ++c) {
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
-      float x = static_cast<float>(static_cast<int>(sr[c][e]));
+      float x = score_biased(sr[c][e]);
       if (MASK && c * 32 + e > lim) x = -INFINITY;
       sr[c][e] = __float_as_uint(x);
     }
@@ -197,7 +204,8 @@ __device__ __forceinline__ void softmax_row(uint32_t (&sr)[4][32], int lim, floa
       a = fmax3(a, __uint_as_float(sr[c][e + 2]), __uint_as_float(sr[c][e + 3]));
     }
   }
-  const float t = fmaxf(scaled_max(fmaxf(mx0, mx1), c0), scaled_max(fmaxf(mx2, mx3), c1));
+  const float t = fmaxf(scaled_max(fmaxf(mx0, mx1) - kRoundMagic, c0),
+                       scaled_max(fmaxf(mx2, mx3) - kRoundMagic, c1));
   const float mn = fmaxf(m, t);
   need = mn > m + kRescaleThreshold;
   alpha = 1.0f;
@@ -217,9 +225,9 @@ __device__ __forceinline__ void softmax_row(uint32_t (&sr)[4][32], int lim, floa
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
         const int i = (2 * hf + q) * 16 + (e >> 1);  // pair index 0..63
-        const float x0 = __uint_as_float(sr[2 * hf + q][e]);
-        const float x1 = __uint_as_float(sr[2 * hf + q][e + 1]);
-        float y0, y1, p0, p1;
+        float x0, x1, y0, y1, p0, p1;
+        fadd2(x0, x1, __uint_as_float(sr[2 * hf + q][e]), __uint_as_float(sr[2 * hf + q][e + 1]),
+              -kRoundMagic, -kRoundMagic);
         ffma2(y0, y1, x0, x1, c, g);
         if (emulated_pair(i & 15)) {
           exp2_poly2(y0, y1, p0, p1);

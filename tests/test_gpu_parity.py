@@ -113,6 +113,34 @@ def test_attention_on_oracle_codes(lib, oracle, name, over):
     assert ok, msg
 
 
+def _planted_jumps(w):
+    """Seeded inputs whose row maxima jump by far more than the lazy-rescale threshold after the
+    first key tile: one direction u is added to every query, and three keys are replaced by
+    large multiples of u (token 300 inside the diagonal tile of rows 256-383, tokens 700 and 901
+    further on), so that rows reaching them see their running max grow by ~20-60 log2 units.
+    The softmax must then void its optimistic P for that step, move the max and rescale O."""
+    q, k, v = make_inputs(w)
+    gen = torch.Generator().manual_seed(77)
+    u = torch.randn(w.d, generator=gen)
+    u = u / u.norm()
+    q = (q.float() + 3.0 * u).half()
+    k = k.float()
+    for t, a in ((300, 40.0), (700, 80.0), (901, 120.0)):
+        k[:, :, t] = a * u
+    return q, k.half(), v
+
+
+@pytest.mark.parametrize("d,causal", [(64, True), (128, True), (128, False)])
+def test_forward_planted_max_jumps(lib, oracle, d, causal):
+    w = WORKLOADS["tiny"].with_(B=1, H=2, Hkv=1, N=1000, d=d, causal=causal)
+    q, k, v = _planted_jumps(w)
+    out = lib.qattn_forward(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+    assert lib.qattn_check_device_status() == 0
+    ref, _ = oracle.forward(np16(q), np16(k), np16(v), w.B, w.H, w.Hkv, w.N, w.d, causal)
+    ok, msg = check_output(out.float().cpu().numpy().reshape(-1, w.d), ref)
+    assert ok, msg
+
+
 def test_forward_variants_agree(lib):
     w = WORKLOADS["prefill4k"].with_(B=1, H=4, Hkv=2, N=777)
     q, k, v = _inputs(w, "cpu")
