@@ -8,7 +8,8 @@
 //  * one CTA owns two 128-row Q tiles of one (batch, head) and streams 128-key K/V tiles;
 //  * warp 8 (TMA): loads both Q tiles once, then K (int8) and V (fp16) tiles into a STAGES-deep
 //    shared-memory ring (128-byte / 64-byte swizzled tiles, mbarrier transaction counts);
-//  * warp 9 (MMA, one thread): S_w = Q_w K^T as tcgen05.mma kind::i8 (M=128, N=128, K=32 per
+//  * warp 9 (MMA; the whole warp runs the loop on warp-uniform descriptors and one elected lane
+//    issues each instruction): S_w = Q_w K^T as tcgen05.mma kind::i8 (M=128, N=128, K=32 per
 //    instruction) into tensor memory, then O_w += P_w V as tcgen05.mma kind::f16 with P read
 //    from tensor memory (M=128, N=d, K=16), fp32 accumulator in tensor memory; issue order
 //    PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1) so that one Q tile's softmax overlaps the other's MMAs;
@@ -345,8 +346,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int x = 0; x < D / 64; ++x)
           tma_load_3d(vdst + x * Cfg::kVBox, &tm_v, &bars->kv_full[s], x * 64, j * kBN, bg);
       }
-    } else if (warp == kMmaWarp && lane == 0) {
+    } else if (warp == kMmaWarp) {
       // ---------------------------------------------------------------- MMA issuer
+      // The whole warp runs this loop, so the descriptors and addresses are warp-uniform values;
+      // one elected lane issues each tcgen05 instruction.
       // Order per key tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1).  tcgen05.mma operations
       // from one thread execute in issue order, so QK_w(j+1) may be issued right behind PV_w(j)
       // although it overwrites the tensor-memory columns PV_w(j) reads P_w from; the softmax of
@@ -358,17 +361,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t dq0 = smem_desc(smem_u32(smem + Cfg::kOffQ), 16, Cfg::kSboQK, Cfg::kSwQK);
       const uint64_t dk0 = smem_desc(smem_u32(smem + Cfg::kOffK), 16, Cfg::kSboQK, Cfg::kSwQK);
       const uint64_t dv0 = smem_desc(smem_u32(smem + Cfg::kOffV), Cfg::kVBox, 1024, kSwizzle128B);
-      bool ok = mbar_wait(&bars->q_full, 0, abort) && mbar_wait(&bars->kv_full[0], 0, abort);
+      bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->q_full, 0, abort) && mbar_wait(&bars->kv_full[0], 0, abort));
       tc_fence_after();
       if (ok) {
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
           if (w == 1 && nw1 == 0) break;
           const uint64_t da = dq0 + static_cast<uint64_t>((w * Cfg::kQTile) >> 4);
-          mma_i8_ss(tmem + w * 128, da, dk0, idq, 0u);
+          mma_i8_ss_warp(tmem + w * 128, da, dk0, idq, 0u);
 #pragma unroll
-          for (int kk = 1; kk < D / 32; ++kk) mma_i8_ss(tmem + w * 128, da + 2 * kk, dk0 + 2 * kk, idq, 1u);
-          mma_commit(&bars->s_full[w]);
+          for (int kk = 1; kk < D / 32; ++kk) mma_i8_ss_warp(tmem + w * 128, da + 2 * kk, dk0 + 2 * kk, idq, 1u);
+          mma_commit_warp(&bars->s_full[w]);
         }
       }
       int s = 0;
@@ -381,31 +384,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int w = 0; w < 2; ++w) {
           const int nw = w == 0 ? nw0 : nw1;
           if (!ok || j >= nw) continue;
-          ok = mbar_wait(&bars->p_full[w], static_cast<uint32_t>(j) & 1u, abort);
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->p_full[w], static_cast<uint32_t>(j) & 1u, abort));
           if (!ok) continue;
           tc_fence_after();
           const uint32_t ts = tmem + w * 128, to = tmem + 256 + w * D;
-          if (j == 0) mma_f16_ts(to, ts, dv, idv, 0u);
-          else mma_f16_ts(to, ts, dv, idv, 1u);
+          if (j == 0) mma_f16_ts_warp(to, ts, dv, idv, 0u);
+          else mma_f16_ts_warp(to, ts, dv, idv, 1u);
 #pragma unroll
-          for (int kk = 1; kk < kBN / 16; ++kk) mma_f16_ts(to, ts + kk * 8, dv + kk * 128, idv, 1u);
-          mma_commit(&bars->pv_done[w]);
+          for (int kk = 1; kk < kBN / 16; ++kk) mma_f16_ts_warp(to, ts + kk * 8, dv + kk * 128, idv, 1u);
+          mma_commit_warp(&bars->pv_done[w]);
           if (j + 1 < nw) {
             if (!next_ready) {
-              ok = mbar_wait(&bars->kv_full[s1], static_cast<uint32_t>((j + 1) / ST) & 1u, abort);
+              ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->kv_full[s1], static_cast<uint32_t>((j + 1) / ST) & 1u, abort));
               if (!ok) continue;
               tc_fence_after();
               next_ready = true;
             }
             const uint64_t da = dq0 + static_cast<uint64_t>((w * Cfg::kQTile) >> 4);
-            mma_i8_ss(ts, da, dk1, idq, 0u);
+            mma_i8_ss_warp(ts, da, dk1, idq, 0u);
 #pragma unroll
-            for (int kk = 1; kk < D / 32; ++kk) mma_i8_ss(ts, da + 2 * kk, dk1 + 2 * kk, idq, 1u);
-            mma_commit(&bars->s_full[w]);
+            for (int kk = 1; kk < D / 32; ++kk) mma_i8_ss_warp(ts, da + 2 * kk, dk1 + 2 * kk, idq, 1u);
+            mma_commit_warp(&bars->s_full[w]);
           }
         }
         if (!ok) break;
-        mma_commit(&bars->kv_empty[s]);
+        mma_commit_warp(&bars->kv_empty[s]);
         s = s1;
       }
     }
