@@ -394,6 +394,36 @@ qattn_status qattn_forward(const void* q, const void* k, const void* v, void* ou
   return s;
 }
 
+namespace {
+
+// Copy streams of the host-buffer forward, created once per device (non-blocking, so they do
+// not serialise with the legacy default stream).
+std::mutex g_copy_mu;
+std::map<int, std::pair<cudaStream_t, cudaStream_t>> g_copy_streams;
+
+qattn_status copy_streams(cudaStream_t* in, cudaStream_t* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_copy_mu);
+  auto it = g_copy_streams.find(dev);
+  if (it == g_copy_streams.end()) {
+    cudaStream_t a = nullptr, b = nullptr;
+    if (cudaStreamCreateWithFlags(&a, cudaStreamNonBlocking) != cudaSuccess) return QATTN_ERR_CUDA;
+    if (cudaStreamCreateWithFlags(&b, cudaStreamNonBlocking) != cudaSuccess) {
+      cudaStreamDestroy(a);
+      return QATTN_ERR_CUDA;
+    }
+    it = g_copy_streams.emplace(dev, std::make_pair(a, b)).first;
+  }
+  *in = it->second.first;
+  *out = it->second.second;
+  return QATTN_OK;
+}
+
+constexpr int kHostChunks = 8;  // pipeline depth of the host-buffer forward
+
+}  // namespace
+
 qattn_status qattn_forward_host(const void* q_host, const void* k_host, const void* v_host,
                                 void* out_host, int B, int H, int Hkv, int N, int d, int causal,
                                 qattn_stream_t stream) {
@@ -402,6 +432,8 @@ qattn_status qattn_forward_host(const void* q_host, const void* k_host, const vo
   if (!q_host || !k_host || !v_host || !out_host) return QATTN_ERR_INVALID_ARG;
   if ((s = device_ok()) != QATTN_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  if ((s = copy_streams(&s_in, &s_out)) != QATTN_OK) return s;
   const size_t qb = sizeof(uint16_t) * static_cast<size_t>(B) * H * N * d;
   const size_t kb = sizeof(uint16_t) * static_cast<size_t>(B) * Hkv * N * d;
   const size_t off_k = align_up(qb), off_v = off_k + align_up(kb), off_o = off_v + align_up(kb);
@@ -409,17 +441,67 @@ qattn_status qattn_forward_host(const void* q_host, const void* k_host, const vo
   void* buf = nullptr;
   if ((s = pool_alloc(&buf, total, st)) != QATTN_OK) return s;
   uint8_t* b8 = static_cast<uint8_t*>(buf);
-  if (cudaMemcpyAsync(b8, q_host, qb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(b8 + off_k, k_host, kb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(b8 + off_v, v_host, kb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+  // Every (batch, kv head) group -- its kv head and the H / Hkv query heads reading it -- is an
+  // independent forward (the smoothing mean is per group), and group f = b * Hkv + g owns
+  // contiguous bytes of q, k, v and out.  The groups are cut into up to kHostChunks chunks; chunk
+  // c's upload (s_in), forward (the caller's stream) and download (s_out) are ordered by events,
+  // so one chunk's copies overlap another chunk's kernels.
+  const int G = B * Hkv, r = H / Hkv;
+  const int nch = G < kHostChunks ? G : kHostChunks;
+  const int per = (G + nch - 1) / nch;
+  const size_t q_grp = sizeof(uint16_t) * static_cast<size_t>(r) * N * d;
+  const size_t k_grp = sizeof(uint16_t) * static_cast<size_t>(N) * d;
+  cudaEvent_t ev[2 * kHostChunks + 2] = {};
+  int nev = 0;
+  for (int i = 0; i < 2 * nch + 2 && s == QATTN_OK; ++i, ++nev)
+    if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) s = QATTN_ERR_CUDA;
+  const char* qh = static_cast<const char*>(q_host);
+  const char* kh = static_cast<const char*>(k_host);
+  const char* vh = static_cast<const char*>(v_host);
+  char* oh = static_cast<char*>(out_host);
+  // s_in and s_out start after the work already queued on the caller's stream (the pool
+  // allocation above and anything before this call)
+  if (s == QATTN_OK && (cudaEventRecord(ev[2 * nch], st) != cudaSuccess ||
+                        cudaStreamWaitEvent(s_in, ev[2 * nch], 0) != cudaSuccess ||
+                        cudaStreamWaitEvent(s_out, ev[2 * nch], 0) != cudaSuccess))
     s = QATTN_ERR_CUDA;
-  if (s == QATTN_OK)
-    s = qattn_forward(b8, b8 + off_k, b8 + off_v, b8 + off_o, B, H, Hkv, N, d, causal, stream);
-  if (s == QATTN_OK &&
-      cudaMemcpyAsync(out_host, b8 + off_o, qb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    s = QATTN_ERR_CUDA;
+  for (int c = 0; c < nch && s == QATTN_OK; ++c) {
+    const int f0 = c * per, nf = (f0 + per <= G ? per : G - f0);
+    if (nf <= 0) break;
+    if (cudaMemcpyAsync(b8 + f0 * q_grp, qh + f0 * q_grp, nf * q_grp, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaMemcpyAsync(b8 + off_k + f0 * k_grp, kh + f0 * k_grp, nf * k_grp, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaMemcpyAsync(b8 + off_v + f0 * k_grp, vh + f0 * k_grp, nf * k_grp, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaEventRecord(ev[c], s_in) != cudaSuccess)
+      s = QATTN_ERR_CUDA;
+  }
+  for (int c = 0; c < nch && s == QATTN_OK; ++c) {
+    const int f0 = c * per, nf = (f0 + per <= G ? per : G - f0);
+    if (nf <= 0) break;
+    if (cudaStreamWaitEvent(st, ev[c], 0) != cudaSuccess) {
+      s = QATTN_ERR_CUDA;
+      break;
+    }
+    // the chunk as a forward of nf "batches" of one kv head and r query heads each
+    s = qattn_forward(b8 + f0 * q_grp, b8 + off_k + f0 * k_grp, b8 + off_v + f0 * k_grp,
+                      b8 + off_o + f0 * q_grp, nf, r, 1, N, d, causal, stream);
+    if (s == QATTN_OK && (cudaEventRecord(ev[nch + c], st) != cudaSuccess ||
+                          cudaStreamWaitEvent(s_out, ev[nch + c], 0) != cudaSuccess ||
+                          cudaMemcpyAsync(oh + f0 * q_grp, b8 + off_o + f0 * q_grp, nf * q_grp,
+                                          cudaMemcpyDeviceToHost, s_out) != cudaSuccess))
+      s = QATTN_ERR_CUDA;
+  }
+  // the caller's stream takes up both copy streams again before the buffer goes back to the pool
+  if (nev < 2 * nch + 2) {
+    // no event, so nothing was queued on the copy streams
+  } else if (cudaEventRecord(ev[2 * nch + 1], s_out) != cudaSuccess ||
+      cudaStreamWaitEvent(st, ev[2 * nch + 1], 0) != cudaSuccess ||
+      cudaEventRecord(ev[2 * nch], s_in) != cudaSuccess ||
+      cudaStreamWaitEvent(st, ev[2 * nch], 0) != cudaSuccess) {
+    if (s == QATTN_OK) s = QATTN_ERR_CUDA;
+  }
   if (cudaFreeAsync(buf, st) != cudaSuccess && s == QATTN_OK) s = QATTN_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess && s == QATTN_OK) s = QATTN_ERR_CUDA;
+  for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
   return s;
 }
 

@@ -127,10 +127,12 @@ qattn_status qattn_forward_ws(const void* q, const void* k, const void* v, void*
 qattn_status qattn_forward(const void* q, const void* k, const void* v, void* out, int B, int H,
                            int Hkv, int N, int d, int causal, qattn_stream_t stream);
 
-/* Forward on HOST buffers: copies q, k, v to the device, runs qattn_forward, copies the result
- * back to out_host, and returns after the copy has finished (the stream is synchronized).  Device
- * buffers come from the library's pool.  Page-locked host memory gives asynchronous copies;
- * pageable memory works but is slower. */
+/* Forward on HOST buffers: copies q, k, v to the device, runs the forward, copies the result
+ * back to out_host, and returns after the copy has finished (the stream is synchronized).  The
+ * (batch, kv head) groups are processed in up to 8 chunks whose uploads, kernels (on `stream`)
+ * and downloads overlap through two copy streams the library keeps per device; results are
+ * identical to qattn_forward.  Device buffers come from the library's pool.  Page-locked host
+ * memory gives asynchronous, overlapped copies; pageable memory works but is slower. */
 qattn_status qattn_forward_host(const void* q_host, const void* k_host, const void* v_host,
                                 void* out_host, int B, int H, int Hkv, int N, int d, int causal,
                                 qattn_stream_t stream);

@@ -159,6 +159,22 @@ def test_forward_variants_agree(lib):
     assert torch.equal(a.cpu(), c) and torch.equal(a.cpu(), d)
 
 
+@pytest.mark.parametrize("pinned", [True, False])
+def test_host_forward_pipeline_chunks(lib, pinned):
+    """qattn_forward_host cuts the (batch, kv head) groups into chunks whose copies and kernels
+    overlap; 6 groups make uneven chunks.  Results must equal the device-buffer forward bit for
+    bit."""
+    w = WORKLOADS["wide64"].with_(B=2, H=6, Hkv=3, N=300, causal=True)
+    q, k, v = _inputs(w, "cpu")
+    a = lib.qattn_forward(q.cuda(), k.cuda(), v.cuda(), causal=True)
+    hq, hk, hv = (t.cpu() for t in (q, k, v))
+    if pinned:
+        hq, hk, hv = hq.pin_memory(), hk.pin_memory(), hv.pin_memory()
+    c = lib.qattn_forward_host(hq, hk, hv, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a.cpu(), c)
+
+
 def test_repeated_calls_are_deterministic(lib):
     w = WORKLOADS["wide64"].with_(B=1, H=2, Hkv=2, N=1024)
     q, k, v = _inputs(w, "cpu")
