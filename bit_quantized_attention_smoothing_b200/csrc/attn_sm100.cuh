@@ -32,6 +32,7 @@
 #include <cstdint>
 
 #include "sm100_ptx.cuh"
+#include "quant.cuh"
 
 namespace qattn {
 
@@ -58,7 +59,8 @@ struct AttnCfg {
   static constexpr int kOffV = kOffK + kStages * kKTile;
   static constexpr int kOffBar = kOffV + kStages * kVTile;
   static constexpr int kBarBytes = 256;
-  static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
+  static constexpr int kOffRed = kOffBar + kBarBytes;  // [Q tile][warp] row maxima (fused Q)
+  static constexpr int kSmemBytes = kOffRed + 64 + 1024;  // + alignment slack
   // K-major int8 operands: rows of D bytes, 8-row swizzle atoms.
   static constexpr uint32_t kSwQK = D == 128 ? kSwizzle128B : kSwizzle64B;
   static constexpr uint32_t kSboQK = 8 * D;
@@ -256,6 +258,95 @@ __device__ __forceinline__ void softmax_row(uint32_t (&sr)[4][32], int lim, floa
   l += acc0 + acc1;
 }
 
+// Fused Q quantization for one 128-row Q tile by its softmax warpgroup (128 threads, tid 0-127,
+// Q tile wt, first row r0): the tile's fp16 values (coalesced 16-byte loads of 8 values; zeros
+// past N), the tile's amax (|x| and max on packed fp16 pairs, exact) through a warp shuffle and
+// a warpgroup barrier, scale = amax / 127 and codes rint(x * (1 / scale)) -- with the correctly
+// rounded quotient x / scale instead where a value lies within 2^-13 of a half-integer, which is
+// quantize_kernel's rule, so codes and scales are bit-identical to it (an 8-value chunk holding
+// such a value is recomputed on its own) -- written into the K-major swizzled layout the TMA
+// would produce (128-byte rows with 128-byte swizzle at d = 128, 64-byte rows with 64-byte
+// swizzle at d = 64).  |x| <= amax keeps every code within [-127, 127].  Returns the scale (0 for
+// an all-zero tile).
+template <int D>
+__device__ __forceinline__ float quantize_q_tile(const uint16_t* __restrict__ q_head, int r0,
+                                                 int N, int tid, int wt, uint8_t* tile,
+                                                 float* red) {
+  constexpr int CPR = D / 8;              // 16-byte input chunks (8 values) per row
+  constexpr int NCH = kBM * CPR / 128;    // chunks per thread
+  const uint4* src = reinterpret_cast<const uint4*>(q_head + static_cast<size_t>(r0) * D);
+  // all NCH loads are issued before any is used: no branch around them (rows past N read row
+  // r0, which exists, and are zeroed afterwards)
+  uint4 v[NCH];
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    const int c = i * 128 + tid;          // chunk index within the tile
+    v[i] = __ldg(src + (r0 + c / CPR < N ? c : 0));
+  }
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    if (r0 + (i * 128 + tid) / CPR >= N) v[i] = make_uint4(0, 0, 0, 0);
+  }
+  __half2 m2 = __floats2half2_rn(0.0f, 0.0f);
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __half2*>(&v[i].x)));
+    m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __half2*>(&v[i].y)));
+    m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __half2*>(&v[i].z)));
+    m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __half2*>(&v[i].w)));
+  }
+  float amax = fmaxf(__low2float(m2), __high2float(m2));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  if ((tid & 31) == 0) red[wt * 4 + (tid >> 5)] = amax;
+  named_bar_sync(1 + wt, 128);
+  amax = fmaxf(fmaxf(red[wt * 4], red[wt * 4 + 1]), fmaxf(red[wt * 4 + 2], red[wt * 4 + 3]));
+  const float s = __fdiv_rn(amax, 127.0f);
+  const float rcp = amax > 0.0f ? __frcp_rn(s) : 0.0f;
+  // 8 codes of input chunk col land in 16-byte output chunk col / 2 of the row, half col % 2;
+  // that 16-byte chunk sits at position (col / 2) ^ (the row's 128-byte line index bits)
+  auto dst = [&](int c) -> uint32_t {
+    const int row = c / CPR, col = c % CPR;
+    const uint32_t swz = D == 128 ? static_cast<uint32_t>(row & 7) : static_cast<uint32_t>((row >> 1) & 3);
+    return smem_u32(tile + row * D + (((static_cast<uint32_t>(col) >> 1) ^ swz) << 4) + ((col & 1) << 3));
+  };
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    const uint32_t hw[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+    uint32_t w[2];
+    bool near_tie = false;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      int r[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t word = hw[2 * k + (e >> 1)];
+        const float y = half_bits_to_float((e & 1) ? (word >> 16) : (word & 0xFFFFu)) * rcp;
+        const float ry = rintf(y);
+        near_tie |= fabsf(y - ry) > 0.4998779296875f;  // within 2^-13 of a half-integer
+        r[e] = static_cast<int>(ry);
+      }
+      w[k] = __byte_perm(__byte_perm(r[0], r[1], 0x0040), __byte_perm(r[2], r[3], 0x0040), 0x5410);
+    }
+    if (__any_sync(0xFFFFFFFFu, near_tie) && near_tie) {
+      // rare: this chunk again with the exact quotient where it decides the rounding
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        float x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t word = hw[2 * k + (e >> 1)];
+          x[e] = quant_code(half_bits_to_float((e & 1) ? (word >> 16) : (word & 0xFFFFu)), s, rcp);
+        }
+        w[k] = pack4_i8(x[0], x[1], x[2], x[3]);
+      }
+    }
+    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(dst(i * 128 + tid)), "r"(w[0]), "r"(w[1])
+                 : "memory");
+  }
+  return amax > 0.0f ? s : 0.0f;
+}
+
 __device__ __forceinline__ void setmaxnreg_inc224() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
 }
@@ -263,10 +354,15 @@ __device__ __forceinline__ void setmaxnreg_dec56() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
 }
 
-template <int D, bool CAUSAL>
+// QF16: Q arrives as fp16 (q16) and the softmax warps quantize their own Q tile into shared
+// memory before the first QK^T (per-tile amax, scale = amax / 127, the same rounding as
+// quantize_kernel); otherwise int8 Q and its scales come from the smoothing + quantization pass
+// (tm_q, q_scale).
+template <int D, bool CAUSAL, bool QF16>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scale,
+                    const uint16_t* __restrict__ q16,
                     const float* __restrict__ k_scale, __half* __restrict__ out, int B, int H,
                     int Hkv, int N, float scale_log2) {
   using Cfg = AttnCfg<D>;
@@ -302,7 +398,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int n_kv = max(nw0, nw1);
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
+    // QF16: one arrive per softmax warp once its rows of the Q tiles are in shared memory
+    mbar_init(&bars->q_full, QF16 ? kSoftmaxThreads / 32 : 1);
     for (int s = 0; s < ST; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
@@ -329,12 +426,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     setmaxnreg_dec56();
     if (warp == kTmaWarp && lane == 0) {
       // ---------------------------------------------------------------- TMA producer
-      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(&bars->q_full, Cfg::kQTile * (has1 ? 2 : 1));
-      tma_load_3d(smem + Cfg::kOffQ, &tm_q, &bars->q_full, 0, tq0 * kBM, bh);
-      if (has1) tma_load_3d(smem + Cfg::kOffQ + Cfg::kQTile, &tm_q, &bars->q_full, 0, tq1 * kBM, bh);
+      if (!QF16) {
+        tma_prefetch_desc(&tm_q);
+        mbar_arrive_expect_tx(&bars->q_full, Cfg::kQTile * (has1 ? 2 : 1));
+        tma_load_3d(smem + Cfg::kOffQ, &tm_q, &bars->q_full, 0, tq0 * kBM, bh);
+        if (has1) tma_load_3d(smem + Cfg::kOffQ + Cfg::kQTile, &tm_q, &bars->q_full, 0, tq1 * kBM, bh);
+      }
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % ST;
         const uint32_t u = static_cast<uint32_t>(j / ST);
@@ -420,10 +519,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int wt = warp >> 2;
     const int row = (warp & 3) * 32 + lane;
     const int nt = wt == 0 ? nw0 : nw1;
+    float sq_fused = 0.0f;
+    if (QF16) {
+      // quantize this warpgroup's Q tile (thread = row) into the MMA's swizzled int8 layout
+      float* red = reinterpret_cast<float*>(smem + Cfg::kOffRed);
+      if (nt > 0)
+        sq_fused = quantize_q_tile<D>(q16 + (static_cast<size_t>(bh) * N) * D,
+                                      (wt == 0 ? tq0 : tq1) * kBM, N, row, wt,
+                                      smem + Cfg::kOffQ + wt * Cfg::kQTile, red);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->q_full);
+    }
     if (nt > 0) {
       const int t = wt == 0 ? tq0 : tq1;
       const int qrow = t * kBM + row;
-      const float sq = __ldg(q_scale + static_cast<size_t>(bh) * nqt + t);
+      const float sq = QF16 ? sq_fused : __ldg(q_scale + static_cast<size_t>(bh) * nqt + t);
       const float* ksc = k_scale + static_cast<size_t>(bg) * nkb;
       const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
       const uint32_t s_tm = tmem + lane_off + wt * 128;

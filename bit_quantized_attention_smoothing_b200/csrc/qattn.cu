@@ -134,6 +134,8 @@ QuantLayout forward_layout(int B, int H, int Hkv, int N, int d) {
   return L;
 }
 
+// Channel sums, then one quantization launch over the Q blocks (unless q is null: the fused
+// forward quantizes Q inside the attention kernel) and the K blocks.
 template <int D>
 qattn_status run_smooth_quant(const void* q, const void* k, int B, int H, int Hkv, int N,
                               int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
@@ -145,7 +147,7 @@ qattn_status run_smooth_quant(const void* q, const void* k, int B, int H, int Hk
   dim3 g1(B * Hkv, (N + kSumRowsPerCta - 1) / kSumRowsPerCta);
   k_channel_sums_kernel<D><<<g1, 256, 0, st>>>(static_cast<const uint16_t*>(k), N, sums);
   if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
-  const long long nq = static_cast<long long>(B) * H * nqb;
+  const long long nq = q ? static_cast<long long>(B) * H * nqb : 0;
   const long long nk = static_cast<long long>(B) * Hkv * nkb;
   if (nq + nk > 0x7FFFFFFFLL) return QATTN_ERR_UNSUPPORTED;
   quantize_kernel<D><<<static_cast<unsigned>(nq + nk), 256, 0, st>>>(
@@ -154,17 +156,19 @@ qattn_status run_smooth_quant(const void* q, const void* k, int B, int H, int Hk
   return launch_status();
 }
 
-template <int D, bool CAUSAL>
-qattn_status run_attn(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+// q is int8 (with q_scale) or, for QF16, the fp16 Q that the kernel quantizes itself.
+template <int D, bool CAUSAL, bool QF16>
+qattn_status run_attn(const void* q, const float* q_scale, const int8_t* k_i8,
                       const float* k_scale, const void* v, void* out, int B, int H, int Hkv,
                       int N, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
-  if (!make_i8_map(&tq, q_i8, D, N, static_cast<long long>(B) * H) ||
+  std::memset(&tq, 0, sizeof(tq));  // unused by the QF16 kernel
+  if ((!QF16 && !make_i8_map(&tq, q, D, N, static_cast<long long>(B) * H)) ||
       !make_i8_map(&tk, k_i8, D, N, static_cast<long long>(B) * Hkv) ||
       !make_v_map(&tv, v, D, N, static_cast<long long>(B) * Hkv))
     return QATTN_ERR_CUDA;
   using Cfg = AttnCfg<D>;
-  auto kern = attn_fwd_kernel<D, CAUSAL>;
+  auto kern = attn_fwd_kernel<D, CAUSAL, QF16>;
   // The kernel moves registers between its warpgroups with setmaxnreg; the split adds up only if
   // the launch allocates exactly kAttnLaunchRegs per thread, so never launch it otherwise.
   static int regs_checked = 0;
@@ -182,18 +186,20 @@ qattn_status run_attn(const int8_t* q_i8, const float* q_scale, const int8_t* k_
   if (grid > 0x7FFFFFFFLL) return QATTN_ERR_UNSUPPORTED;
   const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   kern<<<static_cast<unsigned>(grid), kAttnThreads, Cfg::kSmemBytes, st>>>(
-      tq, tk, tv, q_scale, k_scale, static_cast<__half*>(out), B, H, Hkv, N, scale_log2);
+      tq, tk, tv, q_scale, QF16 ? static_cast<const uint16_t*>(q) : nullptr, k_scale,
+      static_cast<__half*>(out), B, H, Hkv, N, scale_log2);
   return launch_status();
 }
 
-qattn_status dispatch_attn(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+template <bool QF16>
+qattn_status dispatch_attn(const void* q, const float* q_scale, const int8_t* k_i8,
                            const float* k_scale, const void* v, void* out, int B, int H, int Hkv,
                            int N, int d, int causal, cudaStream_t st) {
   if (d == 128)
-    return causal ? run_attn<128, true>(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st)
-                  : run_attn<128, false>(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st);
-  return causal ? run_attn<64, true>(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st)
-                : run_attn<64, false>(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st);
+    return causal ? run_attn<128, true, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st)
+                  : run_attn<128, false, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st);
+  return causal ? run_attn<64, true, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st)
+                : run_attn<64, false, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st);
 }
 
 qattn_status dispatch_smooth_quant(const void* q, const void* k, int B, int H, int Hkv, int N,
@@ -346,8 +352,37 @@ qattn_status qattn_attn_quantized(const int8_t* q_i8, const float* q_scale, cons
   s = check_ptrs(q_i8, q_scale, k_i8, k_scale, v, out);
   if (s != QATTN_OK) return s;
   if ((s = device_ok()) != QATTN_OK) return s;
-  return dispatch_attn(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, d, causal,
-                       reinterpret_cast<cudaStream_t>(stream));
+  return dispatch_attn<false>(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, d, causal,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+qattn_status qattn_smooth_k(const void* k, int B, int Hkv, int N, int d, int8_t* k_i8,
+                            float* k_scale, float* k_mean, void* ws, size_t ws_bytes,
+                            qattn_stream_t stream) {
+  qattn_status s = check_shape(B, Hkv, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(k, k_i8, k_scale);
+  if (s != QATTN_OK) return s;
+  if (k_mean && !aligned16(k_mean)) return QATTN_ERR_MISALIGNED;
+  if (ws == nullptr || ws_bytes < qattn_smooth_quant_workspace(B, Hkv, d))
+    return QATTN_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QATTN_ERR_MISALIGNED;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  return dispatch_smooth_quant(nullptr, k, B, Hkv, Hkv, N, d, nullptr, nullptr, k_i8, k_scale,
+                               k_mean, static_cast<long long*>(ws),
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+qattn_status qattn_attn_fused_q(const void* q, const int8_t* k_i8, const float* k_scale,
+                                const void* v, void* out, int B, int H, int Hkv, int N, int d,
+                                int causal, qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q, k_i8, k_scale, v, out);
+  if (s != QATTN_OK) return s;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  return dispatch_attn<true>(q, nullptr, k_i8, k_scale, v, out, B, H, Hkv, N, d, causal,
+                             reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t qattn_forward_workspace(int B, int H, int Hkv, int N, int d) {
@@ -373,9 +408,13 @@ qattn_status qattn_forward_ws(const void* q, const void* k, const void* v, void*
   float* q_scale = reinterpret_cast<float*>(w + L.q_scale);
   float* k_scale = reinterpret_cast<float*>(w + L.k_scale);
   long long* sums = reinterpret_cast<long long*>(w + L.sums);
+  // Smoothing + quantization of Q and K in one pass, then attention on the int8 operands.  (The
+  // variant with Q quantized inside the attention kernel, qattn_smooth_k + qattn_attn_fused_q,
+  // gives identical results but measured slower: its per-CTA quantization prologue lies on
+  // every CTA's critical path.)
   s = dispatch_smooth_quant(q, k, B, H, Hkv, N, d, q_i8, q_scale, k_i8, k_scale, nullptr, sums, st);
   if (s != QATTN_OK) return s;
-  return dispatch_attn(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, d, causal, st);
+  return dispatch_attn<false>(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, d, causal, st);
 }
 
 qattn_status qattn_forward(const void* q, const void* k, const void* v, void* out, int B, int H,

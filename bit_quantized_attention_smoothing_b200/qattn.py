@@ -27,7 +27,8 @@ KBLOCK = 64
 EXPORTS = [
     "qattn_status_string", "qattn_version", "qattn_smooth_quant_workspace", "qattn_smooth_quant",
     "qattn_smooth_quant_noalloc",
-    "qattn_attn_quantized", "qattn_forward_workspace", "qattn_forward_ws", "qattn_forward",
+    "qattn_attn_quantized", "qattn_smooth_k", "qattn_attn_fused_q",
+    "qattn_forward_workspace", "qattn_forward_ws", "qattn_forward",
     "qattn_forward_host", "qattn_debug_qk_int32", "qattn_debug_wait_timeout",
     "qattn_check_device_status",
 ]
@@ -68,6 +69,10 @@ def _lib():
         L.qattn_smooth_quant_noalloc.restype = i
         L.qattn_attn_quantized.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, P]
         L.qattn_attn_quantized.restype = i
+        L.qattn_smooth_k.argtypes = [P, i, i, i, i, P, P, P, P, sz, P]
+        L.qattn_smooth_k.restype = i
+        L.qattn_attn_fused_q.argtypes = [P, P, P, P, P, i, i, i, i, i, i, P]
+        L.qattn_attn_fused_q.restype = i
         L.qattn_forward_workspace.argtypes = [i, i, i, i, i]
         L.qattn_forward_workspace.restype = sz
         L.qattn_forward_ws.argtypes = [P, P, P, P, i, i, i, i, i, i, P, sz, P]
@@ -162,6 +167,33 @@ def qattn_attn_quantized(q_i8, q_scale, k_i8, k_scale, v, out=None, causal=False
     st = _lib().qattn_attn_quantized(_p(q_i8), _p(q_scale), _p(k_i8), _p(k_scale), _p(v), _p(out),
                                      B, H, Hkv, N, d, int(bool(causal)), _stream(stream))
     _check("qattn_attn_quantized", st)
+    return out
+
+
+def qattn_smooth_k(k, k_i8=None, k_scale=None, k_mean=None, ws=None, stream=None):
+    """K half of the pre-processing: smoothing and per-64-row-block INT8 quantization of K.
+    Returns (k_i8, k_scale, k_mean); k_mean is only written when passed."""
+    B, Hkv, N, d = k.shape
+    dev = k.device
+    nkb = -(-N // KBLOCK)
+    k_i8 = torch.empty(B, Hkv, N, d, dtype=torch.int8, device=dev) if k_i8 is None else k_i8
+    k_scale = torch.empty(B, Hkv, nkb, dtype=torch.float32, device=dev) if k_scale is None else k_scale
+    wsb = qattn_smooth_quant_workspace(B, Hkv, d)
+    if ws is None:
+        ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    st = _lib().qattn_smooth_k(_p(k), B, Hkv, N, d, _p(k_i8), _p(k_scale), _p(k_mean), _p(ws),
+                               ws.numel(), _stream(stream))
+    _check("qattn_smooth_k", st)
+    return k_i8, k_scale, k_mean
+
+
+def qattn_attn_fused_q(q, k_i8, k_scale, v, out=None, causal=False, stream=None):
+    """Attention on fp16 Q (quantized inside the kernel) and qattn_smooth_k's int8 K."""
+    B, H, Hkv, N, d = _dims(q, k_i8)
+    out = torch.empty(B, H, N, d, dtype=torch.float16, device=v.device) if out is None else out
+    st = _lib().qattn_attn_fused_q(_p(q), _p(k_i8), _p(k_scale), _p(v), _p(out), B, H, Hkv, N, d,
+                                   int(bool(causal)), _stream(stream))
+    _check("qattn_attn_fused_q", st)
     return out
 
 

@@ -110,8 +110,34 @@ qattn_status qattn_attn_quantized(const int8_t* q_i8, const float* q_scale, cons
                                   int Hkv, int N, int d, int causal, qattn_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Q quantization fused into the attention kernel: an alternative split of the forward into
+ * two calls.  Results are identical to qattn_smooth_quant + qattn_attn_quantized; on B200 it
+ * measured slower at 32K tokens (each CTA's quantization prologue lies on its critical path), so
+ * qattn_forward does not use it.
+ * ------------------------------------------------------------------------------------------ */
+
+/* K half of the pre-processing (page sec. 3): smooths K (subtracts the per-channel mean over
+ * the tokens of each batch and kv head) and quantizes K' per 64-row block.  k [B][Hkv][N][d]
+ * fp16; writes k_i8 [B][Hkv][N][d], k_scale [B][Hkv][ceil(N/64)] and, when not NULL, k_mean
+ * [B][Hkv][d].  ws: at least qattn_smooth_quant_workspace(B, Hkv, d) bytes, clobbered.  Codes
+ * and scales are bit-identical to qattn_smooth_quant's. */
+qattn_status qattn_smooth_k(const void* k, int B, int Hkv, int N, int d, int8_t* k_i8,
+                            float* k_scale, float* k_mean, void* ws, size_t ws_bytes,
+                            qattn_stream_t stream);
+
+/* Attention as qattn_attn_quantized, but on fp16 Q [B][H][N][d]: each CTA quantizes its own
+ * 128-row Q tiles (the page's per-block INT8 quantization of Q, sec. 3: scale = amax / 127,
+ * round-half-even codes, bit-identical to qattn_smooth_quant's q_i8 and q_scale) in shared
+ * memory before the first Q K^T, so Q makes one trip through HBM instead of three.  k_i8 and
+ * k_scale as written by qattn_smooth_k. */
+qattn_status qattn_attn_fused_q(const void* q, const int8_t* k_i8, const float* k_scale,
+                                const void* v, void* out, int B, int H, int Hkv, int N, int d,
+                                int causal, qattn_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * The whole forward: fp16 q, k, v in, fp16 out (the plug-and-play call of the page's dialogue
- * and sec. 2).  Smoothing + quantization, then attention.
+ * and sec. 2).  Smoothing + quantization (qattn_smooth_quant), then attention
+ * (qattn_attn_quantized).
  * ------------------------------------------------------------------------------------------ */
 
 /* Bytes of device workspace qattn_forward_ws needs (int8 Q and K, scales, channel sums). */

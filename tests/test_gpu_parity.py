@@ -118,6 +118,27 @@ def test_attention_on_oracle_codes(lib, oracle, name, over):
     assert ok, msg
 
 
+@pytest.mark.parametrize("name,over", SMALL, ids=SMALL_IDS)
+def test_fused_q_halves_match_separate_quantization(lib, name, over):
+    """The fused forward's halves: qattn_smooth_k writes the same K codes, scales and means as
+    qattn_smooth_quant, and the attention kernel that quantizes Q in its prologue gives the same
+    output, bit for bit, as the one fed qattn_smooth_quant's int8 Q (its Q codes and scales are
+    pinned to the oracle by test_smooth_quant_bit_exact_small)."""
+    w = WORKLOADS[name].with_(**over)
+    q, k, v = _inputs(w)
+    q_i8, q_s, k_i8, k_s, k_mean = lib.qattn_smooth_quant(q, k)
+    k_mean2 = torch.empty_like(k_mean)
+    k_i8b, k_sb, _ = lib.qattn_smooth_k(k, k_mean=k_mean2)
+    ref = lib.qattn_attn_quantized(q_i8, q_s, k_i8, k_s, v, causal=w.causal)
+    got = lib.qattn_attn_fused_q(q, k_i8b, k_sb, v, causal=w.causal)
+    fwd = lib.qattn_forward(q, k, v, causal=w.causal)
+    torch.cuda.synchronize()
+    assert lib.qattn_check_device_status() == 0
+    assert torch.equal(k_i8, k_i8b) and torch.equal(k_s, k_sb) and torch.equal(k_mean, k_mean2)
+    assert torch.equal(ref, got)
+    assert torch.equal(ref, fwd)
+
+
 def _planted_jumps(w):
     """Seeded inputs whose row maxima jump by far more than the lazy-rescale threshold after the
     first key tile: one direction u is added to every query, and three keys are replaced by
@@ -162,9 +183,9 @@ def test_forward_variants_agree(lib):
 @pytest.mark.parametrize("pinned", [True, False])
 def test_host_forward_pipeline_chunks(lib, pinned):
     """qattn_forward_host cuts the (batch, kv head) groups into chunks whose copies and kernels
-    overlap; 6 groups make uneven chunks.  Results must equal the device-buffer forward bit for
-    bit."""
-    w = WORKLOADS["wide64"].with_(B=2, H=6, Hkv=3, N=300, causal=True)
+    overlap; 9 groups make uneven chunks (2, 2, 2, 2, 1).  Results must equal the device-buffer
+    forward bit for bit."""
+    w = WORKLOADS["wide64"].with_(B=3, H=6, Hkv=3, N=300, causal=True)
     q, k, v = _inputs(w, "cpu")
     a = lib.qattn_forward(q.cuda(), k.cuda(), v.cuda(), causal=True)
     hq, hk, hv = (t.cpu() for t in (q, k, v))
