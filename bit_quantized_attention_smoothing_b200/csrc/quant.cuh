@@ -89,37 +89,42 @@ __device__ __forceinline__ uint32_t pack4_i8(float a, float b, float c, float d)
 
 // One quantization block of R rows x D channels, 256 threads.  src: fp16 rows of the block
 // (head base + r0 * D); mean: per-channel smoothing offsets in shared memory (K) or nullptr (Q).
+// One quantization block of R rows x D values per 256-thread CTA: x = fp16 value (minus the
+// channel mean for K), amax over the block, scale = amax / 127, codes rint(x * (1 / scale)); a
+// group of 8 values holding one within 2^-13 of a half-integer is recomputed with quant_code
+// (the correctly rounded quotient decides there), so every code is rint(x / scale).  Values stay
+// as fp16 pairs in registers between the two passes (the mean is subtracted again when needed),
+// keeping the CTA small enough for several to share an SM.
 template <int D, int R>
 __device__ __forceinline__ void quantize_block_cta(const uint16_t* __restrict__ src, int rows,
                                                    const float* mean_s, int8_t* __restrict__ dst,
                                                    float* __restrict__ scale_out, float* red) {
   constexpr int VPR = D / 8;
   constexpr int VPT = R * VPR / 256;  // vectors per thread
+  static_assert(256 % VPR == 0, "a thread keeps one column group");
   const int tid = threadIdx.x;
   const int cg = tid % VPR;
-  float x[VPT][8];
   float m[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) m[e] = mean_s ? mean_s[cg * 8 + e] : 0.0f;
-  float amax = 0.0f;
+  // every load issued before any is used: rows past the block's end read its first row and are
+  // dropped afterwards
+  uint4 v[VPT];
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int vi = tid + i * 256;
-    const int r = vi / VPR;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < rows) v = __ldg(reinterpret_cast<const uint4*>(src) + vi);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    v[i] = __ldg(reinterpret_cast<const uint4*>(src) + (vi / VPR < rows ? vi : cg));
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    if ((tid + i * 256) / VPR >= rows) continue;
+    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      x[i][2 * e] = half_bits_to_float(w[e] & 0xFFFFu) - m[2 * e];
-      x[i][2 * e + 1] = half_bits_to_float(w[e] >> 16) - m[2 * e + 1];
+      amax = fmaxf(amax, fabsf(half_bits_to_float(w[e] & 0xFFFFu) - m[2 * e]));
+      amax = fmaxf(amax, fabsf(half_bits_to_float(w[e] >> 16) - m[2 * e + 1]));
     }
-    if (r >= rows) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[i][e] = 0.0f;
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[i][e]));
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
@@ -134,23 +139,37 @@ __device__ __forceinline__ void quantize_block_cta(const uint16_t* __restrict__ 
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int vi = tid + i * 256;
-    const int r = vi / VPR;
-    if (r < rows) {
+    const bool in = vi / VPR < rows;
+    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+    float x[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      x[2 * e] = half_bits_to_float(w[e] & 0xFFFFu) - m[2 * e];
+      x[2 * e + 1] = half_bits_to_float(w[e] >> 16) - m[2 * e + 1];
+    }
+    int r[8];
+    bool near_tie = false;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float y = x[e] * rcp;
+      const float ry = rintf(y);
+      near_tie |= fabsf(y - ry) > 0.4998779296875f;  // within 2^-13 of a half-integer
+      r[e] = static_cast<int>(ry);
+    }
+    uint2 out;
+    out.x = __byte_perm(__byte_perm(r[0], r[1], 0x0040), __byte_perm(r[2], r[3], 0x0040), 0x5410);
+    out.y = __byte_perm(__byte_perm(r[4], r[5], 0x0040), __byte_perm(r[6], r[7], 0x0040), 0x5410);
+    if (__any_sync(0xFFFFFFFFu, near_tie) && near_tie) {
       float q[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) q[e] = amax > 0.0f ? quant_code(x[i][e], s, rcp) : 0.0f;
-      uint2 out;
+      for (int e = 0; e < 8; ++e) q[e] = quant_code(x[e], s, rcp);
       out.x = pack4_i8(q[0], q[1], q[2], q[3]);
       out.y = pack4_i8(q[4], q[5], q[6], q[7]);
-      reinterpret_cast<uint2*>(dst)[vi] = out;
     }
+    if (in) reinterpret_cast<uint2*>(dst)[vi] = out;
   }
 }
 
-// Quantizes every Q block and every K' block in one launch: blocks [0, nq) are Q blocks in
-// (b*H + h, block) order, blocks [nq, nq + nk) are K blocks in (b*Hkv + g, block) order.
-// 256 threads.  For K blocks the CTA first forms the channel means of its kv head from the
-// exact sums; the first K block of each kv head also writes them to k_mean (if not null).
 template <int D>
 __global__ void __launch_bounds__(256) quantize_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, int N, int nqb, int nkb,
