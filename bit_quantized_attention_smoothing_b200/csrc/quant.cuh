@@ -178,7 +178,9 @@ __global__ void __launch_bounds__(256) quantize_kernel(
     float* __restrict__ k_mean) {
   __shared__ float mean_s[D];
   __shared__ float red[8];
-  const long long blk = blockIdx.x;
+  // K blocks first: the channel-sum pass has just read K, so its second read mostly hits L2
+  const long long nk = static_cast<long long>(gridDim.x) - nq;
+  const long long blk = blockIdx.x < nk ? nq + blockIdx.x : blockIdx.x - nk;
   if (blk < nq) {
     const long long bh = blk / nqb;
     const int qb = static_cast<int>(blk % nqb);
