@@ -32,7 +32,7 @@ METRIC = "quantized attention fwd TOPS (4·B·H·N²·d/s) and % of B200 INT8 te
 DEFAULT_WORKLOAD = "llama8b_32k"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-ATTN_KERNEL_SOURCES = ["attn_sm100.cuh", "sm100_ptx.cuh", "quant.cuh"]
+ATTN_KERNEL_SOURCES = ["attn_sm100.cuh", "sm100_ptx.cuh"]  # the timed kernel (int8 Q) uses no other source
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_sm100_llama8b_32k.md")
 
 
