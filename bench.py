@@ -202,6 +202,25 @@ def oracle_sample_run(w, q, k, v, target_s):
 # our arm
 # ------------------------------------------------------------------------------------------------
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest of every rank's value (host plumbing: one all-reduce of a scalar over the
+    process group the caller initialised; no data-path collective).  A single rank returns its
+    own value."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_tops(ops_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank processes one full workload per step, so the job does
+    world * ops * steps operations in the slowest rank's time."""
+    return world * ops_per_step * steps / (max_ms / 1e3) / 1e12
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -266,12 +285,9 @@ def run_ours(args):
     if Q.qattn_check_device_status(stream) != 0:
         raise RuntimeError("device status reports a timed-out wait in the timed region")
 
-    t_max = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    total_ms_max = float(t_max.item())
+    total_ms_max = max_over_ranks(total_ms, world, dev)
     ops = w.ops
-    value = world * ops * K / (total_ms_max / 1e3) / 1e12
+    value = weak_scaling_tops(ops, K, world, total_ms_max)
 
     # end to end through the C ABI on host buffers (H2D of q, k, v and D2H of out inside)
     qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
@@ -286,10 +302,8 @@ def run_ours(args):
         Q.qattn_forward_host(qh, kh, vh, oh, w.causal, stream)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = world * ops * ke / (float(e2e_ms.item()) / 1e3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = weak_scaling_tops(ops, ke, world, e2e_ms)
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = oh.numel() * oh.element_size()
 
