@@ -63,6 +63,15 @@ def lib():
         L.oracle_attention_quantized.restype = i
         L.oracle_attention_fp64.argtypes = [P, P, P, i, i, i, i, i, i, i, P, P, ctypes.c_long, P, i]
         L.oracle_attention_fp64.restype = i
+        L.oracle_attention_quantized_sparse.argtypes = [P, P, P, P, P, i, i, i, i, i, i, P, P, P,
+                                                        ctypes.c_long, P, i]
+        L.oracle_attention_quantized_sparse.restype = i
+        L.oracle_block_means.argtypes = [P, ctypes.c_long, i, i, i, P]
+        L.oracle_block_means.restype = None
+        L.oracle_block_scores.argtypes = [P, P, i, i, i, i, i, i, P]
+        L.oracle_block_scores.restype = None
+        L.oracle_select_blocks.argtypes = [P, i, i, i, i, i, P, P]
+        L.oracle_select_blocks.restype = None
         _lib = L
     return _lib
 
@@ -165,6 +174,74 @@ def attention_quantized(q_i8, q_scale, k_i8, k_scale, v, B, H, Hkv, N, d, causal
     lib().oracle_attention_quantized(_ptr(q_i8), _ptr(q_scale), _ptr(k_i8), _ptr(k_scale), _ptr(v),
                                      B, H, Hkv, N, d, 1 if causal else 0, _ptr(row_bh),
                                      _ptr(row_i), row_bh.size, _ptr(out), int(nthreads))
+    return out
+
+
+SBLOCK = 256  # block-sparse selection: query rows per selection block
+KTILE = 128   # block-sparse selection: keys per key tile
+
+
+def block_means(x, outer, N, d, rows_per_block):
+    """Exact per-block channel means (float64 [outer, nblocks, d]) of fp16 x [outer, N, d]."""
+    nb = -(-N // rows_per_block)
+    out = np.zeros((outer, nb, d), dtype=np.float64)
+    lib().oracle_block_means(_ptr(_bits16(x)), outer, N, d, rows_per_block, _ptr(out))
+    return out
+
+
+def block_scores(qmeans, kmeans, B, H, Hkv, d):
+    """Importance of each (query block, key tile) pair: float64 [B*H, nsb, nkt]."""
+    qmeans = np.ascontiguousarray(qmeans, dtype=np.float64)
+    kmeans = np.ascontiguousarray(kmeans, dtype=np.float64)
+    nsb, nkt = qmeans.shape[1], kmeans.shape[1]
+    out = np.zeros((B * H, nsb, nkt), dtype=np.float64)
+    lib().oracle_block_scores(_ptr(qmeans), _ptr(kmeans), B, H, Hkv, nsb, nkt, d, _ptr(out))
+    return out
+
+
+def select_blocks(scores, B, H, N, causal, topk):
+    """(list int32 [B*H, nsb, nkt], count int32 [B*H, nsb]): the selected key tiles of each query
+    block, ascending (entries past count are unused)."""
+    scores = np.ascontiguousarray(scores, dtype=np.float64)
+    nsb, nkt = scores.shape[1], scores.shape[2]
+    lst = np.full((B * H, nsb, nkt), -1, dtype=np.int32)
+    cnt = np.zeros((B * H, nsb), dtype=np.int32)
+    lib().oracle_select_blocks(_ptr(scores), B, H, N, 1 if causal else 0, int(topk), _ptr(lst),
+                               _ptr(cnt))
+    return lst, cnt
+
+
+def block_select(q, k, B, H, Hkv, N, d, causal, topk):
+    """The whole selection from fp16 q, k: means, scores, top-k lists."""
+    qm = block_means(q, B * H, N, d, SBLOCK)
+    km = block_means(k, B * Hkv, N, d, KTILE)
+    return select_blocks(block_scores(qm, km, B, H, Hkv, d), B, H, N, causal, topk)
+
+
+def tile_mask(lst, cnt, N):
+    """uint8 [B*H, nsb, nkt] mask of the selected key tiles."""
+    nkt = -(-N // KTILE)
+    mask = np.zeros(lst.shape[:2] + (nkt,), dtype=np.uint8)
+    for bh in range(lst.shape[0]):
+        for i in range(lst.shape[1]):
+            mask[bh, i, lst[bh, i, :cnt[bh, i]]] = 1
+    return mask
+
+
+def attention_quantized_sparse(q_i8, q_scale, k_i8, k_scale, v, B, H, Hkv, N, d, causal, mask,
+                               rows=None, nthreads=0):
+    """attention_quantized with query row i of head bh seeing only the key tiles with
+    mask[bh, i // 256, tile] != 0."""
+    row_bh, row_i = all_rows(B, H, N) if rows is None else rows
+    row_bh = np.ascontiguousarray(row_bh, dtype=np.int64)
+    row_i = np.ascontiguousarray(row_i, dtype=np.int64)
+    out = np.zeros((row_bh.size, d), dtype=np.float64)
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    lib().oracle_attention_quantized_sparse(
+        _ptr(np.ascontiguousarray(q_i8, dtype=np.int8)), _ptr(np.ascontiguousarray(q_scale, dtype=np.float32)),
+        _ptr(np.ascontiguousarray(k_i8, dtype=np.int8)), _ptr(np.ascontiguousarray(k_scale, dtype=np.float32)),
+        _ptr(_bits16(v)), B, H, Hkv, N, d, 1 if causal else 0, _ptr(mask), _ptr(row_bh), _ptr(row_i),
+        row_bh.size, _ptr(out), int(nthreads))
     return out
 
 

@@ -44,6 +44,8 @@
 
 #define ORACLE_QBLOCK 128
 #define ORACLE_KBLOCK 64
+#define ORACLE_SBLOCK 256  /* block-sparse selection: query rows per selection block */
+#define ORACLE_KTILE 128   /* block-sparse selection: keys per key tile */
 
 /* ------------------------------------------------------------------------------------------------
  * IEEE 754 binary16, written from the format's definition: 1 sign bit, 5 exponent bits (bias 15),
@@ -214,6 +216,7 @@ typedef struct {
     const uint16_t* v16;
     int B, H, Hkv, N, d, causal, quantized;
     const int64_t* row_bh; const int64_t* row_i; long nrows;
+    const uint8_t* tile_mask;  /* block-sparse mode: [B*H][ceil(N/256)][ceil(N/128)], or NULL */
     double* out;
     double* kmean64;   /* full-precision mode: exact per-channel means, [B*Hkv, d] */
     long next;         /* work counter */
@@ -230,6 +233,12 @@ static void attn_one_row(attn_job* J, long r, double* s, double* acc) {
     int nvis = J->causal ? i + 1 : N;
     double inv_sqrt_d = 1.0 / sqrt((double)d);
     double m = -INFINITY;
+    /* block-sparse mode: keys of unselected 128-key tiles are left out (weight 0) */
+    const uint8_t* sel = NULL;
+    if (J->tile_mask) {
+        int nsb = (N + ORACLE_SBLOCK - 1) / ORACLE_SBLOCK, nkt = (N + ORACLE_KTILE - 1) / ORACLE_KTILE;
+        sel = J->tile_mask + (bh * nsb + i / ORACLE_SBLOCK) * (long)nkt;
+    }
     if (J->quantized) {
         int nkb = (N + ORACLE_KBLOCK - 1) / ORACLE_KBLOCK;
         int nqb = (N + ORACLE_QBLOCK - 1) / ORACLE_QBLOCK;
@@ -241,6 +250,7 @@ static void attn_one_row(attn_job* J, long r, double* s, double* acc) {
             for (int c = 0; c < d; ++c) acc32 += (int32_t)qrow[c] * (int32_t)krow[c];
             double sk = (double)J->k_scale[bg * nkb + j / ORACLE_KBLOCK];
             s[j] = (double)acc32 * sq * sk * inv_sqrt_d;
+            if (sel && !sel[j / ORACLE_KTILE]) s[j] = -INFINITY;
             if (s[j] > m) m = s[j];
         }
     } else {
@@ -258,7 +268,7 @@ static void attn_one_row(attn_job* J, long r, double* s, double* acc) {
         }
     }
     double l = 0.0;
-    for (int j = 0; j < nvis; ++j) { s[j] = exp(s[j] - m); l += s[j]; }
+    for (int j = 0; j < nvis; ++j) { s[j] = s[j] == -INFINITY ? 0.0 : exp(s[j] - m); l += s[j]; }
     for (int c = 0; c < d; ++c) acc[c] = 0.0;
     for (int j = 0; j < nvis; ++j) {
         const uint16_t* vrow = J->v16 + (bg * N + j) * (long)d;
@@ -315,6 +325,23 @@ int oracle_attention_quantized(const int8_t* q_i8, const float* q_scale, const i
     return nthreads;
 }
 
+/* oracle_attention_quantized restricted to selected key tiles: query row i of head bh sees key
+ * j only if tile_mask[bh][i / 256][j / 128] != 0 (and j <= i when causal). */
+int oracle_attention_quantized_sparse(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                                      const float* k_scale, const uint16_t* v, int B, int H,
+                                      int Hkv, int N, int d, int causal, const uint8_t* tile_mask,
+                                      const int64_t* row_bh, const int64_t* row_i, long nrows,
+                                      double* out, int nthreads) {
+    attn_job J;
+    memset(&J, 0, sizeof(J));
+    J.q_i8 = q_i8; J.q_scale = q_scale; J.k_i8 = k_i8; J.k_scale = k_scale; J.v16 = v;
+    J.B = B; J.H = H; J.Hkv = Hkv; J.N = N; J.d = d; J.causal = causal; J.quantized = 1;
+    J.row_bh = row_bh; J.row_i = row_i; J.nrows = nrows; J.out = out; J.tile_mask = tile_mask;
+    if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    run_rows(&J, nthreads);
+    return nthreads;
+}
+
 /* Full-precision attention rows, softmax(Q K'^T / sqrt(d)) V in binary64 from the fp16 inputs,
  * with K' = K - (exact binary64 per-channel mean) when smooth != 0, else K' = K.  This is the
  * unquantized reference the quantized result is measured against. */
@@ -339,4 +366,82 @@ int oracle_attention_fp64(const uint16_t* q, const uint16_t* k, const uint16_t* 
     run_rows(&J, nthreads);
     free(J.kmean64);
     return nthreads;
+}
+
+/* ------------------------------------------------------------------------------------------------
+ * Block importance and selection for block-sparse attention.  The page "ThriftAttention:
+ * Selective Mixed Precision for Long-Context FP4 Attention" (gist.science, technical summary,
+ * method, heuristic block selection) scores each (query block, key block) pair by the dot
+ * product of the two blocks' mean vectors and singles out the top-k pairs; its results section
+ * compares against sparse top-k attention, which computes those pairs and drops the rest.  That
+ * dropping variant is what is built here.  Readings: query blocks of 256 rows (a pair of
+ * 128-row attention tiles), key blocks of 128 keys (one key tile); means taken over the block's
+ * rows that exist (< N) of the fp16 inputs, exactly (int64 fixed point, one binary64 rounding);
+ * score = sum over channels c = 0..d-1, in that order, of fma(qmean[c], kmean[c], acc) in
+ * binary64; per query block the candidates are the key blocks it may see (all, or those at or
+ * below its last row when causal), the diagonal key blocks (its own rows' tiles) are always
+ * kept when causal, and the topk highest-scoring other candidates (ties to the lower index)
+ * are added; the list is in ascending order.  The means of K are taken on K itself: subtracting
+ * the channel mean would shift every score of a query block by the same amount.
+ * ---------------------------------------------------------------------------------------------- */
+
+/* means[o][blk][c] of x[o][n][c] over rows n of block blk (rows_per_block rows, the last one
+ * shorter when N is not a multiple). */
+void oracle_block_means(const uint16_t* x, long outer, int N, int d, int rows_per_block,
+                        double* means) {
+    int nb = (N + rows_per_block - 1) / rows_per_block;
+    for (long o = 0; o < outer; ++o)
+        for (int blk = 0; blk < nb; ++blk) {
+            int n0 = blk * rows_per_block;
+            int n1 = n0 + rows_per_block < N ? n0 + rows_per_block : N;
+            for (int c = 0; c < d; ++c) {
+                int64_t sum = 0;
+                for (int n = n0; n < n1; ++n) sum += k_fixed(x[(o * N + n) * (long)d + c]);
+                means[(o * nb + blk) * (long)d + c] = (double)sum / ((double)(n1 - n0) * 16777216.0);
+            }
+        }
+}
+
+/* scores[bh][i][j] = qmeans[bh][i] . kmeans[bh's kv head][j], fma chain over c in order. */
+void oracle_block_scores(const double* qmeans, const double* kmeans, int B, int H, int Hkv, int nsb,
+                         int nkt, int d, double* scores) {
+    for (long bh = 0; bh < (long)B * H; ++bh) {
+        long bg = (bh / H) * Hkv + (bh % H) / (H / Hkv);
+        for (int i = 0; i < nsb; ++i)
+            for (int j = 0; j < nkt; ++j) {
+                double acc = 0.0;
+                for (int c = 0; c < d; ++c)
+                    acc = fma(qmeans[(bh * nsb + i) * (long)d + c], kmeans[(bg * nkt + j) * (long)d + c], acc);
+                scores[(bh * nsb + i) * (long)nkt + j] = acc;
+            }
+    }
+}
+
+/* list[bh][i][0 .. count[bh][i]) = the selected key tiles of query block i, ascending. */
+void oracle_select_blocks(const double* scores, int B, int H, int N, int causal, int topk,
+                          int32_t* list, int32_t* count) {
+    int nsb = (N + ORACLE_SBLOCK - 1) / ORACLE_SBLOCK, nkt = (N + ORACLE_KTILE - 1) / ORACLE_KTILE;
+    uint8_t* pick = (uint8_t*)malloc((size_t)nkt);
+    for (long bh = 0; bh < (long)B * H; ++bh)
+        for (int i = 0; i < nsb; ++i) {
+            const double* sc = scores + (bh * nsb + i) * (long)nkt;
+            int last = causal ? 2 * i + 1 : nkt - 1;       /* highest key tile the block may see */
+            if (last > nkt - 1) last = nkt - 1;
+            memset(pick, 0, (size_t)nkt);
+            if (causal)
+                for (int j = 2 * i; j <= last; ++j) pick[j] = 1;
+            for (int r = 0; r < topk; ++r) {
+                int best = -1;
+                for (int j = 0; j <= last; ++j)
+                    if (!pick[j] && (best < 0 || sc[j] > sc[best])) best = j;
+                if (best < 0) break;
+                pick[best] = 1;
+            }
+            int n = 0;
+            int32_t* out = list + (bh * nsb + i) * (long)nkt;
+            for (int j = 0; j < nkt; ++j)
+                if (pick[j]) out[n++] = j;
+            count[bh * nsb + i] = n;
+        }
+    free(pick);
 }

@@ -375,3 +375,105 @@ def test_worked_example(oracle, causal):
             w1 = 1.0 / (1.0 + math.exp(2.0 * gap))
             ref = v0 + w1 * (v1 - v0)
         np.testing.assert_allclose(out[i], ref, rtol=0, atol=1e-14)
+
+
+# ------------------------------------------------------------------------------------------------
+# Block-sparse selection (block-mean importance, top-k key tiles per 256-row query block)
+# ------------------------------------------------------------------------------------------------
+
+def test_block_means_exact_and_ragged(oracle):
+    """Means of fp16 values over blocks of rows are exact sums (every fp16 value and every
+    partial sum of <= 256 of them is representable in binary64) divided once: equal to numpy's
+    float64 mean bit for bit, including the short last block."""
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((3, 300, 16)) * rng.choice([1e-3, 1.0, 300.0], (3, 300, 16))).astype(np.float16)
+    got = oracle.block_means(x, 3, 300, 16, 128)
+    for o in range(3):
+        for b, (n0, n1) in enumerate([(0, 128), (128, 256), (256, 300)]):
+            ref = x[o, n0:n1].astype(np.float64).mean(axis=0)
+            assert np.array_equal(got[o, b], ref)
+
+
+def test_block_scores_dot_products(oracle):
+    """Scores are the dot products of the query-block and key-block means (GQA mapping of the
+    kv head): exact when every product and partial sum is a small dyadic number, and within
+    binary64 rounding of numpy's dot otherwise."""
+    rng = np.random.default_rng(6)
+    qm = rng.integers(-8, 9, (4, 3, 8)).astype(np.float64) / 4
+    km = rng.integers(-8, 9, (2, 5, 8)).astype(np.float64) / 8
+    s = oracle.block_scores(qm, km, 1, 4, 2, 8)
+    for bh in range(4):
+        assert np.array_equal(s[bh], qm[bh] @ km[bh // 2].T)
+    qm = rng.standard_normal((4, 3, 64))
+    km = rng.standard_normal((2, 5, 64))
+    s = oracle.block_scores(qm, km, 1, 4, 2, 64)
+    for bh in range(4):
+        np.testing.assert_allclose(s[bh], qm[bh] @ km[bh // 2].T, rtol=1e-12, atol=1e-12)
+
+
+def _select_bruteforce(scores, N, causal, topk):
+    nsb, nkt = scores.shape
+    out = []
+    for i in range(nsb):
+        last = min(2 * i + 1, nkt - 1) if causal else nkt - 1
+        forced = set(range(2 * i, last + 1)) if causal else set()
+        cand = sorted((j for j in range(last + 1) if j not in forced), key=lambda j: (-scores[i, j], j))
+        out.append(sorted(forced | set(cand[:topk])))
+    return out
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N,topk", [(1000, 2), (1000, 0), (1000, 50), (257, 1), (128, 3)])
+def test_select_blocks_bruteforce(oracle, causal, N, topk):
+    """Selection against a plain Python ranking (score descending, lower index first on ties):
+    the diagonal tiles of a causal block are always in, then the topk best other tiles it may
+    see; lists ascending.  Scores drawn from a few values so that ties occur."""
+    rng = np.random.default_rng(N + topk)
+    nsb, nkt = -(-N // 256), -(-N // 128)
+    scores = rng.integers(0, 4, (3, nsb, nkt)).astype(np.float64)
+    lst, cnt = oracle.select_blocks(scores, 1, 3, N, causal, topk)
+    for bh in range(3):
+        ref = _select_bruteforce(scores[bh], N, causal, topk)
+        for i in range(nsb):
+            assert list(lst[bh, i, :cnt[bh, i]]) == ref[i]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sparse_attention_all_tiles_is_dense(oracle, causal):
+    """With every tile a query block may see selected, the block-sparse attention is the dense
+    quantized attention, bit for bit."""
+    w = WORKLOADS["tiny"].with_(B=1, H=2, Hkv=1, N=300, causal=causal)
+    q, k, v = make_inputs(w)
+    sq = oracle.smooth_quant(_np16(q), _np16(k), w.B, w.H, w.Hkv, w.N, w.d)
+    lst, cnt = oracle.block_select(_np16(q), _np16(k), w.B, w.H, w.Hkv, w.N, w.d, causal, 10**6)
+    mask = oracle.tile_mask(lst, cnt, w.N)
+    args = (sq["q_i8"], sq["q_scale"], sq["k_i8"], sq["k_scale"], _np16(v), w.B, w.H, w.Hkv, w.N, w.d, causal)
+    dense = oracle.attention_quantized(*args)
+    sparse = oracle.attention_quantized_sparse(*args, mask)
+    assert np.array_equal(dense, sparse)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sparse_attention_bruteforce(oracle, causal):
+    """Block-sparse attention against a plain numpy softmax over the int8 scores with the keys
+    of unselected tiles removed."""
+    w = WORKLOADS["tiny"].with_(B=1, H=2, Hkv=1, N=640, d=64, causal=causal)
+    q, k, v = make_inputs(w)
+    sq = oracle.smooth_quant(_np16(q), _np16(k), w.B, w.H, w.Hkv, w.N, w.d)
+    lst, cnt = oracle.block_select(_np16(q), _np16(k), w.B, w.H, w.Hkv, w.N, w.d, causal, 1)
+    mask = oracle.tile_mask(lst, cnt, w.N)
+    assert mask.sum() < mask.size  # something is dropped
+    got = oracle.attention_quantized_sparse(sq["q_i8"], sq["q_scale"], sq["k_i8"], sq["k_scale"],
+                                            _np16(v), w.B, w.H, w.Hkv, w.N, w.d, causal, mask)
+    vv = _np16(v).view(np.float16).astype(np.float64)
+    for bh in range(2):
+        s = sq["q_i8"][0, bh].astype(np.int64) @ sq["k_i8"][0, 0].astype(np.int64).T
+        s = s * sq["q_scale"][0, bh][np.arange(w.N) // 128, None].astype(np.float64)
+        s = s * sq["k_scale"][0, 0][np.arange(w.N) // 64][None, :].astype(np.float64) / math.sqrt(w.d)
+        keep = mask[bh][np.arange(w.N)[:, None] // 256, np.arange(w.N)[None, :] // 128].astype(bool)
+        if causal:
+            keep &= np.tril(np.ones((w.N, w.N), dtype=bool))
+        s = np.where(keep, s, -np.inf)
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        ref = (p @ vv[0, 0]) / p.sum(axis=1, keepdims=True)
+        np.testing.assert_allclose(got[bh * w.N:(bh + 1) * w.N], ref, rtol=0, atol=1e-12)
