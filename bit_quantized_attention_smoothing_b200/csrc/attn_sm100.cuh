@@ -362,7 +362,8 @@ template <int D, bool CAUSAL, bool QF16>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scale,
-                    const uint16_t* __restrict__ q16,
+                    const uint16_t* __restrict__ q16, const int* __restrict__ kv_list,
+                    const int* __restrict__ kv_count,
                     const float* __restrict__ k_scale, __half* __restrict__ out, int B, int H,
                     int Hkv, int N, float scale_log2) {
   using Cfg = AttnCfg<D>;
@@ -393,9 +394,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int bg = b * Hkv + g;
   const int tq0 = 2 * pair, tq1 = 2 * pair + 1;
   const bool has1 = tq1 < nqt;
-  const int nw0 = CAUSAL ? tq0 + 1 : nkt;
-  const int nw1 = has1 ? (CAUSAL ? tq1 + 1 : nkt) : 0;
+  // Block-sparse: the CTA streams only the key tiles listed for its 256 query rows (ascending;
+  // kv_list null = all of them).  Causal lists end with the diagonal tiles tq0, tq1 (when they
+  // exist); tile 0 stops before tq1.
+  const int* klist = kv_list ? kv_list + (static_cast<size_t>(bh) * npairs + pair) * nkt : nullptr;
+  int nw0, nw1;
+  if (klist) {
+    const int cnt = kv_count[static_cast<size_t>(bh) * npairs + pair];
+    nw1 = has1 ? cnt : 0;
+    nw0 = (CAUSAL && cnt > 0 && __ldg(klist + cnt - 1) > tq0) ? cnt - 1 : cnt;
+  } else {
+    nw0 = CAUSAL ? tq0 + 1 : nkt;
+    nw1 = has1 ? (CAUSAL ? tq1 + 1 : nkt) : 0;
+  }
   const int n_kv = max(nw0, nw1);
+  auto ktile = [&](int j) -> int { return klist ? __ldg(klist + j) : j; };
 
   if (threadIdx.x == 0) {
     // QF16: one arrive per softmax warp once its rows of the Q tiles are in shared memory
@@ -439,11 +452,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t u = static_cast<uint32_t>(j / ST);
         if (!mbar_wait(&bars->kv_empty[s], (u & 1u) ^ 1u, abort)) break;
         mbar_arrive_expect_tx(&bars->kv_full[s], Cfg::kKTile + Cfg::kVTile);
-        tma_load_3d(smem + Cfg::kOffK + s * Cfg::kKTile, &tm_k, &bars->kv_full[s], 0, j * kBN, bg);
+        const int kt = ktile(j);
+        tma_load_3d(smem + Cfg::kOffK + s * Cfg::kKTile, &tm_k, &bars->kv_full[s], 0, kt * kBN, bg);
         uint8_t* vdst = smem + Cfg::kOffV + s * Cfg::kVTile;
 #pragma unroll
         for (int x = 0; x < D / 64; ++x)
-          tma_load_3d(vdst + x * Cfg::kVBox, &tm_v, &bars->kv_full[s], x * 64, j * kBN, bg);
+          tma_load_3d(vdst + x * Cfg::kVBox, &tm_v, &bars->kv_full[s], x * 64, kt * kBN, bg);
       }
     } else if (warp == kMmaWarp) {
       // ---------------------------------------------------------------- MMA issuer
@@ -541,11 +555,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t o_tm = tmem + lane_off + 256 + wt * D;
       float m = -INFINITY, l = 0.0f;
       bool ok = true;
-      float ks0 = __ldg(ksc);
-      float ks1 = nkb > 1 ? __ldg(ksc + 1) : 0.0f;
+      int kt = ktile(0);
+      float ks0 = __ldg(ksc + 2 * kt);
+      float ks1 = 2 * kt + 1 < nkb ? __ldg(ksc + 2 * kt + 1) : 0.0f;
       for (int j = 0; j < nt; ++j) {
-        const float nks0 = (2 * j + 2 < nkb) ? __ldg(ksc + 2 * j + 2) : 0.0f;
-        const float nks1 = (2 * j + 3 < nkb) ? __ldg(ksc + 2 * j + 3) : 0.0f;
+        const int nkt_next = j + 1 < nt ? ktile(j + 1) : 0;
+        const float nks0 = (2 * nkt_next < nkb) ? __ldg(ksc + 2 * nkt_next) : 0.0f;
+        const float nks1 = (2 * nkt_next + 1 < nkb) ? __ldg(ksc + 2 * nkt_next + 1) : 0.0f;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full[wt], static_cast<uint32_t>(j) & 1u, abort));
         if (!ok) break;
         tc_fence_after();
@@ -554,12 +570,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int c = 0; c < 4; ++c) tmem_ld32(s_tm + c * 32, sr[c]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
-        int lim = N - 1 - j * kBN;
-        if (CAUSAL && j == t) lim = min(lim, row);
+        int lim = N - 1 - kt * kBN;
+        if (CAUSAL && kt == t) lim = min(lim, row);
         const float c0 = sq * ks0 * scale_log2;
         const float c1 = sq * ks1 * scale_log2;
         ks0 = nks0;
         ks1 = nks1;
+        kt = nkt_next;
         // warp-uniform, so that every lane runs the same tensor-memory access sequence
         const bool masked = __any_sync(0xFFFFFFFFu, lim < kBN - 1);
         float alpha;

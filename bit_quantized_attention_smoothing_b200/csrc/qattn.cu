@@ -14,6 +14,7 @@
 #include "qattn.h"
 #include "attn_sm100.cuh"
 #include "quant.cuh"
+#include "block_sparse.cuh"
 
 namespace {
 
@@ -160,7 +161,8 @@ qattn_status run_smooth_quant(const void* q, const void* k, int B, int H, int Hk
 template <int D, bool CAUSAL, bool QF16>
 qattn_status run_attn(const void* q, const float* q_scale, const int8_t* k_i8,
                       const float* k_scale, const void* v, void* out, int B, int H, int Hkv,
-                      int N, cudaStream_t st) {
+                      int N, cudaStream_t st, const int* kv_list = nullptr,
+                      const int* kv_count = nullptr) {
   CUtensorMap tq, tk, tv;
   std::memset(&tq, 0, sizeof(tq));  // unused by the QF16 kernel
   if ((!QF16 && !make_i8_map(&tq, q, D, N, static_cast<long long>(B) * H)) ||
@@ -186,7 +188,7 @@ qattn_status run_attn(const void* q, const float* q_scale, const int8_t* k_i8,
   if (grid > 0x7FFFFFFFLL) return QATTN_ERR_UNSUPPORTED;
   const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   kern<<<static_cast<unsigned>(grid), kAttnThreads, Cfg::kSmemBytes, st>>>(
-      tq, tk, tv, q_scale, QF16 ? static_cast<const uint16_t*>(q) : nullptr, k_scale,
+      tq, tk, tv, q_scale, QF16 ? static_cast<const uint16_t*>(q) : nullptr, kv_list, kv_count, k_scale,
       static_cast<__half*>(out), B, H, Hkv, N, scale_log2);
   return launch_status();
 }
@@ -194,12 +196,61 @@ qattn_status run_attn(const void* q, const float* q_scale, const int8_t* k_i8,
 template <bool QF16>
 qattn_status dispatch_attn(const void* q, const float* q_scale, const int8_t* k_i8,
                            const float* k_scale, const void* v, void* out, int B, int H, int Hkv,
-                           int N, int d, int causal, cudaStream_t st) {
+                           int N, int d, int causal, cudaStream_t st, const int* kv_list = nullptr,
+                           const int* kv_count = nullptr) {
   if (d == 128)
-    return causal ? run_attn<128, true, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st)
-                  : run_attn<128, false, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st);
-  return causal ? run_attn<64, true, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st)
-                : run_attn<64, false, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st);
+    return causal ? run_attn<128, true, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, kv_list, kv_count)
+                  : run_attn<128, false, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, kv_list, kv_count);
+  return causal ? run_attn<64, true, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, kv_list, kv_count)
+                : run_attn<64, false, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, kv_list, kv_count);
+}
+
+// Block selection workspace: query-block means, key-tile means, scores (binary64).
+struct SelLayout {
+  int nsb, nkt;
+  size_t qmeans, kmeans, scores, total;
+};
+
+SelLayout sel_layout(int B, int H, int Hkv, int N, int d) {
+  SelLayout L;
+  L.nsb = (N + kSelQRows - 1) / kSelQRows;
+  L.nkt = (N + kSelKRows - 1) / kSelKRows;
+  size_t off = 0;
+  L.qmeans = off;
+  off = align_up(off + sizeof(double) * B * H * L.nsb * d);
+  L.kmeans = off;
+  off = align_up(off + sizeof(double) * B * Hkv * L.nkt * d);
+  L.scores = off;
+  off = align_up(off + sizeof(double) * B * H * static_cast<size_t>(L.nsb) * L.nkt);
+  L.total = off;
+  return L;
+}
+
+template <int D>
+qattn_status run_block_select(const void* q, const void* k, int B, int H, int Hkv, int N,
+                              int causal, int topk, int* list, int* count, uint8_t* ws,
+                              cudaStream_t st) {
+  const SelLayout L = sel_layout(B, H, Hkv, N, D);
+  double* qm = reinterpret_cast<double*>(ws + L.qmeans);
+  double* km = reinterpret_cast<double*>(ws + L.kmeans);
+  double* sc = reinterpret_cast<double*>(ws + L.scores);
+  if (static_cast<long long>(B) * H > 65535 * 1024LL) return QATTN_ERR_UNSUPPORTED;
+  block_means_kernel<D><<<dim3(B * H, L.nsb), 256, 0, st>>>(static_cast<const uint16_t*>(q), N,
+                                                           kSelQRows, qm);
+  block_means_kernel<D><<<dim3(B * Hkv, L.nkt), 256, 0, st>>>(static_cast<const uint16_t*>(k), N,
+                                                             kSelKRows, km);
+  if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
+  const int smem = 2 * kScoreTile * D * static_cast<int>(sizeof(double));
+  if (cudaFuncSetAttribute(block_scores_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return QATTN_ERR_CUDA;
+  if (B * H > 65535) return QATTN_ERR_UNSUPPORTED;
+  dim3 gs((L.nkt + kScoreTile - 1) / kScoreTile, (L.nsb + kScoreTile - 1) / kScoreTile, B * H);
+  block_scores_kernel<D><<<gs, 256, smem, st>>>(qm, km, H, Hkv, L.nsb, L.nkt, sc);
+  if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
+  block_select_kernel<<<dim3(L.nsb, B * H), 256, L.nkt, st>>>(sc, L.nsb, L.nkt, causal, topk,
+                                                              list, count);
+  return launch_status();
 }
 
 qattn_status dispatch_smooth_quant(const void* q, const void* k, int B, int H, int Hkv, int N,
@@ -371,6 +422,42 @@ qattn_status qattn_smooth_k(const void* k, int B, int Hkv, int N, int d, int8_t*
   return dispatch_smooth_quant(nullptr, k, B, Hkv, Hkv, N, d, nullptr, nullptr, k_i8, k_scale,
                                k_mean, static_cast<long long*>(ws),
                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t qattn_block_select_workspace(int B, int H, int Hkv, int N, int d) {
+  if (check_shape(B, H, Hkv, N, d) != QATTN_OK) return 0;
+  return sel_layout(B, H, Hkv, N, d).total;
+}
+
+qattn_status qattn_block_select(const void* q, const void* k, int B, int H, int Hkv, int N, int d,
+                                int causal, int topk, int* kv_list, int* kv_count, void* ws,
+                                size_t ws_bytes, qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q, k, kv_list, kv_count);
+  if (s != QATTN_OK) return s;
+  if (topk < 0) return QATTN_ERR_INVALID_ARG;
+  if (ws == nullptr || ws_bytes < sel_layout(B, H, Hkv, N, d).total) return QATTN_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QATTN_ERR_MISALIGNED;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  return d == 128 ? run_block_select<128>(q, k, B, H, Hkv, N, causal, topk, kv_list, kv_count, w, st)
+                  : run_block_select<64>(q, k, B, H, Hkv, N, causal, topk, kv_list, kv_count, w, st);
+}
+
+qattn_status qattn_attn_quantized_sparse(const int8_t* q_i8, const float* q_scale,
+                                         const int8_t* k_i8, const float* k_scale, const void* v,
+                                         void* out, int B, int H, int Hkv, int N, int d,
+                                         int causal, const int* kv_list, const int* kv_count,
+                                         qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q_i8, q_scale, k_i8, k_scale, v, out, kv_list, kv_count);
+  if (s != QATTN_OK) return s;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  return dispatch_attn<false>(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, d, causal,
+                              reinterpret_cast<cudaStream_t>(stream), kv_list, kv_count);
 }
 
 qattn_status qattn_attn_fused_q(const void* q, const int8_t* k_i8, const float* k_scale,

@@ -28,6 +28,7 @@ EXPORTS = [
     "qattn_status_string", "qattn_version", "qattn_smooth_quant_workspace", "qattn_smooth_quant",
     "qattn_smooth_quant_noalloc",
     "qattn_attn_quantized", "qattn_smooth_k", "qattn_attn_fused_q",
+    "qattn_block_select_workspace", "qattn_block_select", "qattn_attn_quantized_sparse",
     "qattn_forward_workspace", "qattn_forward_ws", "qattn_forward",
     "qattn_forward_host", "qattn_debug_qk_int32", "qattn_debug_wait_timeout",
     "qattn_check_device_status",
@@ -73,6 +74,12 @@ def _lib():
         L.qattn_smooth_k.restype = i
         L.qattn_attn_fused_q.argtypes = [P, P, P, P, P, i, i, i, i, i, i, P]
         L.qattn_attn_fused_q.restype = i
+        L.qattn_block_select_workspace.argtypes = [i, i, i, i, i]
+        L.qattn_block_select_workspace.restype = sz
+        L.qattn_block_select.argtypes = [P, P, i, i, i, i, i, i, i, P, P, P, sz, P]
+        L.qattn_block_select.restype = i
+        L.qattn_attn_quantized_sparse.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, P, P, P]
+        L.qattn_attn_quantized_sparse.restype = i
         L.qattn_forward_workspace.argtypes = [i, i, i, i, i]
         L.qattn_forward_workspace.restype = sz
         L.qattn_forward_ws.argtypes = [P, P, P, P, i, i, i, i, i, i, P, sz, P]
@@ -194,6 +201,36 @@ def qattn_attn_fused_q(q, k_i8, k_scale, v, out=None, causal=False, stream=None)
     st = _lib().qattn_attn_fused_q(_p(q), _p(k_i8), _p(k_scale), _p(v), _p(out), B, H, Hkv, N, d,
                                    int(bool(causal)), _stream(stream))
     _check("qattn_attn_fused_q", st)
+    return out
+
+
+def qattn_block_select(q, k, topk, causal=False, kv_list=None, kv_count=None, ws=None,
+                       stream=None):
+    """Key tiles per 256-row query block by the block-mean score, top-k (plus the causal
+    diagonals).  Returns (kv_list int32 [B*H, nsb, nkt], kv_count int32 [B*H, nsb])."""
+    B, H, Hkv, N, d = _dims(q, k)
+    nsb, nkt = -(-N // 256), -(-N // 128)
+    dev = q.device
+    kv_list = torch.full((B * H, nsb, nkt), -1, dtype=torch.int32, device=dev) if kv_list is None else kv_list
+    kv_count = torch.empty(B * H, nsb, dtype=torch.int32, device=dev) if kv_count is None else kv_count
+    wsb = int(_lib().qattn_block_select_workspace(B, H, Hkv, N, d))
+    if ws is None:
+        ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    st = _lib().qattn_block_select(_p(q), _p(k), B, H, Hkv, N, d, int(bool(causal)), int(topk),
+                                   _p(kv_list), _p(kv_count), _p(ws), ws.numel(), _stream(stream))
+    _check("qattn_block_select", st)
+    return kv_list, kv_count
+
+
+def qattn_attn_quantized_sparse(q_i8, q_scale, k_i8, k_scale, v, kv_list, kv_count, out=None,
+                                causal=False, stream=None):
+    """qattn_attn_quantized over the listed key tiles only."""
+    B, H, Hkv, N, d = _dims(q_i8, k_i8)
+    out = torch.empty(B, H, N, d, dtype=torch.float16, device=v.device) if out is None else out
+    st = _lib().qattn_attn_quantized_sparse(_p(q_i8), _p(q_scale), _p(k_i8), _p(k_scale), _p(v),
+                                            _p(out), B, H, Hkv, N, d, int(bool(causal)),
+                                            _p(kv_list), _p(kv_count), _stream(stream))
+    _check("qattn_attn_quantized_sparse", st)
     return out
 
 

@@ -110,6 +110,42 @@ qattn_status qattn_attn_quantized(const int8_t* q_i8, const float* q_scale, cons
                                   int Hkv, int N, int d, int causal, qattn_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Block-sparse attention.  The page "ThriftAttention: Selective Mixed Precision for
+ * Long-Context FP4 Attention" (technical summary, method, heuristic block selection) rates each
+ * (query block, key block) pair by the dot product of the blocks' mean vectors and singles out
+ * the top-k pairs; its results compare against sparse top-k attention, which computes only those
+ * pairs.  That sparse variant, on this library's quantized attention: query blocks of 256 rows
+ * (one attention CTA), key blocks of 128 keys (one key tile).
+ * ------------------------------------------------------------------------------------------ */
+
+/* Bytes of device workspace qattn_block_select needs (binary64 block means and scores). */
+size_t qattn_block_select_workspace(int B, int H, int Hkv, int N, int d);
+
+/* Selects the key tiles each query block computes.  q [B][H][N][d], k [B][Hkv][N][d] fp16.
+ * Query block i of head bh (rows 256 i .. 256 i + 255) and key tile j (keys 128 j .. 128 j + 127)
+ * score qmean_i . kmean_j, where the means are exact over the block's rows that exist (< N) and
+ * the dot product is a binary64 fma chain in channel order.  The list of block i holds, when
+ * causal, its diagonal tiles 2i and 2i + 1 (those < ceil(N/128)), and then the topk
+ * highest-scoring other tiles it may see (ties to the lower index), in ascending order.
+ * Writes kv_list [B*H][ceil(N/256)][ceil(N/128)] (entries past the count are not written) and
+ * kv_count [B*H][ceil(N/256)], both int32.  ws: at least qattn_block_select_workspace() bytes,
+ * clobbered.  Lists are bit-exact functions of the inputs. */
+qattn_status qattn_block_select(const void* q, const void* k, int B, int H, int Hkv, int N, int d,
+                                int causal, int topk, int* kv_list, int* kv_count, void* ws,
+                                size_t ws_bytes, qattn_stream_t stream);
+
+/* qattn_attn_quantized over the selected key tiles only: query rows of block i see the keys of
+ * the tiles in kv_list[bh][i][0 .. kv_count[bh][i]) (and, when causal, only keys <= their own
+ * index); the other tiles are neither loaded nor multiplied.  With every tile listed the result
+ * equals qattn_attn_quantized's bit for bit.  Lists as written by qattn_block_select; a causal
+ * list must hold its block's diagonal tiles (every row needs a key). */
+qattn_status qattn_attn_quantized_sparse(const int8_t* q_i8, const float* q_scale,
+                                         const int8_t* k_i8, const float* k_scale, const void* v,
+                                         void* out, int B, int H, int Hkv, int N, int d,
+                                         int causal, const int* kv_list, const int* kv_count,
+                                         qattn_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * Q quantization fused into the attention kernel: an alternative split of the forward into
  * two calls.  Results are identical to qattn_smooth_quant + qattn_attn_quantized; on B200 it
  * measured slower at 32K tokens (each CTA's quantization prologue lies on its critical path), so
