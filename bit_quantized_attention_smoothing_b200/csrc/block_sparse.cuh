@@ -23,41 +23,55 @@ constexpr int kSelQRows = 256;  // query rows per selection block (one attention
 constexpr int kSelKRows = 128;  // keys per key tile
 
 // means[o][blk][c] = mean over the rows of block blk (rows_per_block rows; the last block holds
-// the rest) of x[o][n][c].  grid (outer, nblocks), 256 threads.
+// the rest) of x[o][n][c].  grid (outer, nblocks), 256 threads: each thread sums 8 channels
+// (one 16-byte load per row) of every (256 / (D / 8))-th row.
 template <int D>
 __global__ void __launch_bounds__(256) block_means_kernel(const uint16_t* __restrict__ x, int N,
                                                           int rows_per_block,
                                                           double* __restrict__ means) {
-  constexpr int PH = 256 / D;  // row phases per channel
-  __shared__ long long part[PH][D];
+  constexpr int VPR = D / 8;        // 16-byte vectors per row
+  constexpr int RPI = 256 / VPR;    // rows per iteration of the CTA
+  __shared__ long long part[RPI][D];
   const long long o = blockIdx.x;
   const int blk = blockIdx.y;
   const int nb = gridDim.y;
-  const int c = threadIdx.x % D, ph = threadIdx.x / D;
+  const int cg = threadIdx.x % VPR, r_in = threadIdx.x / VPR;
   const int n0 = blk * rows_per_block;
   const int n1 = min(N, n0 + rows_per_block);
-  const uint16_t* src = x + static_cast<size_t>(o) * N * D;
-  long long s = 0;
-  for (int n = n0 + ph; n < n1; n += PH)
-    s += __float2ll_rn(__half2float(__ushort_as_half(src[static_cast<size_t>(n) * D + c])) * 16777216.0f);
-  part[ph][c] = s;
-  __syncthreads();
-  if (threadIdx.x < D) {
-    long long t = 0;
+  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(o) * N * D);
+  long long acc[8];
 #pragma unroll
-    for (int p = 0; p < PH; ++p) t += part[p][threadIdx.x];
-    means[(static_cast<size_t>(o) * nb + blk) * D + threadIdx.x] =
+  for (int e = 0; e < 8; ++e) acc[e] = 0;
+  for (int n = n0 + r_in; n < n1; n += RPI) {
+    const uint4 v = __ldg(src + static_cast<size_t>(n) * VPR + cg);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc[2 * e] += __float2ll_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(w[e] & 0xFFFFu))) * 16777216.0f);
+      acc[2 * e + 1] += __float2ll_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(w[e] >> 16))) * 16777216.0f);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[r_in][cg * 8 + e] = acc[e];
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += 256) {
+    long long t = 0;
+    for (int r = 0; r < RPI; ++r) t += part[r][c];
+    means[(static_cast<size_t>(o) * nb + blk) * D + c] =
         __ddiv_rn(__ll2double_rn(t), static_cast<double>(n1 - n0) * 16777216.0);
   }
 }
 
 // scores[bh][i][j] for a 32 x 32 tile of (query block i, key tile j) per CTA; grid
-// (ceil(nkt/32), ceil(nsb/32), B*H), 256 threads, each 4 scores.
+// (ceil(nkt/32), ceil(nsb/32), B*H), 256 threads, each 4 scores computed side by side (4
+// independent fma chains).  Causal: tiles no query block of the CTA may see are skipped (their
+// scores are never read).
 constexpr int kScoreTile = 32;
 template <int D>
 __global__ void __launch_bounds__(256) block_scores_kernel(const double* __restrict__ qmeans,
                                                            const double* __restrict__ kmeans,
                                                            int H, int Hkv, int nsb, int nkt,
+                                                           int causal,
                                                            double* __restrict__ scores) {
   extern __shared__ double sm[];
   double* qs = sm;                        // [32][D]
@@ -65,6 +79,7 @@ __global__ void __launch_bounds__(256) block_scores_kernel(const double* __restr
   const long long bh = blockIdx.z;
   const long long bg = (bh / H) * Hkv + (bh % H) / (H / Hkv);
   const int i0 = blockIdx.y * kScoreTile, j0 = blockIdx.x * kScoreTile;
+  if (causal && j0 > 2 * (i0 + kScoreTile - 1) + 1) return;
   for (int e = threadIdx.x; e < kScoreTile * D; e += 256) {
     const int r = e / D, c = e % D;
     qs[e] = i0 + r < nsb ? qmeans[(static_cast<size_t>(bh) * nsb + i0 + r) * D + c] : 0.0;
@@ -72,40 +87,59 @@ __global__ void __launch_bounds__(256) block_scores_kernel(const double* __restr
   }
   __syncthreads();
   const int jj = threadIdx.x % kScoreTile;
-  for (int ii = threadIdx.x / kScoreTile; ii < kScoreTile; ii += 256 / kScoreTile) {
-    if (i0 + ii >= nsb || j0 + jj >= nkt) continue;
-    double acc = 0.0;
-    for (int c = 0; c < D; ++c) acc = __fma_rn(qs[ii * D + c], ks[jj * D + c], acc);
-    scores[(static_cast<size_t>(bh) * nsb + i0 + ii) * nkt + j0 + jj] = acc;
+  const int ib = threadIdx.x / kScoreTile;  // rows ib, ib + 8, ib + 16, ib + 24
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int c = 0; c < D; ++c) {
+    const double kv = ks[jj * D + c];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) acc[r] = __fma_rn(qs[(ib + 8 * r) * D + c], kv, acc[r]);
+  }
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int ii = ib + 8 * r;
+    if (i0 + ii < nsb && j0 + jj < nkt)
+      scores[(static_cast<size_t>(bh) * nsb + i0 + ii) * nkt + j0 + jj] = acc[r];
   }
 }
 
-// Selection for query block i of head bh: grid (nsb, B*H), 256 threads.  list[bh][i][0..count)
-// ascending; entries past count are left alone.
+// Selection, one warp per query block (block i = blockIdx.x * 8 + warp of head blockIdx.y):
+// lane l holds the scores of tiles l, l + 32, ... (up to kSelMaxTiles / 32 of them) in
+// registers, and each of the topk rounds takes the warp-wide best unpicked candidate (highest
+// score, lowest index among equal scores) by shuffles.  list[bh][i][0..count) ascending; entries
+// past count are left alone.
+constexpr int kSelMaxTiles = 1024;  // N <= 2^17 keys
 __global__ void __launch_bounds__(256) block_select_kernel(const double* __restrict__ scores,
                                                            int nsb, int nkt, int causal, int topk,
                                                            int* __restrict__ list,
                                                            int* __restrict__ count) {
-  extern __shared__ unsigned char sel_smem[];
-  unsigned char* pick = sel_smem;  // [nkt]
-  __shared__ double best_s[8];
-  __shared__ int best_j[8];
+  constexpr int PER = kSelMaxTiles / 32;
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (i >= nsb) return;
   const long long bh = blockIdx.y;
-  const int i = blockIdx.x;
   const double* sc = scores + (static_cast<size_t>(bh) * nsb + i) * nkt;
   int last = causal ? 2 * i + 1 : nkt - 1;  // highest key tile the block may see
   if (last > nkt - 1) last = nkt - 1;
-  for (int j = threadIdx.x; j < nkt; j += 256) pick[j] = (causal && j >= 2 * i && j <= last) ? 1 : 0;
-  __syncthreads();
+  const int lo_forced = causal ? 2 * i : nkt;  // tiles lo_forced .. last are always kept
+  double v[PER];
+  uint32_t picked = 0;                         // bit t: tile lane + 32 t taken
+#pragma unroll
+  for (int t = 0; t < PER; ++t) {
+    const int j = lane + 32 * t;
+    v[t] = j <= last ? sc[j] : 0.0;
+    if (j >= lo_forced && j <= last) picked |= 1u << t;
+  }
   for (int r = 0; r < topk; ++r) {
-    // the best unpicked candidate: highest score, lowest index among equal scores
     double bs = 0.0;
     int bj = -1;
-    for (int j = threadIdx.x; j <= last; j += 256)
-      if (!pick[j] && (bj < 0 || sc[j] > bs)) {
-        bs = sc[j];
+#pragma unroll
+    for (int t = 0; t < PER; ++t) {
+      const int j = lane + 32 * t;
+      if (j <= last && !((picked >> t) & 1u) && (bj < 0 || v[t] > bs)) {
+        bs = v[t];
         bj = j;
       }
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
       const double os = __shfl_xor_sync(0xFFFFFFFFu, bs, off);
@@ -115,34 +149,22 @@ __global__ void __launch_bounds__(256) block_select_kernel(const double* __restr
         bj = oj;
       }
     }
-    if ((threadIdx.x & 31) == 0) {
-      best_s[threadIdx.x >> 5] = bs;
-      best_j[threadIdx.x >> 5] = bj;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      double s = 0.0;
-      int jb = -1;
-      for (int w = 0; w < 8; ++w)
-        if (best_j[w] >= 0 && (jb < 0 || best_s[w] > s || (best_s[w] == s && best_j[w] < jb))) {
-          s = best_s[w];
-          jb = best_j[w];
-        }
-      best_j[0] = jb;
-      if (jb >= 0) pick[jb] = 1;
-    }
-    __syncthreads();
-    const bool done = best_j[0] < 0;
-    __syncthreads();
-    if (done) break;
+    if (bj < 0) break;  // warp-uniform: every candidate taken
+    if ((bj & 31) == lane) picked |= 1u << (bj >> 5);
   }
-  if (threadIdx.x == 0) {
-    int* out = list + (static_cast<size_t>(bh) * nsb + i) * nkt;
-    int n = 0;
-    for (int j = 0; j < nkt; ++j)
-      if (pick[j]) out[n++] = j;
-    count[static_cast<size_t>(bh) * nsb + i] = n;
+  // ascending list: tiles in order t-major within each lane are lane + 32 t; a warp-wide prefix
+  // count per 32-tile stripe gives each picked tile its position
+  int* out = list + (static_cast<size_t>(bh) * nsb + i) * nkt;
+  int base = 0;
+#pragma unroll
+  for (int t = 0; t < PER; ++t) {
+    if (32 * t > last) break;
+    const bool p = (picked >> t) & 1u;
+    const unsigned m = __ballot_sync(0xFFFFFFFFu, p);
+    if (p) out[base + __popc(m & ((1u << lane) - 1u))] = lane + 32 * t;
+    base += __popc(m);
   }
+  if (lane == 0) count[static_cast<size_t>(bh) * nsb + i] = base;
 }
 
 }  // namespace qattn

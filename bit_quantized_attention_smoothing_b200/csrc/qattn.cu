@@ -246,10 +246,10 @@ qattn_status run_block_select(const void* q, const void* k, int B, int H, int Hk
     return QATTN_ERR_CUDA;
   if (B * H > 65535) return QATTN_ERR_UNSUPPORTED;
   dim3 gs((L.nkt + kScoreTile - 1) / kScoreTile, (L.nsb + kScoreTile - 1) / kScoreTile, B * H);
-  block_scores_kernel<D><<<gs, 256, smem, st>>>(qm, km, H, Hkv, L.nsb, L.nkt, sc);
+  block_scores_kernel<D><<<gs, 256, smem, st>>>(qm, km, H, Hkv, L.nsb, L.nkt, causal, sc);
   if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
-  block_select_kernel<<<dim3(L.nsb, B * H), 256, L.nkt, st>>>(sc, L.nsb, L.nkt, causal, topk,
-                                                              list, count);
+  block_select_kernel<<<dim3((L.nsb + 7) / 8, B * H), 256, 0, st>>>(sc, L.nsb, L.nkt, causal,
+                                                                    topk, list, count);
   return launch_status();
 }
 
@@ -437,6 +437,7 @@ qattn_status qattn_block_select(const void* q, const void* k, int B, int H, int 
   s = check_ptrs(q, k, kv_list, kv_count);
   if (s != QATTN_OK) return s;
   if (topk < 0) return QATTN_ERR_INVALID_ARG;
+  if ((N + kSelKRows - 1) / kSelKRows > kSelMaxTiles) return QATTN_ERR_UNSUPPORTED;
   if (ws == nullptr || ws_bytes < sel_layout(B, H, Hkv, N, d).total) return QATTN_ERR_WORKSPACE;
   if (!aligned16(ws)) return QATTN_ERR_MISALIGNED;
   if ((s = device_ok()) != QATTN_OK) return s;

@@ -204,6 +204,10 @@ def qattn_attn_fused_q(q, k_i8, k_scale, v, out=None, causal=False, stream=None)
     return out
 
 
+def qattn_block_select_workspace(B: int, H: int, Hkv: int, N: int, d: int) -> int:
+    return int(_lib().qattn_block_select_workspace(B, H, Hkv, N, d))
+
+
 def qattn_block_select(q, k, topk, causal=False, kv_list=None, kv_count=None, ws=None,
                        stream=None):
     """Key tiles per 256-row query block by the block-mean score, top-k (plus the causal

@@ -129,7 +129,8 @@ size_t qattn_block_select_workspace(int B, int H, int Hkv, int N, int d);
  * highest-scoring other tiles it may see (ties to the lower index), in ascending order.
  * Writes kv_list [B*H][ceil(N/256)][ceil(N/128)] (entries past the count are not written) and
  * kv_count [B*H][ceil(N/256)], both int32.  ws: at least qattn_block_select_workspace() bytes,
- * clobbered.  Lists are bit-exact functions of the inputs. */
+ * clobbered.  Lists are bit-exact functions of the inputs.  N <= 131072 (else
+ * QATTN_ERR_UNSUPPORTED). */
 qattn_status qattn_block_select(const void* q, const void* k, int B, int H, int Hkv, int N, int d,
                                 int causal, int topk, int* kv_list, int* kv_count, void* ws,
                                 size_t ws_bytes, qattn_stream_t stream);
