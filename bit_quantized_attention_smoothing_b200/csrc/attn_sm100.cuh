@@ -555,11 +555,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t o_tm = tmem + lane_off + 256 + wt * D;
       float m = -INFINITY, l = 0.0f;
       bool ok = true;
+      // key tiles of steps j and j + 1 in registers; the list entry of step j + 2 is loaded one
+      // step ahead, so the K scales of step j + 1 never wait on a dependent list load
       int kt = ktile(0);
+      int kt1 = nt > 1 ? ktile(1) : 0;
       float ks0 = __ldg(ksc + 2 * kt);
       float ks1 = 2 * kt + 1 < nkb ? __ldg(ksc + 2 * kt + 1) : 0.0f;
       for (int j = 0; j < nt; ++j) {
-        const int nkt_next = j + 1 < nt ? ktile(j + 1) : 0;
+        const int nkt_next = kt1;
+        kt1 = j + 2 < nt ? ktile(j + 2) : 0;
         const float nks0 = (2 * nkt_next < nkb) ? __ldg(ksc + 2 * nkt_next) : 0.0f;
         const float nks1 = (2 * nkt_next + 1 < nkb) ? __ldg(ksc + 2 * nkt_next + 1) : 0.0f;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full[wt], static_cast<uint32_t>(j) & 1u, abort));
