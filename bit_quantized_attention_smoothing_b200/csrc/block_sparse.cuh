@@ -74,8 +74,8 @@ __global__ void __launch_bounds__(256) block_scores_kernel(const double* __restr
                                                            int causal,
                                                            double* __restrict__ scores) {
   extern __shared__ double sm[];
-  double* qs = sm;                        // [32][D]
-  double* ks = sm + kScoreTile * D;       // [32][D]
+  double* qs = sm;                        // [32][D]: row-major (a warp reads one row: broadcast)
+  double* ks = sm + kScoreTile * D;       // [D][32]: channel-major (a warp reads 32 consecutive)
   const long long bh = blockIdx.z;
   const long long bg = (bh / H) * Hkv + (bh % H) / (H / Hkv);
   const int i0 = blockIdx.y * kScoreTile, j0 = blockIdx.x * kScoreTile;
@@ -83,14 +83,14 @@ __global__ void __launch_bounds__(256) block_scores_kernel(const double* __restr
   for (int e = threadIdx.x; e < kScoreTile * D; e += 256) {
     const int r = e / D, c = e % D;
     qs[e] = i0 + r < nsb ? qmeans[(static_cast<size_t>(bh) * nsb + i0 + r) * D + c] : 0.0;
-    ks[e] = j0 + r < nkt ? kmeans[(static_cast<size_t>(bg) * nkt + j0 + r) * D + c] : 0.0;
+    ks[c * kScoreTile + r] = j0 + r < nkt ? kmeans[(static_cast<size_t>(bg) * nkt + j0 + r) * D + c] : 0.0;
   }
   __syncthreads();
   const int jj = threadIdx.x % kScoreTile;
   const int ib = threadIdx.x / kScoreTile;  // rows ib, ib + 8, ib + 16, ib + 24
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
   for (int c = 0; c < D; ++c) {
-    const double kv = ks[jj * D + c];
+    const double kv = ks[c * kScoreTile + jj];
 #pragma unroll
     for (int r = 0; r < 4; ++r) acc[r] = __fma_rn(qs[(ib + 8 * r) * D + c], kv, acc[r]);
   }
@@ -130,14 +130,31 @@ __global__ void __launch_bounds__(256) block_select_kernel(const double* __restr
     if (j >= lo_forced && j <= last) picked |= 1u << t;
   }
   for (int r = 0; r < topk; ++r) {
-    double bs = 0.0;
-    int bj = -1;
+    // the lane's best unpicked candidate, as four independent scans over t = p (mod 4) (each
+    // keeps the lowest tile among equal scores), merged with the same rule; stripes past the
+    // last visible tile are skipped (warp-uniform)
+    double ps[4] = {0.0, 0.0, 0.0, 0.0};
+    int pj[4] = {-1, -1, -1, -1};
 #pragma unroll
-    for (int t = 0; t < PER; ++t) {
-      const int j = lane + 32 * t;
-      if (j <= last && !((picked >> t) & 1u) && (bj < 0 || v[t] > bs)) {
-        bs = v[t];
-        bj = j;
+    for (int tg = 0; tg < PER / 4; ++tg) {
+      if (128 * tg > last) break;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int t = 4 * tg + q;
+        const int j = lane + 32 * t;
+        if (j <= last && !((picked >> t) & 1u) && (pj[q] < 0 || v[t] > ps[q])) {
+          ps[q] = v[t];
+          pj[q] = j;
+        }
+      }
+    }
+    double bs = ps[0];
+    int bj = pj[0];
+#pragma unroll
+    for (int q = 1; q < 4; ++q) {
+      if (pj[q] >= 0 && (bj < 0 || ps[q] > bs || (ps[q] == bs && pj[q] < bj))) {
+        bs = ps[q];
+        bj = pj[q];
       }
     }
 #pragma unroll
