@@ -18,7 +18,9 @@
 //    scale block (3-input max), dequantization and exp2 argument with packed fp32x2 FMAs, MUFU
 //    ex2, P packed to fp16 and written back over the scores' tensor-memory columns, row sum of the
 //    fp16-rounded P; lazy rescaling of O only when the running max grows by more than 2^8; P
-//    scaled into the top of the fp16 range;
+//    scaled into the top of the fp16 range; the two warpgroups' steps are kept half a step apart
+//    (each starts a step when the other is half through its exponentials), so the MUFU-bound
+//    passes of the two tiles alternate instead of contending;
 //  * causal: key tiles above the diagonal are never loaded or multiplied; the diagonal tile is
 //    masked in registers (a compile-time-specialised path); CTAs are launched heaviest-first;
 //  * grouped-query attention: query head h reads kv head h / (H / Hkv); CTAs of the heads that
@@ -75,6 +77,7 @@ struct __align__(16) AttnBars {
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t pv_done[2];
+  uint64_t mx_done[2];  // Q tile w's softmax half through a step's exponentials (4 arrives)
   uint32_t tmem_base;
   int abort;
 };
@@ -185,12 +188,13 @@ __device__ __forceinline__ constexpr bool emulated_pair(int i) { return (kExp2Em
 // masked keys (MASK; key offset above lim) -> -inf, row maximum per 64-key K scale block, lazy
 // update of the running max m (alpha = rescale factor, need = O must be rescaled), then
 // P = 2^(x * c - m + offset) packed as fp16 pairs (even key in the low half) and stored over the
-// row's first 64 TMEM columns, and the row sum of the fp16-rounded P.  MASK is a compile-time
-// switch so the unmasked steps carry no per-element tests.
+// row's first 64 TMEM columns, and the row sum of the fp16-rounded P.  Once the first 64 keys'
+// P are stored, the warp arrives on mx_bar (the other Q tile's softmax waits for it).  MASK is a
+// compile-time switch so the unmasked steps carry no per-element tests.
 template <bool MASK>
 __device__ __forceinline__ void softmax_row(uint32_t (&sr)[4][32], int lim, float c0, float c1,
                                             bool first, float& m, float& l, float& alpha,
-                                            bool& need, uint32_t s_tm) {
+                                            bool& need, uint32_t s_tm, uint64_t* mx_bar) {
   float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
@@ -254,6 +258,11 @@ __device__ __forceinline__ void softmax_row(uint32_t (&sr)[4][32], int lim, floa
     // keys 64 * hf .. 64 * hf + 63 -> P columns 32 * hf .. 32 * hf + 31; all scores are in
     // registers by now, so these columns are free
     tmem_st32(s_tm + hf * 32, pk);
+    if (hf == 0) {
+      // half of the row's exponentials done: the other Q tile's softmax may start its step
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(mx_bar);
+    }
   }
   l += acc0 + acc1;
 }
@@ -421,6 +430,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&bars->s_full[w], 1);
       mbar_init(&bars->p_full[w], 4);  // one arrive per softmax warp of the Q tile
       mbar_init(&bars->pv_done[w], 1);
+      mbar_init(&bars->mx_done[w], 4);
     }
     bars->abort = 0;
     fence_mbar_init();
@@ -566,6 +576,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         kt1 = j + 2 < nt ? ktile(j + 2) : 0;
         const float nks0 = (2 * nkt_next < nkb) ? __ldg(ksc + 2 * nkt_next) : 0.0f;
         const float nks1 = (2 * nkt_next + 1 < nkb) ? __ldg(ksc + 2 * nkt_next + 1) : 0.0f;
+        // The two Q tiles' softmax steps are kept half a step apart, so that their MUFU-bound
+        // exponential passes do not run at the same time: tile 1's step j starts once tile 0's
+        // step j is half through its exponentials, tile 0's step j once tile 1's step j - 1 is
+        // (mx_done[w], one arrive per warp per step).  Without this the two tiles settle nearly in
+        // phase and each step's softmax runs ~40 % longer.  Tile 0 has no step nw0 (causal, one
+        // key tile fewer than tile 1), so tile 1's last step is not gated; neither barrier gets two
+        // phases ahead of its waiter, since each tile's next arrive needs the other's.
+        if (wt == 1 && j < nw0)
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->mx_done[0], static_cast<uint32_t>(j) & 1u, abort));
+        else if (wt == 0 && j > 0 && j - 1 < nw1)
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->mx_done[1], static_cast<uint32_t>(j - 1) & 1u, abort));
+        if (!ok) break;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full[wt], static_cast<uint32_t>(j) & 1u, abort));
         if (!ok) break;
         tc_fence_after();
@@ -585,8 +607,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const bool masked = __any_sync(0xFFFFFFFFu, lim < kBN - 1);
         float alpha;
         bool need;
-        if (masked) softmax_row<true>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm);
-        else softmax_row<false>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm);
+        if (masked) softmax_row<true>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, &bars->mx_done[wt]);
+        else softmax_row<false>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, &bars->mx_done[wt]);
         if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
           // O holds PV up to tile j-1 (complete: QK(j) was issued after PV(j-1)), and PV(j)
           // waits for this warp's arrive below.
