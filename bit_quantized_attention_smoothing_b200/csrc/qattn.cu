@@ -521,6 +521,48 @@ qattn_status qattn_forward(const void* q, const void* k, const void* v, void* ou
   return s;
 }
 
+qattn_status qattn_forward_sparse(const void* q, const void* k, const void* v, void* out, int B,
+                                  int H, int Hkv, int N, int d, int causal, int topk,
+                                  qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q, k, v, out);
+  if (s != QATTN_OK) return s;
+  // non-causal with topk 0 would leave every row without a key
+  if (topk < 0 || (!causal && topk == 0)) return QATTN_ERR_INVALID_ARG;
+  if ((N + kSelKRows - 1) / kSelKRows > kSelMaxTiles) return QATTN_ERR_UNSUPPORTED;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // one stream-ordered workspace: the quantized operands, the selection's scratch and the
+  // tile lists (kv_list [B*H][ceil(N/256)][ceil(N/128)], kv_count [B*H][ceil(N/256)])
+  const QuantLayout L = forward_layout(B, H, Hkv, N, d);
+  const SelLayout S = sel_layout(B, H, Hkv, N, d);
+  const size_t off_sel = L.total;
+  const size_t off_list = align_up(off_sel + S.total);
+  const size_t n_list = static_cast<size_t>(B) * H * S.nsb * S.nkt;
+  const size_t off_count = align_up(off_list + sizeof(int) * n_list);
+  const size_t total = align_up(off_count + sizeof(int) * static_cast<size_t>(B) * H * S.nsb);
+  void* ws = nullptr;
+  if ((s = pool_alloc(&ws, total, st)) != QATTN_OK) return s;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int8_t* q_i8 = reinterpret_cast<int8_t*>(w + L.q_i8);
+  int8_t* k_i8 = reinterpret_cast<int8_t*>(w + L.k_i8);
+  float* q_scale = reinterpret_cast<float*>(w + L.q_scale);
+  float* k_scale = reinterpret_cast<float*>(w + L.k_scale);
+  long long* sums = reinterpret_cast<long long*>(w + L.sums);
+  int* kv_list = reinterpret_cast<int*>(w + off_list);
+  int* kv_count = reinterpret_cast<int*>(w + off_count);
+  s = dispatch_smooth_quant(q, k, B, H, Hkv, N, d, q_i8, q_scale, k_i8, k_scale, nullptr, sums, st);
+  if (s == QATTN_OK)
+    s = d == 128 ? run_block_select<128>(q, k, B, H, Hkv, N, causal, topk, kv_list, kv_count, w + off_sel, st)
+                 : run_block_select<64>(q, k, B, H, Hkv, N, causal, topk, kv_list, kv_count, w + off_sel, st);
+  if (s == QATTN_OK)
+    s = dispatch_attn<false>(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, d, causal, st,
+                             kv_list, kv_count);
+  if (cudaFreeAsync(ws, st) != cudaSuccess && s == QATTN_OK) s = QATTN_ERR_CUDA;
+  return s;
+}
+
 namespace {
 
 // Copy streams of the host-buffer forward, created once per device (non-blocking, so they do

@@ -29,6 +29,7 @@ EXPORTS = [
     "qattn_smooth_quant_noalloc",
     "qattn_attn_quantized", "qattn_smooth_k", "qattn_attn_fused_q",
     "qattn_block_select_workspace", "qattn_block_select", "qattn_attn_quantized_sparse",
+    "qattn_forward_sparse",
     "qattn_forward_workspace", "qattn_forward_ws", "qattn_forward",
     "qattn_forward_host", "qattn_debug_qk_int32", "qattn_debug_wait_timeout",
     "qattn_check_device_status",
@@ -80,6 +81,8 @@ def _lib():
         L.qattn_block_select.restype = i
         L.qattn_attn_quantized_sparse.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, P, P, P]
         L.qattn_attn_quantized_sparse.restype = i
+        L.qattn_forward_sparse.argtypes = [P, P, P, P, i, i, i, i, i, i, i, P]
+        L.qattn_forward_sparse.restype = i
         L.qattn_forward_workspace.argtypes = [i, i, i, i, i]
         L.qattn_forward_workspace.restype = sz
         L.qattn_forward_ws.argtypes = [P, P, P, P, i, i, i, i, i, i, P, sz, P]
@@ -224,6 +227,17 @@ def qattn_block_select(q, k, topk, causal=False, kv_list=None, kv_count=None, ws
                                    _p(kv_list), _p(kv_count), _p(ws), ws.numel(), _stream(stream))
     _check("qattn_block_select", st)
     return kv_list, kv_count
+
+
+def qattn_forward_sparse(q, k, v, topk, out=None, causal=False, stream=None):
+    """The whole block-sparse forward (smoothing + quantization, top-k key-tile selection,
+    sparse attention) in one call; fp16 in, fp16 out."""
+    B, H, Hkv, N, d = _dims(q, k)
+    out = torch.empty(B, H, N, d, dtype=torch.float16, device=q.device) if out is None else out
+    st = _lib().qattn_forward_sparse(_p(q), _p(k), _p(v), _p(out), B, H, Hkv, N, d,
+                                     int(bool(causal)), int(topk), _stream(stream))
+    _check("qattn_forward_sparse", st)
+    return out
 
 
 def qattn_attn_quantized_sparse(q_i8, q_scale, k_i8, k_scale, v, kv_list, kv_count, out=None,

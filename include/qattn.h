@@ -146,6 +146,16 @@ qattn_status qattn_attn_quantized_sparse(const int8_t* q_i8, const float* q_scal
                                          int causal, const int* kv_list, const int* kv_count,
                                          qattn_stream_t stream);
 
+/* The whole block-sparse forward in one call: smoothing + quantization, key-tile selection with
+ * topk (qattn_block_select's rule) and the sparse attention, fp16 in, fp16 out; results equal
+ * those of the three calls.  The workspace (quantized operands, selection scratch, tile lists)
+ * is taken stream-ordered from the library's per-device pool and returned.  Errors as
+ * qattn_block_select (topk < 0, or topk == 0 without causal, which would leave rows with no
+ * key: QATTN_ERR_INVALID_ARG; N > 131072: QATTN_ERR_UNSUPPORTED) and qattn_forward. */
+qattn_status qattn_forward_sparse(const void* q, const void* k, const void* v, void* out, int B,
+                                  int H, int Hkv, int N, int d, int causal, int topk,
+                                  qattn_stream_t stream);
+
 /* ------------------------------------------------------------------------------------------
  * Q quantization fused into the attention kernel: an alternative split of the forward into
  * two calls.  Results are identical to qattn_smooth_quant + qattn_attn_quantized; on B200 it

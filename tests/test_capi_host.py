@@ -100,3 +100,17 @@ def test_workspace_and_alignment_checks():
     assert L.qattn_debug_wait_timeout(1000, None, None) == 1
     assert L.qattn_debug_wait_timeout(-1, P(16), None) == 1
     assert L.qattn_debug_wait_timeout(3_000_000_000, P(16), None) == 1
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((None, P(32), P(48), P(64), 1, 4, 2, 256, 128, 1, 4, None), 1),     # null pointer
+    ((P(16), P(32), P(48), P(64), 1, 4, 3, 256, 128, 1, 4, None), 1),    # H % Hkv != 0
+    ((P(16), P(32), P(48), P(64), 1, 4, 2, 256, 128, 1, -1, None), 1),   # topk < 0
+    ((P(16), P(32), P(48), P(64), 1, 4, 2, 256, 128, 0, 0, None), 1),    # no key for any row
+    ((P(16), P(32), P(48), P(64), 1, 4, 2, 256, 96, 1, 4, None), 2),     # d
+    ((P(16), P(32), P(48), P(64), 1, 4, 2, 131073, 128, 1, 4, None), 2), # past the selection limit
+    ((P(16), P(33), P(48), P(64), 1, 4, 2, 256, 128, 1, 4, None), 3),    # misaligned
+])
+def test_forward_sparse_argument_checks(args, expect):
+    L = Q.load()
+    assert L.qattn_forward_sparse(*args) == expect

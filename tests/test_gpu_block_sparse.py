@@ -85,3 +85,17 @@ def test_all_tiles_listed_equals_dense(lib, causal):
     sparse = lib.qattn_attn_quantized_sparse(q_i8, q_s, k_i8, k_s, v, kl, kc, causal=causal)
     torch.cuda.synchronize()
     assert torch.equal(dense, sparse)
+
+
+@pytest.mark.parametrize("causal,topk", [(True, 2), (False, 3), (True, 0)])
+def test_forward_sparse_one_call_equals_the_three_calls(lib, causal, topk):
+    """qattn_forward_sparse (one call, its own workspace) gives the same output, bit for bit, as
+    smoothing + quantization, selection and the sparse attention called one by one."""
+    w = WORKLOADS["llama8b_32k"].with_(H=4, Hkv=2, N=1300, causal=causal)
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    q_i8, q_s, k_i8, k_s, _ = lib.qattn_smooth_quant(q, k)
+    kl, kc = lib.qattn_block_select(q, k, topk, causal=causal)
+    ref = lib.qattn_attn_quantized_sparse(q_i8, q_s, k_i8, k_s, v, kl, kc, causal=causal)
+    got = lib.qattn_forward_sparse(q, k, v, topk, causal=causal)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
