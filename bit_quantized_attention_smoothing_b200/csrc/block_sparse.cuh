@@ -62,43 +62,62 @@ __global__ void __launch_bounds__(256) block_means_kernel(const uint16_t* __rest
   }
 }
 
-// scores[bh][i][j] for a 32 x 32 tile of (query block i, key tile j) per CTA; grid
-// (ceil(nkt/32), ceil(nsb/32), B*H), 256 threads, each 4 scores computed side by side (4
-// independent fma chains).  Causal: tiles no query block of the CTA may see are skipped (their
-// scores are never read).
-constexpr int kScoreTile = 32;
+// scores[bh][i][j] for a 64 x 64 tile of (query block i, key tile j) per CTA; grid
+// (ceil(nkt/64), ceil(nsb/64), B*H), 256 threads, each 4 x 4 scores (rows ty + 16 r, columns
+// tx + 16 s) from 8 shared-memory loads per channel.  The means pass through shared memory 32
+// channels at a time, channel-major (a warp's loads are broadcasts or 16 consecutive doubles);
+// every score is still one fma per channel in channel order.  Causal: tiles no query block of
+// the CTA may see are skipped (their scores are never read).
+constexpr int kScoreTile = 64;
+constexpr int kScoreChunk = 32;
 template <int D>
 __global__ void __launch_bounds__(256) block_scores_kernel(const double* __restrict__ qmeans,
                                                            const double* __restrict__ kmeans,
                                                            int H, int Hkv, int nsb, int nkt,
                                                            int causal,
                                                            double* __restrict__ scores) {
-  extern __shared__ double sm[];
-  double* qs = sm;                        // [32][D]: row-major (a warp reads one row: broadcast)
-  double* ks = sm + kScoreTile * D;       // [D][32]: channel-major (a warp reads 32 consecutive)
+  __shared__ double qs[kScoreChunk][kScoreTile + 1];
+  __shared__ double ks[kScoreChunk][kScoreTile + 1];
   const long long bh = blockIdx.z;
   const long long bg = (bh / H) * Hkv + (bh % H) / (H / Hkv);
   const int i0 = blockIdx.y * kScoreTile, j0 = blockIdx.x * kScoreTile;
   if (causal && j0 > 2 * (i0 + kScoreTile - 1) + 1) return;
-  for (int e = threadIdx.x; e < kScoreTile * D; e += 256) {
-    const int r = e / D, c = e % D;
-    qs[e] = i0 + r < nsb ? qmeans[(static_cast<size_t>(bh) * nsb + i0 + r) * D + c] : 0.0;
-    ks[c * kScoreTile + r] = j0 + r < nkt ? kmeans[(static_cast<size_t>(bg) * nkt + j0 + r) * D + c] : 0.0;
-  }
-  __syncthreads();
-  const int jj = threadIdx.x % kScoreTile;
-  const int ib = threadIdx.x / kScoreTile;  // rows ib, ib + 8, ib + 16, ib + 24
-  double acc[4] = {0.0, 0.0, 0.0, 0.0};
-  for (int c = 0; c < D; ++c) {
-    const double kv = ks[c * kScoreTile + jj];
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  double acc[4][4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) acc[r] = __fma_rn(qs[(ib + 8 * r) * D + c], kv, acc[r]);
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[r][c] = 0.0;
+  for (int c0 = 0; c0 < D; c0 += kScoreChunk) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < kScoreTile * kScoreChunk; e += 256) {
+      const int r = e / kScoreChunk, c = e % kScoreChunk;
+      qs[c][r] = i0 + r < nsb ? qmeans[(static_cast<size_t>(bh) * nsb + i0 + r) * D + c0 + c] : 0.0;
+      ks[c][r] = j0 + r < nkt ? kmeans[(static_cast<size_t>(bg) * nkt + j0 + r) * D + c0 + c] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int c = 0; c < kScoreChunk; ++c) {
+      double qv[4], kv[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) qv[r] = qs[c][ty + 16 * r];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) kv[u] = ks[c][tx + 16 * u];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[r][u] = __fma_rn(qv[r], kv[u], acc[r][u]);
+    }
   }
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
-    const int ii = ib + 8 * r;
-    if (i0 + ii < nsb && j0 + jj < nkt)
-      scores[(static_cast<size_t>(bh) * nsb + i0 + ii) * nkt + j0 + jj] = acc[r];
+    const int ii = ty + 16 * r;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int jj = tx + 16 * u;
+      if (i0 + ii < nsb && j0 + jj < nkt)
+        scores[(static_cast<size_t>(bh) * nsb + i0 + ii) * nkt + j0 + jj] = acc[r][u];
+    }
   }
 }
 

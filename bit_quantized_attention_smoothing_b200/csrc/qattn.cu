@@ -240,13 +240,9 @@ qattn_status run_block_select(const void* q, const void* k, int B, int H, int Hk
   block_means_kernel<D><<<dim3(B * Hkv, L.nkt), 256, 0, st>>>(static_cast<const uint16_t*>(k), N,
                                                              kSelKRows, km);
   if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
-  const int smem = 2 * kScoreTile * D * static_cast<int>(sizeof(double));
-  if (cudaFuncSetAttribute(block_scores_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem) != cudaSuccess)
-    return QATTN_ERR_CUDA;
   if (B * H > 65535) return QATTN_ERR_UNSUPPORTED;
   dim3 gs((L.nkt + kScoreTile - 1) / kScoreTile, (L.nsb + kScoreTile - 1) / kScoreTile, B * H);
-  block_scores_kernel<D><<<gs, 256, smem, st>>>(qm, km, H, Hkv, L.nsb, L.nkt, causal, sc);
+  block_scores_kernel<D><<<gs, 256, 0, st>>>(qm, km, H, Hkv, L.nsb, L.nkt, causal, sc);
   if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
   block_select_kernel<<<dim3((L.nsb + 7) / 8, B * H), 256, 0, st>>>(sc, L.nsb, L.nkt, causal,
                                                                     topk, list, count);
