@@ -123,15 +123,24 @@ __global__ void __launch_bounds__(256) block_scores_kernel(const double* __restr
 
 // Selection, one warp per query block (block i = blockIdx.x * 8 + warp of head blockIdx.y):
 // lane l holds the scores of tiles l, l + 32, ... (up to kSelMaxTiles / 32 of them) in
-// registers, and each of the topk rounds takes the warp-wide best unpicked candidate (highest
-// score, lowest index among equal scores) by shuffles.  list[bh][i][0..count) ascending; entries
-// past count are left alone.
+// registers as order-preserving 64-bit keys (binary64 bits with the sign flipped, negative values
+// complemented; -0 taken as +0, so equal scores give equal keys).  The topk candidates with the
+// highest scores, lowest index among equal scores, are found without ranking them: a bisection
+// over the key bits (from the highest bit on which the candidates differ) finds the topk-th
+// largest key T, with one warp-wide count per bit; every candidate above T is taken, and of those
+// equal to T the lowest-indexed ones.  list[bh][i][0..count) ascending; entries past count are
+// left alone.
 constexpr int kSelMaxTiles = 1024;  // N <= 2^17 keys
+__device__ __forceinline__ uint64_t score_key(double v) {
+  const uint64_t u = static_cast<uint64_t>(__double_as_longlong(v + 0.0));
+  return (u >> 63) ? ~u : (u | (1ull << 63));
+}
 __global__ void __launch_bounds__(256) block_select_kernel(const double* __restrict__ scores,
                                                            int nsb, int nkt, int causal, int topk,
                                                            int* __restrict__ list,
                                                            int* __restrict__ count) {
   constexpr int PER = kSelMaxTiles / 32;
+  constexpr uint32_t kFull = 0xFFFFFFFFu;
   const int lane = threadIdx.x & 31;
   const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (i >= nsb) return;
@@ -140,53 +149,79 @@ __global__ void __launch_bounds__(256) block_select_kernel(const double* __restr
   int last = causal ? 2 * i + 1 : nkt - 1;  // highest key tile the block may see
   if (last > nkt - 1) last = nkt - 1;
   const int lo_forced = causal ? 2 * i : nkt;  // tiles lo_forced .. last are always kept
-  double v[PER];
-  uint32_t picked = 0;                         // bit t: tile lane + 32 t taken
+  const int cand_end = min(last + 1, lo_forced);  // candidates: tiles 0 .. cand_end - 1
+  const int kk = min(topk, cand_end);
+  uint64_t key[PER];
+  uint32_t picked = 0;  // bit t: tile lane + 32 t taken
+  uint32_t cand = 0;    // bit t: tile lane + 32 t is a candidate
 #pragma unroll
   for (int t = 0; t < PER; ++t) {
     const int j = lane + 32 * t;
-    v[t] = j <= last ? sc[j] : 0.0;
+    key[t] = j < cand_end ? score_key(sc[j]) : 0ull;
+    if (j < cand_end) cand |= 1u << t;
     if (j >= lo_forced && j <= last) picked |= 1u << t;
   }
-  for (int r = 0; r < topk; ++r) {
-    // the lane's best unpicked candidate, as four independent scans over t = p (mod 4) (each
-    // keeps the lowest tile among equal scores), merged with the same rule; stripes past the
-    // last visible tile are skipped (warp-uniform)
-    double ps[4] = {0.0, 0.0, 0.0, 0.0};
-    int pj[4] = {-1, -1, -1, -1};
+  if (kk == cand_end) {
+    picked |= cand;
+  } else if (kk > 0) {
+    // bits common to every candidate key fix the top of T
+    uint64_t k_and = ~0ull, k_or = 0ull;
 #pragma unroll
-    for (int tg = 0; tg < PER / 4; ++tg) {
-      if (128 * tg > last) break;
+    for (int t = 0; t < PER; ++t) {
+      if (32 * t >= cand_end) break;
+      if ((cand >> t) & 1u) {
+        k_and &= key[t];
+        k_or |= key[t];
+      }
+    }
+    const uint32_t and_hi = __reduce_and_sync(kFull, static_cast<uint32_t>(k_and >> 32));
+    const uint32_t and_lo = __reduce_and_sync(kFull, static_cast<uint32_t>(k_and));
+    const uint32_t or_hi = __reduce_or_sync(kFull, static_cast<uint32_t>(k_or >> 32));
+    const uint32_t or_lo = __reduce_or_sync(kFull, static_cast<uint32_t>(k_or));
+    const uint64_t kand = (static_cast<uint64_t>(and_hi) << 32) | and_lo;
+    const uint64_t diff = kand ^ ((static_cast<uint64_t>(or_hi) << 32) | or_lo);
+    const int top = diff ? 63 - __clzll(static_cast<long long>(diff)) : -1;
+    // T = the largest key with at least kk candidate keys >= T
+    uint64_t T = top >= 63 ? 0ull : (kand >> (top + 1)) << (top + 1);
+    for (int bit = top; bit >= 0; --bit) {
+      const uint64_t thr = T | (1ull << bit);
+      uint32_t n = 0;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int t = 4 * tg + q;
-        const int j = lane + 32 * t;
-        if (j <= last && !((picked >> t) & 1u) && (pj[q] < 0 || v[t] > ps[q])) {
-          ps[q] = v[t];
-          pj[q] = j;
+      for (int t = 0; t < PER; ++t) {
+        if (32 * t >= cand_end) break;
+        n += ((cand >> t) & 1u) && key[t] >= thr ? 1u : 0u;
+      }
+      if (__reduce_add_sync(kFull, n) >= static_cast<uint32_t>(kk)) T = thr;
+    }
+    // every candidate above T, then the lowest-indexed ones equal to T
+    uint32_t n_gt = 0;
+#pragma unroll
+    for (int t = 0; t < PER; ++t) {
+      if (32 * t >= cand_end) break;
+      if (((cand >> t) & 1u) && key[t] > T) {
+        picked |= 1u << t;
+        ++n_gt;
+      }
+    }
+    int need = kk - static_cast<int>(__reduce_add_sync(kFull, n_gt));
+#pragma unroll
+    for (int t = 0; t < PER; ++t) {
+      if (need <= 0 || 32 * t >= cand_end) break;
+      const uint32_t eq = __ballot_sync(kFull, ((cand >> t) & 1u) && key[t] == T);
+      const int ne = __popc(eq);
+      const uint32_t take = ne <= need ? eq : [&] {
+        // the need lowest set bits of eq
+        uint32_t m = eq, r = 0;
+        for (int x = 0; x < need; ++x) {
+          const uint32_t lowbit = m & (~m + 1u);
+          r |= lowbit;
+          m ^= lowbit;
         }
-      }
+        return r;
+      }();
+      if ((take >> lane) & 1u) picked |= 1u << t;
+      need -= __popc(take);
     }
-    double bs = ps[0];
-    int bj = pj[0];
-#pragma unroll
-    for (int q = 1; q < 4; ++q) {
-      if (pj[q] >= 0 && (bj < 0 || ps[q] > bs || (ps[q] == bs && pj[q] < bj))) {
-        bs = ps[q];
-        bj = pj[q];
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const double os = __shfl_xor_sync(0xFFFFFFFFu, bs, off);
-      const int oj = __shfl_xor_sync(0xFFFFFFFFu, bj, off);
-      if (oj >= 0 && (bj < 0 || os > bs || (os == bs && oj < bj))) {
-        bs = os;
-        bj = oj;
-      }
-    }
-    if (bj < 0) break;  // warp-uniform: every candidate taken
-    if ((bj & 31) == lane) picked |= 1u << (bj >> 5);
   }
   // ascending list: tiles in order t-major within each lane are lane + 32 t; a warp-wide prefix
   // count per 32-tile stripe gives each picked tile its position
@@ -196,7 +231,7 @@ __global__ void __launch_bounds__(256) block_select_kernel(const double* __restr
   for (int t = 0; t < PER; ++t) {
     if (32 * t > last) break;
     const bool p = (picked >> t) & 1u;
-    const unsigned m = __ballot_sync(0xFFFFFFFFu, p);
+    const unsigned m = __ballot_sync(kFull, p);
     if (p) out[base + __popc(m & ((1u << lane) - 1u))] = lane + 32 * t;
     base += __popc(m);
   }

@@ -99,3 +99,24 @@ def test_forward_sparse_one_call_equals_the_three_calls(lib, causal, topk):
     got = lib.qattn_forward_sparse(q, k, v, topk, causal=causal)
     torch.cuda.synchronize()
     assert torch.equal(got, ref)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("pattern", ["all_equal", "two_kinds"])
+def test_block_select_ties_bit_exact(lib, oracle, causal, pattern):
+    """Equal scores: K built from repeated 128-row tiles, so key tiles share their block means and
+    their scores tie exactly; the selection must take the lowest-indexed among equal scores, as
+    the oracle does."""
+    w = WORKLOADS["tiny"].with_(B=1, H=2, Hkv=1, N=128 * 24, d=128, causal=causal)
+    q, k, _ = make_inputs(w)
+    tile = k[:, :, :128, :]
+    if pattern == "all_equal":
+        k = tile.repeat(1, 1, 24, 1).contiguous()
+    else:
+        other = k[:, :, 128:256, :]
+        k = torch.cat([tile if (t % 3) else other for t in range(24)], dim=2).contiguous()
+    for topk in (1, 3, 7):
+        gl, gc = lib.qattn_block_select(q.cuda(), k.cuda(), topk, causal=causal)
+        torch.cuda.synchronize()
+        rl, rc = oracle.block_select(np16(q), np16(k), w.B, w.H, w.Hkv, w.N, w.d, causal, topk)
+        _lists_equal(gl, gc, rl, rc)
