@@ -19,8 +19,8 @@
 //    ex2, P packed to fp16 and written back over the scores' tensor-memory columns, row sum of the
 //    fp16-rounded P; lazy rescaling of O only when the running max grows by more than 2^8; P
 //    scaled into the top of the fp16 range; the two warpgroups' steps are kept half a step apart
-//    (each starts a step when the other is half through its exponentials), so the MUFU-bound
-//    passes of the two tiles alternate instead of contending;
+//    (a warp starts a step when the other tile's warp on its SM sub-partition is half through its
+//    exponentials), so the MUFU-bound passes of the two tiles alternate instead of contending;
 //  * causal: key tiles above the diagonal are never loaded or multiplied; the diagonal tile is
 //    masked in registers (a compile-time-specialised path); CTAs are launched heaviest-first;
 //  * grouped-query attention: query head h reads kv head h / (H / Hkv); CTAs of the heads that
@@ -77,7 +77,7 @@ struct __align__(16) AttnBars {
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t pv_done[2];
-  uint64_t mx_done[2];  // Q tile w's softmax half through a step's exponentials (4 arrives)
+  uint64_t mx_done[2][4];  // warp (w, quadrant) half through a step's exponentials (1 arrive)
   uint32_t tmem_base;
   int abort;
 };
@@ -430,7 +430,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&bars->s_full[w], 1);
       mbar_init(&bars->p_full[w], 4);  // one arrive per softmax warp of the Q tile
       mbar_init(&bars->pv_done[w], 1);
-      mbar_init(&bars->mx_done[w], 4);
+      for (int qd = 0; qd < 4; ++qd) mbar_init(&bars->mx_done[w][qd], 1);
     }
     bars->abort = 0;
     fence_mbar_init();
@@ -577,16 +577,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float nks0 = (2 * nkt_next < nkb) ? __ldg(ksc + 2 * nkt_next) : 0.0f;
         const float nks1 = (2 * nkt_next + 1 < nkb) ? __ldg(ksc + 2 * nkt_next + 1) : 0.0f;
         // The two Q tiles' softmax steps are kept half a step apart, so that their MUFU-bound
-        // exponential passes do not run at the same time: tile 1's step j starts once tile 0's
-        // step j is half through its exponentials, tile 0's step j once tile 1's step j - 1 is
-        // (mx_done[w], one arrive per warp per step).  Without this the two tiles settle nearly in
-        // phase and each step's softmax runs ~40 % longer.  Tile 0 has no step nw0 (causal, one
-        // key tile fewer than tile 1), so tile 1's last step is not gated; neither barrier gets two
-        // phases ahead of its waiter, since each tile's next arrive needs the other's.
+        // exponential passes do not run at the same time: tile 1's warp of a TMEM lane quadrant
+        // (and SM sub-partition) starts step j once tile 0's warp of that quadrant is half through
+        // its exponentials of step j, tile 0's warp starts step j once tile 1's is half through
+        // step j - 1 (mx_done[w][quadrant], one arrive per step).  Without this the two tiles
+        // settle nearly in phase and each step's softmax runs ~40 % longer.  Tile 0 has no step
+        // nw0 (causal, one key tile fewer than tile 1), so tile 1's last step is not gated;
+        // neither barrier gets two phases ahead of its waiter, since each warp's next arrive needs
+        // its partner's.
         if (wt == 1 && j < nw0)
-          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->mx_done[0], static_cast<uint32_t>(j) & 1u, abort));
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->mx_done[0][warp & 3], static_cast<uint32_t>(j) & 1u, abort));
         else if (wt == 0 && j > 0 && j - 1 < nw1)
-          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->mx_done[1], static_cast<uint32_t>(j - 1) & 1u, abort));
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->mx_done[1][warp & 3], static_cast<uint32_t>(j - 1) & 1u, abort));
         if (!ok) break;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full[wt], static_cast<uint32_t>(j) & 1u, abort));
         if (!ok) break;
@@ -607,8 +609,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const bool masked = __any_sync(0xFFFFFFFFu, lim < kBN - 1);
         float alpha;
         bool need;
-        if (masked) softmax_row<true>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, &bars->mx_done[wt]);
-        else softmax_row<false>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, &bars->mx_done[wt]);
+        if (masked) softmax_row<true>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, &bars->mx_done[wt][warp & 3]);
+        else softmax_row<false>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, &bars->mx_done[wt][warp & 3]);
         if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
           // O holds PV up to tile j-1 (complete: QK(j) was issued after PV(j-1)), and PV(j)
           // waits for this warp's arrive below.
