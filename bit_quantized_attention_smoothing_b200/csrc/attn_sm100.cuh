@@ -24,7 +24,8 @@
 //  * causal: key tiles above the diagonal are never loaded or multiplied; the diagonal tile is
 //    masked in registers (a compile-time-specialised path); CTAs are launched heaviest-first;
 //  * grouped-query attention: query head h reads kv head h / (H / Hkv); CTAs of the heads that
-//    share a kv head are adjacent in launch order so their K/V tiles are reused from L2.
+//    share a kv head are adjacent in launch order so their K/V tiles are reused from L2
+//    (non-causal: the pairs of one head run together, since each reads the head's whole K/V).
 //
 // Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d), O_1 [256+d,256+2d).
 #pragma once
@@ -394,9 +395,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int nkt = (N + kBN - 1) / kBN;
   const int nkb = (N + 63) / 64;
   const int BH = B * H;
-  int pair = blockIdx.x / BH;
-  const int bh = blockIdx.x % BH;
-  if (CAUSAL) pair = npairs - 1 - pair;
+  // Launch order.  Causal: pairs heaviest first, all heads of a pair together (the K/V prefix
+  // they read is shared by the heads of a kv head and stays in L2).  Non-causal: every CTA reads
+  // its head's whole K/V, so the pairs of one head run together and reuse it from L2 (all heads at
+  // once would need every head's K/V resident).
+  const int pair = CAUSAL ? npairs - 1 - static_cast<int>(blockIdx.x / BH)
+                          : static_cast<int>(blockIdx.x % npairs);
+  const int bh = CAUSAL ? static_cast<int>(blockIdx.x % BH) : static_cast<int>(blockIdx.x / npairs);
   const int b = bh / H;
   const int h = bh % H;
   const int g = h / (H / Hkv);
