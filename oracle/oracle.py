@@ -72,6 +72,16 @@ def lib():
         L.oracle_block_scores.restype = None
         L.oracle_select_blocks.argtypes = [P, i, i, i, i, i, P, P]
         L.oracle_select_blocks.restype = None
+        L.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_e2m1_decode.restype = ctypes.c_double
+        L.oracle_e2m1_encode.argtypes = [ctypes.c_float]
+        L.oracle_e2m1_encode.restype = ctypes.c_uint8
+        L.oracle_ue4m3_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_ue4m3_decode.restype = ctypes.c_double
+        L.oracle_ue4m3_encode.argtypes = [ctypes.c_float]
+        L.oracle_ue4m3_encode.restype = ctypes.c_uint8
+        L.oracle_quant_nvfp4.argtypes = [P, P, i, i, i, i, P, P, P]
+        L.oracle_quant_nvfp4.restype = i
         _lib = L
     return _lib
 
@@ -263,3 +273,57 @@ def forward(q, k, v, B, H, Hkv, N, d, causal, rows=None, nthreads=0, smooth=True
     out = attention_quantized(sq["q_i8"], sq["q_scale"], sq["k_i8"], sq["k_scale"], v,
                               B, H, Hkv, N, d, causal, rows=rows, nthreads=nthreads)
     return out, sq
+
+
+# ---- NVFP4 quantization (the FP4 path's operand format; the C file states the readings) ----
+
+def e2m1_encode(x: float) -> int:
+    return int(lib().oracle_e2m1_encode(float(x)))
+
+
+def e2m1_decode(code: int) -> float:
+    return lib().oracle_e2m1_decode(int(code))
+
+
+def ue4m3_encode(x: float) -> int:
+    return int(lib().oracle_ue4m3_encode(float(x)))
+
+
+def ue4m3_decode(code: int) -> float:
+    return lib().oracle_ue4m3_decode(int(code))
+
+
+def quant_nvfp4(x, mean=None, along_rows=False):
+    """NVFP4 codes of fp16 x [S, R, C] (optionally minus mean [S, C]).
+
+    Returns (codes uint8, scales uint8, gscale float32 [S]); codes hold two E2M1 codes per byte
+    (lower index in the low nibble).  along_rows=False: 16-blocks along C, codes [S, R, C/2],
+    scales [S, R, C/16].  along_rows=True: 16-blocks along R, transposed, R padded with zeros to
+    Rp = 16 * ceil(R / 16): codes [S, C, Rp/2], scales [S, C, Rp/16]."""
+    x = _bits16(x)
+    S, R, C = x.shape
+    Rp = -(-R // 16) * 16
+    if along_rows:
+        codes = np.zeros((S, C, Rp // 2), dtype=np.uint8)
+        scales = np.zeros((S, C, Rp // 16), dtype=np.uint8)
+    else:
+        codes = np.zeros((S, R, C // 2), dtype=np.uint8)
+        scales = np.zeros((S, R, C // 16), dtype=np.uint8)
+    g = np.zeros(S, dtype=np.float32)
+    mp = None if mean is None else _ptr(np.ascontiguousarray(mean, dtype=np.float32))
+    rc = lib().oracle_quant_nvfp4(_ptr(x), mp, S, R, C, 1 if along_rows else 0, _ptr(codes),
+                                  _ptr(scales), _ptr(g))
+    if rc != 0:
+        raise ValueError("oracle_quant_nvfp4: bad argument")
+    return codes, scales, g
+
+
+def nvfp4_dequant(codes, scales, gscale):
+    """float64 values of NVFP4 data laid out as quant_nvfp4 returns it: [S, rows, 2 * bytes]."""
+    e2m1 = np.array([e2m1_decode(c) for c in range(16)])
+    e4m3 = np.array([ue4m3_decode(c) if c != 0x7F else np.nan for c in range(256)])
+    lo = e2m1[codes & 15]
+    hi = e2m1[codes >> 4]
+    vals = np.stack([lo, hi], axis=-1).reshape(codes.shape[:-1] + (2 * codes.shape[-1],))
+    sc = np.repeat(e4m3[scales], 16, axis=-1) * np.asarray(gscale, dtype=np.float64)[:, None, None]
+    return vals * sc

@@ -445,3 +445,150 @@ void oracle_select_blocks(const double* scores, int B, int H, int N, int causal,
         }
     free(pick);
 }
+
+/* ------------------------------------------------------------------------------------------------
+ * NVFP4 quantization: the operand format of the FP4 path of the ThriftAttention page
+ * ("ThriftAttention: Selective Mixed Precision for Long-Context FP4 Attention",
+ * gist.science/ja/paper/2605.23081, method section, "FP4 path": the blocks that are not promoted
+ * to FP16 are computed in FP4 using the NVFP4 micro-scaling format of Blackwell GPUs).
+ * The page names the format but does not define it.  The reading used here is the format as NVIDIA
+ * publishes it: FP4 E2M1 elements in blocks of 16, one unsigned FP8 E4M3 scale per block and one
+ * binary32 scale per tensor; the tensor is one (batch, head) slice.  Steps, every binary32
+ * operation rounded once to nearest-even:
+ *   x'    = (float)x - mean[c]          (mean optional: the smoothing of K, subtracted per channel)
+ *   amax  = max |x'| over the slice;    g = amax / 2688  (2688 = 448 * 6: largest scale * largest
+ *                                                         element)
+ *   per block of 16:  bmax = max |x'|;  s = E4M3(bmax / (6 * g))   (6 * g rounded first)
+ *                     sc = s * g;       code_i = E2M1(x'_i / sc)
+ *   decoded value x^ = E2M1value(code) * E4M3value(s) * g.
+ * Both conversions round to nearest, ties to even, and saturate to the largest finite value
+ * (448, 6).  A block whose scale rounds to 0, and every block of a slice with amax == 0, gets
+ * scale byte 0 and codes 0.  A code whose value is zero is written as +0 (code 0).
+ * Packing: two codes per byte, the element with the lower index in bits 0-3.
+ * ---------------------------------------------------------------------------------------------- */
+
+/* E2M1 value of a 4-bit code: 1 sign bit, 2 exponent bits (bias 1), 1 fraction bit; exponent 0
+ * encodes 0 and 0.5 (subnormal), no infinities or NaN.  Magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+double oracle_e2m1_decode(uint8_t code) {
+    int e = (code >> 1) & 3, m = code & 1;
+    double v = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return (code & 8) ? -v : v;
+}
+
+/* Nearest E2M1 code to x, ties to the even fraction bit, |x| >= 6 saturating to 6.  Inside each
+ * binade of the format the representable magnitudes are the integer multiples of one spacing
+ * (0.5 below 2, 1 in [2, 4), 2 in [4, 8)), so rounding is rint(|x| / spacing) with ties to even,
+ * and an even multiple is exactly an even fraction bit. */
+uint8_t oracle_e2m1_encode(float x) {
+    double m = fabs((double)x);
+    double spacing = (m < 2.0) ? 0.5 : (m < 4.0) ? 1.0 : 2.0;
+    double v = rint(m / spacing) * spacing;    /* exact: spacing is a power of two */
+    if (v > 6.0) v = 6.0;
+    uint8_t mag;
+    if (v < 2.0) mag = (uint8_t)(v * 2.0);                      /* 0, 0.5, 1, 1.5 -> 0..3 */
+    else if (v < 4.0) mag = (uint8_t)(4 + (int)(v - 2.0));      /* 2, 3 -> 4, 5 */
+    else mag = (uint8_t)(v == 4.0 ? 6 : 7);                     /* 4, 6 -> 6, 7 */
+    if (mag == 0) return 0;
+    return (x < 0.0f) ? (uint8_t)(mag | 8) : mag;
+}
+
+/* Value of an unsigned E4M3 byte (the FP8 E4M3 format with the sign bit 0): 4 exponent bits
+ * (bias 7), 3 fraction bits; exponent 0 encodes subnormals m * 2^-9; 0x7F is NaN, 448 the
+ * largest finite value. */
+double oracle_ue4m3_decode(uint8_t code) {
+    int e = (code >> 3) & 15, m = code & 7;
+    if (code == 0x7F) return NAN;
+    return (e == 0) ? ldexp((double)m, -9) : ldexp((double)(8 + m), e - 10);
+}
+
+/* Nearest E4M3 byte to x >= 0, ties to the even fraction bit, values above 448 saturating to 448. */
+uint8_t oracle_ue4m3_encode(float x) {
+    double v = (double)x;
+    if (!(v > 0.0)) return 0;
+    if (v >= 448.0) return 0x7E;
+    if (v < ldexp(1.0, -6)) {                  /* subnormal range: units of 2^-9 */
+        return (uint8_t)rint(ldexp(v, 9));     /* 8 is the smallest normal, code 0x08: still right */
+    }
+    int e;
+    (void)frexp(v, &e);
+    e -= 1;                                    /* v in [2^e, 2^(e+1)), e in [-6, 8] */
+    double q = rint(ldexp(v, 3 - e));          /* 4-bit significand in [8, 16] */
+    if (q == 16.0) { q = 8.0; e += 1; }
+    int code = ((e + 7) << 3) | ((int)q - 8);
+    return (uint8_t)(code > 0x7E ? 0x7E : code);
+}
+
+/* One block of 16 values (binary32, already smoothed) with the slice's global scale g. */
+static void nvfp4_block(const float* x, float g, uint8_t* codes16, uint8_t* scale) {
+    float bmax = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        float a = fabsf(x[i]);
+        if (a > bmax) bmax = a;
+    }
+    uint8_t s = 0;
+    if (g > 0.0f) {
+        float sixg = 6.0f * g;
+        float t = bmax / sixg;
+        s = oracle_ue4m3_encode(t);
+    }
+    *scale = s;
+    if (s == 0) {
+        for (int i = 0; i < 16; ++i) codes16[i] = 0;
+        return;
+    }
+    float sc = (float)oracle_ue4m3_decode(s) * g;   /* the E4M3 value is exact in binary32 */
+    for (int i = 0; i < 16; ++i) {
+        float q = x[i] / sc;
+        codes16[i] = oracle_e2m1_encode(q);
+    }
+}
+
+/* x: fp16 [S][R][C]; mean: binary32 [S][C] or NULL.
+ * along_rows == 0: blocks of 16 consecutive channels of one row (C % 16 == 0);
+ *   codes [S][R][C/2] bytes, scales [S][R][C/16].
+ * along_rows == 1: blocks of 16 consecutive rows of one channel, written transposed; rows
+ *   R .. Rp-1 (Rp = R rounded up to 16) are zero padding;
+ *   codes [S][C][Rp/2] bytes, scales [S][C][Rp/16].
+ * gscale [S]: g of each slice.  Returns 0, or -1 on a bad argument. */
+int oracle_quant_nvfp4(const uint16_t* x, const float* mean, int S, int R, int C, int along_rows,
+                       uint8_t* codes, uint8_t* scales, float* gscale) {
+    if (S < 1 || R < 1 || C < 1) return -1;
+    if (!along_rows && C % 16 != 0) return -1;
+    int Rp = (R + 15) / 16 * 16;
+    float* xs = (float*)malloc(sizeof(float) * (size_t)R * C);
+    float blk[16];
+    uint8_t c16[16];
+    for (long s = 0; s < S; ++s) {
+        float amax = 0.0f;
+        for (long r = 0; r < R; ++r)
+            for (int c = 0; c < C; ++c) {
+                float v = (float)oracle_f16_to_f64(x[(s * R + r) * C + c]);
+                if (mean) v = v - mean[s * C + c];
+                xs[r * C + c] = v;
+                if (fabsf(v) > amax) amax = fabsf(v);
+            }
+        float g = amax / 2688.0f;
+        gscale[s] = g;
+        if (!along_rows) {
+            for (long r = 0; r < R; ++r)
+                for (int b = 0; b < C / 16; ++b) {
+                    nvfp4_block(xs + r * C + b * 16, g, c16, scales + (s * R + r) * (C / 16) + b);
+                    uint8_t* out = codes + (s * R + r) * (C / 2) + b * 8;
+                    for (int i = 0; i < 8; ++i) out[i] = (uint8_t)(c16[2 * i] | (c16[2 * i + 1] << 4));
+                }
+        } else {
+            for (int c = 0; c < C; ++c)
+                for (int b = 0; b < Rp / 16; ++b) {
+                    for (int i = 0; i < 16; ++i) {
+                        long r = (long)b * 16 + i;
+                        blk[i] = (r < R) ? xs[r * C + c] : 0.0f;
+                    }
+                    nvfp4_block(blk, g, c16, scales + (s * C + c) * (Rp / 16) + b);
+                    uint8_t* out = codes + (s * C + c) * (Rp / 2) + b * 8;
+                    for (int i = 0; i < 8; ++i) out[i] = (uint8_t)(c16[2 * i] | (c16[2 * i + 1] << 4));
+                }
+        }
+    }
+    free(xs);
+    return 0;
+}

@@ -1,0 +1,208 @@
+"""Pins of the oracle's NVFP4 quantizer (no GPU).
+
+The FP4 path of the ThriftAttention page (gist.science/ja/paper/2605.23081, method section, "FP4
+path") computes its blocks in the NVFP4 micro-scaling format: E2M1 elements, one unsigned E4M3
+scale per 16 elements and one binary32 scale per tensor (here per (batch, head) slice).  The
+encoders are pinned to torch's float8_e4m3fn conversion and to brute-force nearest searches over
+the formats' value sets; the block quantizer to closed-form inputs (values on the E2M1 grid times
+a power of two come back unchanged), to a transposition identity, to the smoothing identity and to
+the zero and tiny-scale special cases.
+"""
+import numpy as np
+import pytest
+import torch
+
+# E2M1 magnitudes of codes 0..7 as the format lists them (sign in bit 3).
+E2M1_MAG = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def _e2m1_bruteforce(x):
+    """Nearest E2M1 code to x over the 15 distinct values; ties to the code with fraction bit 0;
+    a zero result is code 0."""
+    best = None
+    for code in range(16):
+        v = E2M1_MAG[code & 7] * (-1.0 if code & 8 else 1.0)
+        if code == 8:
+            continue  # -0: zero is written as code 0
+        dist = abs(float(x) - v)
+        if best is None or dist < best[0] or (dist == best[0] and (code & 1) == 0 and best[1] & 1):
+            best = (dist, code)
+    return best[1]
+
+
+def _e4m3_torch(x):
+    t = torch.tensor(np.asarray(x, dtype=np.float32).ravel()).to(torch.float8_e4m3fn)
+    return t.view(torch.uint8).numpy()
+
+
+def test_e2m1_decode_table(oracle):
+    got = [oracle.e2m1_decode(c) for c in range(16)]
+    want = E2M1_MAG + [-v for v in E2M1_MAG]
+    assert got == want
+
+
+def test_e2m1_encode_bruteforce(oracle):
+    rng = np.random.default_rng(11)
+    grid = np.arange(-9.0, 9.0, 1.0 / 64)                     # every tie and midpoint of the grid
+    mids = [(a + b) / 2 for a, b in zip(E2M1_MAG, E2M1_MAG[1:])]
+    xs = np.concatenate([grid, mids, [-m for m in mids], rng.standard_normal(3000) * 3,
+                         [1e-30, -1e-30, 0.0, -0.0, 6.0, 6.9, 7.0, 1e9, -1e9]]).astype(np.float32)
+    for x in xs:
+        assert oracle.e2m1_encode(float(x)) == _e2m1_bruteforce(x), float(x)
+
+
+def test_ue4m3_decode_vs_torch(oracle):
+    codes = np.arange(127, dtype=np.uint8)
+    ref = torch.tensor(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.ue4m3_decode(int(c)) for c in codes])
+    np.testing.assert_array_equal(got, ref)
+    assert oracle.ue4m3_decode(0x7E) == 448.0
+
+
+def test_ue4m3_encode_vs_torch_in_range(oracle):
+    vals = torch.arange(127, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mids = (vals[:-1] + vals[1:]) / 2
+    rng = np.random.default_rng(12)
+    xs = np.concatenate([vals, mids, np.nextafter(mids, 0), np.nextafter(mids, 1e9),
+                         rng.uniform(0, 448, 4000), 2.0 ** rng.uniform(-14, 8.8, 4000)])
+    xs = xs[(xs >= 0) & (xs <= 448)].astype(np.float32)
+    ref = _e4m3_torch(xs)
+    got = np.array([oracle.ue4m3_encode(float(x)) for x in xs], dtype=np.uint8)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, [(float(xs[i]), int(got[i]), int(ref[i])) for i in bad[:5]]
+
+
+def test_ue4m3_encode_saturates(oracle):
+    for x in [448.0, 448.5, 463.9, 464.0, 480.0, 1e4, 3e38]:
+        assert oracle.ue4m3_encode(x) == 0x7E
+    assert oracle.ue4m3_encode(0.0) == 0 and oracle.ue4m3_encode(2.0 ** -11) == 0
+    assert oracle.ue4m3_encode(2.0 ** -10) == 0          # tie between 0 and 2^-9: even code 0
+    assert oracle.ue4m3_encode(3 * 2.0 ** -10) == 2      # tie between 2^-9 and 2^-8: even code 2
+
+
+def _grid_slices(rng, S, R, C, along_rows):
+    """fp16 slices whose values are E2M1 grid values times 2^-3, every 16-block with a maximum of
+    6, 3 or 1.5 (times 2^-3) and at least one block per slice with maximum 6.  Returns the fp16
+    array (in the quantizer's input layout) and the expected codes of every element, in block
+    layout [S, rows, blocks, 16]."""
+    rows, cols = (C, R) if along_rows else (R, C)       # rows of blocks, then the blocked axis
+    nb = cols // 16
+    vals = np.zeros((S, rows, nb, 16))
+    codes = np.zeros((S, rows, nb, 16), dtype=np.int64)
+    code_of = {v: i for i, v in enumerate(E2M1_MAG)}
+    for s in range(S):
+        for r in range(rows):
+            for b in range(nb):
+                top = 6.0 if (r == 0 and b == 0) else rng.choice([6.0, 3.0, 1.5])
+                mult = 6.0 / top                           # the factor the scale will apply
+                allowed = [v for v in E2M1_MAG if v <= top]
+                mag = rng.choice(allowed, size=16)
+                mag[rng.integers(16)] = top
+                sign = rng.choice([-1.0, 1.0], size=16)
+                vals[s, r, b] = sign * mag / 8
+                for i in range(16):
+                    c = code_of[mag[i] * mult]
+                    codes[s, r, b, i] = 0 if c == 0 else c | (8 if sign[i] < 0 else 0)
+    x = vals.reshape(S, rows, cols)
+    if along_rows:
+        x = x.transpose(0, 2, 1)
+    return np.ascontiguousarray(x.astype(np.float16)), codes
+
+
+def _unpack(codes):
+    return np.stack([codes & 15, codes >> 4], axis=-1).reshape(codes.shape[:-1] + (-1,))
+
+
+@pytest.mark.parametrize("along_rows", [False, True])
+def test_nvfp4_grid_values_come_back_exactly(oracle, along_rows):
+    rng = np.random.default_rng(13 + along_rows)
+    S, R, C = 2, 48, 64
+    x, want = _grid_slices(rng, S, R, C, along_rows)
+    codes, scales, g = oracle.quant_nvfp4(x, along_rows=along_rows)
+    got = _unpack(codes).reshape(want.shape)
+    np.testing.assert_array_equal(got, want)
+    # scale of a block = E4M3(448 * bmax / amax): 448, 224, 112 for maxima 6, 3, 1.5
+    bmax = np.abs(x.astype(np.float64)).transpose(0, 2, 1) if along_rows else np.abs(x.astype(np.float64))
+    bmax = bmax.reshape(want.shape).max(-1) * 8
+    expect_scale = np.select([bmax == 6, bmax == 3, bmax == 1.5], [0x7E, 0x76, 0x6E])
+    np.testing.assert_array_equal(scales.reshape(expect_scale.shape), expect_scale)
+    assert np.all(g == np.float32(0.75) / np.float32(2688))
+    # and the decoded values are the inputs up to the rounding of g (relative 2^-23)
+    deq = oracle.nvfp4_dequant(codes, scales, g)
+    xin = x.astype(np.float64).transpose(0, 2, 1) if along_rows else x.astype(np.float64)
+    np.testing.assert_allclose(deq, xin, rtol=3e-7, atol=0)
+
+
+def test_nvfp4_transposed_equals_rows_of_the_transpose(oracle):
+    rng = np.random.default_rng(14)
+    S, R, C = 3, 37, 24                                    # ragged R, C not a multiple of 16
+    x = (rng.standard_normal((S, R, C)) * np.exp(rng.standard_normal((S, 1, C)))).astype(np.float16)
+    codes, scales, g = oracle.quant_nvfp4(x, along_rows=True)
+    Rp = 48
+    xt = np.zeros((S, C, Rp), dtype=np.float16)
+    xt[:, :, :R] = x.transpose(0, 2, 1)
+    c2, s2, g2 = oracle.quant_nvfp4(xt, along_rows=False)
+    np.testing.assert_array_equal(codes, c2)
+    np.testing.assert_array_equal(scales, s2)
+    np.testing.assert_array_equal(g, g2)
+    assert not np.any(_unpack(codes)[:, :, R:])            # padding rows are code 0
+
+
+def test_nvfp4_mean_is_subtracted(oracle):
+    rng = np.random.default_rng(15)
+    S, R, C = 2, 20, 32
+    x = (rng.integers(-256, 257, size=(S, R, C)) / 64).astype(np.float16)   # exact in fp16
+    mean = (rng.integers(-32, 33, size=(S, C)) / 8).astype(np.float32)
+    diff = (x.astype(np.float64) - mean[:, None, :]).astype(np.float16)     # |diff| < 8: exact
+    assert np.array_equal(diff.astype(np.float64), x.astype(np.float64) - mean[:, None, :])
+    for along_rows in (False, True):
+        a = oracle.quant_nvfp4(x, mean=mean, along_rows=along_rows)
+        b = oracle.quant_nvfp4(diff, along_rows=along_rows)
+        for u, v in zip(a, b):
+            np.testing.assert_array_equal(u, v)
+
+
+def test_nvfp4_zero_and_tiny_blocks(oracle):
+    x = np.zeros((3, 16, 32), dtype=np.float16)
+    x[1, 0, 0] = 1000.0                                    # amax of slice 1
+    x[1, 1, :16] = 1e-4                                    # scale 1e-4 / (6 g) < 2^-10 -> 0
+    x[1, 2, :16] = 0.01                                    # subnormal E4M3 scale
+    x[2, :, :] = -0.0
+    codes, scales, g = oracle.quant_nvfp4(x)
+    assert g[0] == 0 and g[2] == 0
+    assert not codes[0].any() and not scales[0].any() and not codes[2].any() and not scales[2].any()
+    assert scales[1, 0, 0] == 0x7E and (codes[1, 0, 0] & 15) == 7     # 1000 -> 6 * 448 * g
+    assert scales[1, 1, 0] == 0 and not codes[1, 1, :8].any()
+    t = np.float32(np.float16(0.01)) / (np.float32(6) * g[1])
+    assert scales[1, 2, 0] == _e4m3_torch([t])[0] and 0 < scales[1, 2, 0] < 8
+
+
+def test_nvfp4_random_blocks_against_independent_encoders(oracle):
+    """Every scale byte is torch's E4M3 of bmax / (6 g) and every code the brute-force nearest
+    E2M1 of x / sc (binary32 quotients, numpy float32 arithmetic); the decoded error is at most
+    one scale step below saturation."""
+    rng = np.random.default_rng(16)
+    S, R, C = 2, 24, 64
+    x = rng.standard_normal((S, R, C)) * np.exp(2 * rng.standard_normal((S, R, 1)))
+    x[0, 3, 5] = 300.0                                     # an outlier sets the slice scale
+    x = x.astype(np.float16)
+    mean = rng.standard_normal((S, C)).astype(np.float32) * 0.1
+    codes, scales, g = oracle.quant_nvfp4(x, mean=mean)
+    xs = x.astype(np.float32) - mean[:, None, :]
+    blocks = xs.reshape(S, R, C // 16, 16)
+    bmax = np.abs(blocks).max(-1)
+    t = bmax / (np.float32(6) * g[:, None, None])
+    np.testing.assert_array_equal(scales, _e4m3_torch(t).reshape(scales.shape))
+    e4 = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    sc = e4[scales] * g[:, None, None]
+    q = blocks / sc[..., None]
+    got = _unpack(codes).reshape(blocks.shape)
+    flat_q, flat_c = q.ravel(), got.ravel()
+    for i in range(0, flat_q.size, 7):                     # a seventh of the elements, all kinds
+        assert flat_c[i] == _e2m1_bruteforce(flat_q[i]), (i, float(flat_q[i]))
+    deq = oracle.nvfp4_dequant(codes, scales, g).reshape(blocks.shape)
+    err = np.abs(deq - blocks.astype(np.float64))
+    unsat = np.abs(q) <= 6
+    assert np.all(err[unsat] <= 1.0001 * np.broadcast_to(sc[..., None], q.shape)[unsat])
+    # the block holding the slice maximum has the largest scale and a code of magnitude 6
+    assert scales[0, 3, 0] == 0x7E and (got[0, 3, 0, 5] & 7) == 7
