@@ -15,6 +15,7 @@
 #include "attn_sm100.cuh"
 #include "quant.cuh"
 #include "block_sparse.cuh"
+#include "nvfp4.cuh"
 
 namespace {
 
@@ -714,6 +715,45 @@ qattn_status qattn_debug_wait_timeout(long long limit_cycles, int* gave_up,
   if (s != QATTN_OK) return s;
   wait_timeout_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_cycles,
                                                                                   gave_up);
+  return launch_status();
+}
+
+qattn_status qattn_quant_nvfp4(const void* x, const float* mean, int S, int R, int C,
+                               int along_rows, uint8_t* codes, uint8_t* scales, float* gscale,
+                               qattn_stream_t stream) {
+  if (S < 1 || R < 1 || C < 1) return QATTN_ERR_INVALID_ARG;
+  if (C % 16 != 0 || S > 65535 || static_cast<long long>(R) * C > (1LL << 31))
+    return QATTN_ERR_UNSUPPORTED;
+  qattn_status s = check_ptrs(x, codes, scales, gscale);
+  if (s != QATTN_OK) return s;
+  if (mean && !aligned16(mean)) return QATTN_ERR_MISALIGNED;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const uint16_t* xh = static_cast<const uint16_t*>(x);
+  unsigned* amax_bits = reinterpret_cast<unsigned*>(gscale);
+  if (cudaMemsetAsync(gscale, 0, sizeof(float) * static_cast<size_t>(S), st) != cudaSuccess)
+    return QATTN_ERR_CUDA;
+  // slice maxima: about 16 resident CTAs per SM over all slices, at least 4 vectors a thread
+  const long long nvec = static_cast<long long>(R) * C / 8;
+  long long gx = (nvec + 1023) / 1024;
+  const long long cap = (148LL * 16 + S - 1) / S;
+  if (gx > cap) gx = cap;
+  if (gx < 1) gx = 1;
+  nvfp4_amax_kernel<<<dim3(static_cast<unsigned>(gx), S), 256, 0, st>>>(xh, mean, R, C, amax_bits);
+  if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
+  if (along_rows) {
+    const int Rp = (R + 15) / 16 * 16;
+    const dim3 grid((Rp + kNvfp4Tile - 1) / kNvfp4Tile, (C + kNvfp4Tile - 1) / kNvfp4Tile, S);
+    nvfp4_quant_cols_kernel<<<grid, 256, 0, st>>>(xh, mean, R, C, Rp, amax_bits, codes, scales);
+  } else {
+    const long long total = static_cast<long long>(S) * R * (C / 16);
+    long long blocks = (total + 255) / 256;
+    if (blocks > 148LL * 32) blocks = 148LL * 32;
+    nvfp4_quant_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(xh, mean, R, C, total,
+                                                                          amax_bits, codes, scales);
+  }
+  if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
+  nvfp4_finalize_kernel<<<(S + 255) / 256, 256, 0, st>>>(gscale, S);
   return launch_status();
 }
 

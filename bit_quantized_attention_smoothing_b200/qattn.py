@@ -32,7 +32,7 @@ EXPORTS = [
     "qattn_forward_sparse",
     "qattn_forward_workspace", "qattn_forward_ws", "qattn_forward",
     "qattn_forward_host", "qattn_debug_qk_int32", "qattn_debug_wait_timeout",
-    "qattn_check_device_status",
+    "qattn_quant_nvfp4", "qattn_check_device_status",
 ]
 
 
@@ -95,6 +95,8 @@ def _lib():
         L.qattn_debug_qk_int32.restype = i
         L.qattn_debug_wait_timeout.argtypes = [ctypes.c_longlong, P, P]
         L.qattn_debug_wait_timeout.restype = i
+        L.qattn_quant_nvfp4.argtypes = [P, P, i, i, i, i, P, P, P, P]
+        L.qattn_quant_nvfp4.restype = i
         L.qattn_check_device_status.argtypes = [P]
         L.qattn_check_device_status.restype = i
         _L = L
@@ -250,6 +252,32 @@ def qattn_attn_quantized_sparse(q_i8, q_scale, k_i8, k_scale, v, kv_list, kv_cou
                                             _p(kv_list), _p(kv_count), _stream(stream))
     _check("qattn_attn_quantized_sparse", st)
     return out
+
+
+def qattn_quant_nvfp4(x, mean=None, along_rows=False, stream=None):
+    """NVFP4 quantization of fp16 x [S, R, C] (optionally minus mean, float32 [S, C]).
+
+    Returns (codes, scales, gscale): uint8 codes with two E2M1 codes per byte, uint8 E4M3 block
+    scales, float32 [S] slice scales.  along_rows=False: 16-blocks along C, codes [S, R, C/2],
+    scales [S, R, C/16]; along_rows=True: 16-blocks along R, transposed and zero-padded to
+    Rp = 16 * ceil(R / 16): codes [S, C, Rp/2], scales [S, C, Rp/16]."""
+    assert x.dim() == 3 and x.dtype == torch.float16, "x: fp16 [S, R, C]"
+    S, R, C = x.shape
+    if mean is not None:
+        assert mean.dtype == torch.float32 and tuple(mean.shape) == (S, C), "mean: float32 [S, C]"
+    dev = x.device
+    if along_rows:
+        Rp = -(-R // 16) * 16
+        codes = torch.empty(S, C, Rp // 2, dtype=torch.uint8, device=dev)
+        scales = torch.empty(S, C, Rp // 16, dtype=torch.uint8, device=dev)
+    else:
+        codes = torch.empty(S, R, C // 2, dtype=torch.uint8, device=dev)
+        scales = torch.empty(S, R, max(C // 16, 1), dtype=torch.uint8, device=dev)
+    gscale = torch.empty(S, dtype=torch.float32, device=dev)
+    st = _lib().qattn_quant_nvfp4(_p(x), _p(mean), S, R, C, int(bool(along_rows)), _p(codes),
+                                  _p(scales), _p(gscale), _stream(stream))
+    _check("qattn_quant_nvfp4", st)
+    return codes, scales, gscale
 
 
 def qattn_forward_workspace(B: int, H: int, Hkv: int, N: int, d: int) -> int:

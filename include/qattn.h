@@ -211,6 +211,37 @@ qattn_status qattn_forward_host(const void* q_host, const void* k_host, const vo
                                 qattn_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * NVFP4 quantization: the operand format of the FP4 path on the ThriftAttention page
+ * ("ThriftAttention: Selective Mixed Precision for Long-Context FP4 Attention",
+ * gist.science/ja/paper/2605.23081, method section, "FP4 path": the blocks not promoted to FP16
+ * are computed in FP4 with Blackwell's NVFP4 micro-scaling format).  The page does not define
+ * the format; this follows NVIDIA's published definition.
+ * ------------------------------------------------------------------------------------------ */
+
+/* Quantizes fp16 x [S][R][C] (S independent slices, e.g. the (batch, head) slices of Q, K or V)
+ * to NVFP4: E2M1 codes, one unsigned E4M3 scale byte per 16 values, one binary32 scale per slice.
+ * With binary32 operations rounded once to nearest-even:
+ *   x' = (float)x - mean[s][c] (mean: binary32 [S][C], or NULL for none; the smoothing of K),
+ *   g = max|x'| over the slice / 2688,
+ *   per block of 16: s = E4M3(max|x'| / (6 * g)), code = E2M1(x' / (E4M3value(s) * g)),
+ * both conversions nearest-even and saturating (448, 6); decoded x' ~ E2M1value * E4M3value * g.
+ * A block whose scale rounds to 0 (and every block of an all-zero slice) has scale 0, codes 0;
+ * a zero code is always +0.  Two codes per byte, the lower-indexed element in bits 0-3.
+ *   along_rows == 0: blocks of 16 consecutive channels of a row (Q and K along d);
+ *     codes uint8 [S][R][C/2], scales uint8 [S][R][C/16].
+ *   along_rows != 0: blocks of 16 consecutive rows of a channel, written transposed (V along the
+ *     tokens, the contraction dimension of P V); rows R .. Rp-1, Rp = R rounded up to 16, are
+ *     zero padding; codes uint8 [S][C][Rp/2], scales uint8 [S][C][Rp/16].
+ *   gscale: float [S], the g of each slice (also used as scratch during the call).
+ * Requirements: C % 16 == 0, S <= 65535, R * C <= 2^31; all pointers device, 16-byte aligned.
+ * Errors: INVALID_ARG for non-positive sizes or a NULL buffer (mean may be NULL), UNSUPPORTED
+ * for the limits above, MISALIGNED, CUDA.  Three kernels and one memset on `stream`; results
+ * are a deterministic function of the inputs (bit-exact against a plain CPU implementation). */
+qattn_status qattn_quant_nvfp4(const void* x, const float* mean, int S, int R, int C,
+                               int along_rows, uint8_t* codes, uint8_t* scales, float* gscale,
+                               qattn_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * Checks.
  * ------------------------------------------------------------------------------------------ */
 

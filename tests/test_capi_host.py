@@ -114,3 +114,19 @@ def test_workspace_and_alignment_checks():
 def test_forward_sparse_argument_checks(args, expect):
     L = Q.load()
     assert L.qattn_forward_sparse(*args) == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((None, None, 2, 64, 128, 0, P(16), P(32), P(48), None), 1),        # null x
+    ((P(16), None, 2, 64, 128, 0, P(16), None, P(48), None), 1),        # null scales
+    ((P(16), None, 0, 64, 128, 0, P(16), P(32), P(48), None), 1),       # S < 1
+    ((P(16), None, 2, 0, 128, 1, P(16), P(32), P(48), None), 1),        # R < 1
+    ((P(16), None, 2, 64, 120, 0, P(16), P(32), P(48), None), 2),       # C % 16 != 0
+    ((P(16), None, 65536, 64, 128, 0, P(16), P(32), P(48), None), 2),   # S past the grid limit
+    ((P(16), None, 1, 1 << 24, 256, 1, P(16), P(32), P(48), None), 2),  # R * C > 2^31
+    ((P(16), P(20), 2, 64, 128, 0, P(16), P(32), P(48), None), 3),      # misaligned mean
+    ((P(16), None, 2, 64, 128, 0, P(16), P(32), P(52), None), 3),       # misaligned gscale
+])
+def test_quant_nvfp4_argument_checks(args, expect):
+    L = Q.load()
+    assert L.qattn_quant_nvfp4(*args) == expect

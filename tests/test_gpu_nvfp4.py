@@ -1,0 +1,140 @@
+"""NVFP4 quantization on the GPU against the oracle (FP4 path of the ThriftAttention page, method
+section; the format per NVIDIA's definition: E2M1 codes, E4M3 scale per 16 values, binary32
+scale per slice).
+
+Codes, block scales and slice scales are integer / bit-pattern results of the same binary32
+operations on both sides, so every byte and every float is compared exactly: small ragged cases
+of both block directions with and without a channel mean, the degenerate cases (all-zero slice,
+blocks whose scale rounds to 0, fp16 subnormals, a single row), the workload generator's Q, K
+(smoothed with the oracle's channel means) and V, and at full size (Q, K, V of the 32K-token
+Llama-8B-shaped workload, the launch shapes a full-size FP4 path would use) sampled slices.
+"""
+import numpy as np
+import pytest
+import torch
+
+from bit_quantized_attention_smoothing_b200.workloads import WORKLOADS, make_inputs
+from conftest import np16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from bit_quantized_attention_smoothing_b200 import qattn as Q
+    Q.load()
+    return Q
+
+
+def _draw(kind, S, R, C, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((S, R, C))
+    if kind == "rowscale":
+        x *= np.exp(1.5 * rng.standard_normal((S, R, 1)))
+    elif kind == "channel":
+        x = x * np.exp(rng.standard_normal((S, 1, C))) + 3 * rng.standard_normal((S, 1, C))
+    elif kind == "outlier":
+        idx = rng.integers(0, x.size, size=max(1, x.size // 500))
+        x.flat[idx] *= 200.0
+    elif kind == "zero_slice":
+        x[0] = 0.0
+        x[1, :3] *= 1e-5                      # blocks whose E4M3 scale rounds to 0 or is subnormal
+        x[1, 5, :16] = -0.0
+    elif kind == "tiny":
+        x *= 3e-6                             # fp16 subnormals
+    return np.clip(x, -60000, 60000).astype(np.float16)
+
+
+def _compare(lib, oracle, x16, mean, along_rows):
+    xg = torch.from_numpy(x16).cuda()
+    mg = None if mean is None else torch.from_numpy(mean).cuda()
+    codes, scales, g = lib.qattn_quant_nvfp4(xg, mg, along_rows=along_rows)
+    torch.cuda.synchronize()
+    rc, rs, rg = oracle.quant_nvfp4(x16, mean=mean, along_rows=along_rows)
+    c, s, gg = codes.cpu().numpy(), scales.cpu().numpy(), g.cpu().numpy()
+    assert c.shape == rc.shape and s.shape == rs.shape
+    assert np.array_equal(gg.view(np.uint32), rg.view(np.uint32)), (gg, rg)
+    bad = np.argwhere(s != rs)
+    assert bad.size == 0, f"{bad.shape[0]} scale bytes differ, first at {bad[0]}: {s[tuple(bad[0])]} vs {rs[tuple(bad[0])]}"
+    bad = np.argwhere(c != rc)
+    assert bad.size == 0, f"{bad.shape[0]} code bytes differ, first at {bad[0]}: {c[tuple(bad[0])]:#04x} vs {rc[tuple(bad[0])]:#04x}"
+    return c, s, gg
+
+
+CASES = [
+    (3, 200, 128, False, False, "rowscale"),
+    (3, 200, 128, True, False, "rowscale"),
+    (2, 37, 48, True, True, "channel"),
+    (2, 37, 48, False, True, "channel"),
+    (4, 1000, 64, True, True, "outlier"),
+    (4, 1000, 64, False, True, "outlier"),
+    (1, 1, 16, False, False, "normal"),
+    (1, 1, 16, True, False, "normal"),
+    (2, 130, 128, False, False, "zero_slice"),
+    (2, 130, 128, True, False, "zero_slice"),
+    (5, 64, 80, True, False, "tiny"),
+    (5, 64, 80, False, True, "tiny"),
+]
+
+
+@pytest.mark.parametrize("S,R,C,along_rows,with_mean,kind", CASES,
+                         ids=[f"S{c[0]}-R{c[1]}-C{c[2]}-{'rows' if c[3] else 'cols'}-"
+                              f"{'mean' if c[4] else 'nomean'}-{c[5]}" for c in CASES])
+def test_quant_nvfp4_bit_exact(lib, oracle, S, R, C, along_rows, with_mean, kind):
+    x = _draw(kind, S, R, C, seed=S * 1000 + R + C + 7 * along_rows)
+    mean = None
+    if with_mean:
+        mean = np.random.default_rng(R).standard_normal((S, C)).astype(np.float32)
+    _compare(lib, oracle, x, mean, along_rows)
+
+
+def test_quant_nvfp4_workload_q_k_v(lib, oracle):
+    """The attention operands of a small workload: Q and smoothed K along d (K's mean is the
+    oracle's exact channel mean), V along the tokens."""
+    w = WORKLOADS["llama8b_32k"].with_(H=4, Hkv=2, N=1500)
+    q, k, v = make_inputs(w, device="cpu")
+    sums = oracle.k_channel_sums(np16(k), w.B, w.Hkv, w.N, w.d)
+    mean = np.array([oracle.lib().oracle_mean_from_sum(int(s), w.N) for s in sums.ravel()],
+                    dtype=np.float32).reshape(w.B * w.Hkv, w.d)
+    qs = q.reshape(w.B * w.H, w.N, w.d).numpy()
+    ks = k.reshape(w.B * w.Hkv, w.N, w.d).numpy()
+    vs = v.reshape(w.B * w.Hkv, w.N, w.d).numpy()
+    _compare(lib, oracle, qs, None, False)
+    _compare(lib, oracle, ks, mean, False)
+    _compare(lib, oracle, vs, None, True)
+
+
+def test_quant_nvfp4_full_size_sampled_slices(lib, oracle):
+    """Q [32 x 32768 x 128], K [8 x 32768 x 128] and V (along the tokens) of the 32K-token
+    workload quantized whole on the GPU; the oracle recomputes sampled slices (each slice's
+    result depends only on that slice)."""
+    w = WORKLOADS["llama8b_32k"]
+    q, k, v = make_inputs(w, device="cuda")
+    for x, along_rows, picks in ((q, False, (0, w.H - 1)), (k, False, (3,)), (v, True, (5,))):
+        S = x.shape[0] * x.shape[1]
+        xs = x.reshape(S, w.N, w.d)
+        codes, scales, g = lib.qattn_quant_nvfp4(xs, None, along_rows=along_rows)
+        torch.cuda.synchronize()
+        for s in picks:
+            x16 = np16(xs[s:s + 1])
+            rc, rs, rg = oracle.quant_nvfp4(x16.view(np.float16), along_rows=along_rows)
+            assert np.array_equal(g[s:s + 1].cpu().numpy().view(np.uint32), rg.view(np.uint32))
+            assert np.array_equal(scales[s:s + 1].cpu().numpy(), rs)
+            assert np.array_equal(codes[s:s + 1].cpu().numpy(), rc)
+        del codes, scales, g
+    assert lib.qattn_check_device_status() == 0
+
+
+def test_quant_nvfp4_dequantized_error(lib, oracle):
+    """The decoded GPU result stays within one block-scale step of the input below saturation
+    (the format's own bound: half the largest E2M1 spacing, 2, times the block scale)."""
+    x16 = _draw("rowscale", 2, 256, 128, seed=3)
+    c, s, g = _compare(lib, oracle, x16, None, False)
+    deq = oracle.nvfp4_dequant(c, s, g)
+    e4 = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    sc = np.repeat(e4[s], 16, axis=-1) * g.astype(np.float64)[:, None, None]
+    err = np.abs(deq - x16.astype(np.float64))
+    sat = np.abs(x16.astype(np.float64)) > 6 * sc
+    assert np.all(err[~sat] <= 1.0001 * sc[~sat])
