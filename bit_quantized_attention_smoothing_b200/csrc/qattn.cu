@@ -16,6 +16,7 @@
 #include "quant.cuh"
 #include "block_sparse.cuh"
 #include "nvfp4.cuh"
+#include "fp4_sm100.cuh"
 
 namespace {
 
@@ -100,6 +101,13 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem
 bool make_i8_map(CUtensorMap* m, const void* base, int d, int N, long long outer) {
   return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, outer, d, 128,
                   d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+// NVFP4 codes [outer][N][d/2] bytes: tiles of 128 rows x d/2 bytes, swizzled to match the
+// FP4 MMA descriptors (64-byte rows for d = 128, 32-byte rows for d = 64).
+bool make_fp4_map(CUtensorMap* m, const void* base, int d, int N, long long outer) {
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d / 2, N, outer, d / 2, 128,
+                  d == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
 // fp16 V [outer][N][d]: boxes of 64 columns (128 bytes) x 128 rows, 128-byte swizzle.
@@ -703,6 +711,46 @@ qattn_status qattn_debug_qk_int32(const int8_t* q_i8, const int8_t* k_i8, int32_
                              smem) != cudaSuccess)
       return QATTN_ERR_CUDA;
     qk_int32_kernel<64><<<grid, 128, smem, st>>>(tq, tk, s_out, bh, bg, qt0, kt0, nkt * 128);
+  }
+  return launch_status();
+}
+
+qattn_status qattn_debug_qk_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales,
+                                  const float* q_g, const uint8_t* k_codes,
+                                  const uint8_t* k_scales, const float* k_g, float* s_out, int B,
+                                  int H, int Hkv, int N, int d, int b, int h, int qt0, int nqt,
+                                  int kt0, int nkt, qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q_codes, q_scales, q_g, k_codes, k_scales, k_g, s_out);
+  if (s != QATTN_OK) return s;
+  const int ntiles = (N + 127) / 128;
+  if (b < 0 || b >= B || h < 0 || h >= H || qt0 < 0 || nqt < 1 || kt0 < 0 || nkt < 1 ||
+      qt0 + nqt > ntiles || kt0 + nkt > ntiles || nqt > 65535 || nkt > 65535)
+    return QATTN_ERR_INVALID_ARG;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  CUtensorMap tq, tk;
+  if (!make_fp4_map(&tq, q_codes, d, N, static_cast<long long>(B) * H) ||
+      !make_fp4_map(&tk, k_codes, d, N, static_cast<long long>(B) * Hkv))
+    return QATTN_ERR_CUDA;
+  // 100 KB of shared memory per CTA caps residency at 2 CTAs (512 TMEM columns) per SM.
+  const int smem = 100 * 1024;
+  const int bh = b * H + h;
+  const int bg = b * Hkv + h / (H / Hkv);
+  dim3 grid(nqt, nkt);
+  if (d == 128) {
+    if (cudaFuncSetAttribute(qk_nvfp4_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return QATTN_ERR_CUDA;
+    qk_nvfp4_kernel<128><<<grid, 128, smem, st>>>(tq, tk, q_scales, k_scales, q_g, k_g, s_out, N,
+                                                  bh, bg, qt0, kt0, nkt * 128);
+  } else {
+    if (cudaFuncSetAttribute(qk_nvfp4_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return QATTN_ERR_CUDA;
+    qk_nvfp4_kernel<64><<<grid, 128, smem, st>>>(tq, tk, q_scales, k_scales, q_g, k_g, s_out, N,
+                                                 bh, bg, qt0, kt0, nkt * 128);
   }
   return launch_status();
 }

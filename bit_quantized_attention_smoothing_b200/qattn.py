@@ -32,7 +32,7 @@ EXPORTS = [
     "qattn_forward_sparse",
     "qattn_forward_workspace", "qattn_forward_ws", "qattn_forward",
     "qattn_forward_host", "qattn_debug_qk_int32", "qattn_debug_wait_timeout",
-    "qattn_quant_nvfp4", "qattn_check_device_status",
+    "qattn_quant_nvfp4", "qattn_debug_qk_nvfp4", "qattn_check_device_status",
 ]
 
 
@@ -97,6 +97,8 @@ def _lib():
         L.qattn_debug_wait_timeout.restype = i
         L.qattn_quant_nvfp4.argtypes = [P, P, i, i, i, i, P, P, P, P]
         L.qattn_quant_nvfp4.restype = i
+        L.qattn_debug_qk_nvfp4.argtypes = [P, P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, i, P]
+        L.qattn_debug_qk_nvfp4.restype = i
         L.qattn_check_device_status.argtypes = [P]
         L.qattn_check_device_status.restype = i
         _L = L
@@ -323,6 +325,20 @@ def qattn_debug_qk_int32(q_i8, k_i8, b, h, qt0, nqt, kt0, nkt, s_out=None, strea
     st = _lib().qattn_debug_qk_int32(_p(q_i8), _p(k_i8), _p(s_out), B, H, Hkv, N, d, b, h, qt0,
                                      nqt, kt0, nkt, _stream(stream))
     _check("qattn_debug_qk_int32", st)
+    return s_out
+
+
+def qattn_debug_qk_nvfp4(q_nvfp4, k_nvfp4, B, H, Hkv, N, d, b, h, qt0, nqt, kt0, nkt,
+                         s_out=None, stream=None):
+    """FP4 score tiles from NVFP4 Q and K, each the (codes, scales, gscale) triple that
+    qattn_quant_nvfp4 returns along the channels (slices B*H for Q, B*Hkv for K)."""
+    qc, qs, qg = q_nvfp4
+    kc, ks, kg = k_nvfp4
+    if s_out is None:
+        s_out = torch.empty(nqt * 128, nkt * 128, dtype=torch.float32, device=qc.device)
+    st = _lib().qattn_debug_qk_nvfp4(_p(qc), _p(qs), _p(qg), _p(kc), _p(ks), _p(kg), _p(s_out),
+                                     B, H, Hkv, N, d, b, h, qt0, nqt, kt0, nkt, _stream(stream))
+    _check("qattn_debug_qk_nvfp4", st)
     return s_out
 
 

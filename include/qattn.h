@@ -254,6 +254,21 @@ qattn_status qattn_debug_qk_int32(const int8_t* q_i8, const int8_t* k_i8, int32_
                                   int H, int Hkv, int N, int d, int b, int h, int qt0, int nqt,
                                   int kt0, int nkt, qattn_stream_t stream);
 
+/* FP4 score tiles through the block-scaled tensor cores: S = gQ gK * sum over the d channels of
+ * E2M1(q) E4M3(sq) * E2M1(k) E4M3(sk), i.e. the dot products of the decoded NVFP4 rows, computed
+ * by TMA -> tcgen05.mma kind::mxf4nvf4 (block16 UE4M3 scales in tensor memory, f32 accumulator)
+ * -> tcgen05.ld: the Q K^T of the FP4 path (ThriftAttention page, method section, "FP4 path").
+ * Inputs as qattn_quant_nvfp4 writes them along the channels with S = B*H slices for Q and
+ * B*Hkv for K: q_codes [B*H][N][d/2], q_scales [B*H][N][d/16], q_g [B*H]; k_* likewise with Hkv.
+ * Tiles as in qattn_debug_qk_int32 (query tiles qt0 .. qt0+nqt-1, key tiles kt0 .. kt0+nkt-1 of
+ * batch b, query head h, its kv head h / (H / Hkv)); s_out: device float [nqt*128][nkt*128],
+ * rows or keys past N read as zero. */
+qattn_status qattn_debug_qk_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales,
+                                  const float* q_g, const uint8_t* k_codes,
+                                  const uint8_t* k_scales, const float* k_g, float* s_out, int B,
+                                  int H, int Hkv, int N, int d, int b, int h, int qt0, int nqt,
+                                  int kt0, int nkt, qattn_stream_t stream);
+
 /* Failure-detection check: launches one block that waits on an mbarrier nothing arrives on,
  * with a wait limit of limit_cycles SM clock cycles (0 .. the kernels' own limit of 2e9), so the
  * bounded-wait path runs out on purpose.  The kernel then records QATTN_ERR_TIMEOUT in the device

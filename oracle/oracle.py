@@ -5,8 +5,10 @@ leg are the only callers.  The product (the CUDA library and its Python binding)
 this module.
 
 The C source states the method and the readings it follows (SageAttention summary page,
-aibr.jp/archives/102657, sec. 2-4).  This wrapper only marshals numpy arrays; every step of the
-arithmetic is in the C file.  fp16 arrays travel as their uint16 bit patterns.
+aibr.jp/archives/102657, sec. 2-4).  This wrapper marshals numpy arrays; every step of the INT8
+path's arithmetic is in the C file.  The NVFP4 quantizer is in the C file too; decoding NVFP4 data
+and the FP4 score product (decode, then a float64 matmul) are the numpy functions at the end.
+fp16 arrays travel as their uint16 bit patterns.
 """
 from __future__ import annotations
 
@@ -327,3 +329,25 @@ def nvfp4_dequant(codes, scales, gscale):
     vals = np.stack([lo, hi], axis=-1).reshape(codes.shape[:-1] + (2 * codes.shape[-1],))
     sc = np.repeat(e4m3[scales], 16, axis=-1) * np.asarray(gscale, dtype=np.float64)[:, None, None]
     return vals * sc
+
+
+def qk_nvfp4(q_codes, q_scales, q_g, k_codes, k_scales, k_g, H, Hkv, b, h, r0, nr, c0, nc):
+    """FP4 scores of batch b, query head h: rows r0 .. r0+nr-1 of Q against keys c0 .. c0+nc-1
+    of the kv head h // (H // Hkv), from NVFP4 data laid out as quant_nvfp4 writes it along the
+    channels (slices = batch * heads).  S = sum over channels of decoded q * decoded k, i.e. per
+    16-channel block the exact integer-valued product sum of the E2M1 codes times the two E4M3
+    block scales, times gQ * gK; float64.  Rows or keys past the end read as zero.  Returns
+    (S, M) with M = |Q| |K|^T, the magnitude sum that bounds accumulation error."""
+    bh = b * H + h
+    bg = b * Hkv + h // (H // Hkv)
+
+    def rows(codes, scales, g, s, r, n):
+        sl = slice(r, min(r + n, codes.shape[1]))
+        x = nvfp4_dequant(codes[s:s + 1, sl], scales[s:s + 1, sl], np.asarray(g)[s:s + 1])[0]
+        out = np.zeros((n, x.shape[1]))
+        out[: x.shape[0]] = x
+        return out
+
+    Q = rows(q_codes, q_scales, q_g, bh, r0, nr)
+    K = rows(k_codes, k_scales, k_g, bg, c0, nc)
+    return Q @ K.T, np.abs(Q) @ np.abs(K).T

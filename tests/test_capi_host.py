@@ -130,3 +130,14 @@ def test_forward_sparse_argument_checks(args, expect):
 def test_quant_nvfp4_argument_checks(args, expect):
     L = Q.load()
     assert L.qattn_quant_nvfp4(*args) == expect
+
+
+def test_debug_qk_nvfp4_argument_checks():
+    L = Q.load()
+    a = (P(16), P(32), P(48), P(64), P(80), P(96), P(112))
+    assert L.qattn_debug_qk_nvfp4(None, *a[1:], 1, 4, 2, 256, 128, 0, 0, 0, 1, 0, 1, None) == 1
+    assert L.qattn_debug_qk_nvfp4(*a, 1, 4, 3, 256, 128, 0, 0, 0, 1, 0, 1, None) == 1    # H % Hkv
+    assert L.qattn_debug_qk_nvfp4(*a, 1, 4, 2, 256, 128, 0, 0, 1, 2, 0, 1, None) == 1    # tiles
+    assert L.qattn_debug_qk_nvfp4(*a, 1, 4, 2, 256, 128, 0, 4, 0, 1, 0, 1, None) == 1    # head
+    assert L.qattn_debug_qk_nvfp4(*a, 1, 4, 2, 256, 96, 0, 0, 0, 1, 0, 1, None) == 2     # d
+    assert L.qattn_debug_qk_nvfp4(P(17), *a[1:], 1, 4, 2, 256, 128, 0, 0, 0, 1, 0, 1, None) == 3

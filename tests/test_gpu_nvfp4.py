@@ -138,3 +138,89 @@ def test_quant_nvfp4_dequantized_error(lib, oracle):
     err = np.abs(deq - x16.astype(np.float64))
     sat = np.abs(x16.astype(np.float64)) > 6 * sc
     assert np.all(err[~sat] <= 1.0001 * sc[~sat])
+
+
+# ---- FP4 scores through tcgen05.mma kind::mxf4nvf4 (block16 UE4M3 scales) ----
+#
+# The tensor core sums 16-element E2M1 products (exact) weighted by the two block scales into an
+# f32 accumulator; against the exact float64 score the only error is the f32 accumulation over
+# the d / 16 blocks and the final product with gQ gK, a few units of 2^-24 of the magnitude sum
+# M = |Q| |K|^T.  The bound used: |S_gpu - S| <= 2^-20 * M.
+FP4_REL = 2.0 ** -20
+
+
+def _check_scores(got, S, M, what):
+    err = np.abs(got.astype(np.float64) - S)
+    ratio = float((err / np.maximum(M, 1e-300)).max())
+    print(what, "max |err| / M =", ratio)
+    assert np.all(err <= FP4_REL * M + 1e-30), (what, ratio)
+
+
+def _upload(t):
+    return tuple(torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in t)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_qk_nvfp4_random_codes_and_scales(lib, oracle, d):
+    """Arbitrary code bytes and per-block scale bytes (no quantizer structure), so that every
+    block's scale is independent: checks where each scale byte lands in tensor memory."""
+    rng = np.random.default_rng(40 + d)
+    B, H, Hkv, N = 1, 2, 1, 300
+    qc = rng.integers(0, 256, size=(B * H, N, d // 2), dtype=np.uint8)
+    kc = rng.integers(0, 256, size=(B * Hkv, N, d // 2), dtype=np.uint8)
+    qs = rng.integers(0x20, 0x50, size=(B * H, N, d // 16), dtype=np.uint8)
+    ks = rng.integers(0x20, 0x50, size=(B * Hkv, N, d // 16), dtype=np.uint8)
+    qg = np.array([1.0, 0.5], dtype=np.float32)
+    kg = np.array([2.0], dtype=np.float32)
+    gq, gk = _upload((qc, qs, qg)), _upload((kc, ks, kg))
+    nt = 3
+    for h in range(H):
+        got = lib.qattn_debug_qk_nvfp4(gq, gk, B, H, Hkv, N, d, 0, h, 0, nt, 0, nt).cpu().numpy()
+        S, M = oracle.qk_nvfp4(qc, qs, qg, kc, ks, kg, H, Hkv, 0, h, 0, nt * 128, 0, nt * 128)
+        _check_scores(got, S, M, f"random d{d} h{h}")
+    assert lib.qattn_check_device_status() == 0
+
+
+@pytest.mark.parametrize("name,over", [("llama8b_32k", {"H": 4, "Hkv": 2, "N": 700}),
+                                       ("wide64", {"B": 2, "H": 2, "Hkv": 1, "N": 333})])
+def test_qk_nvfp4_on_oracle_quantized_workload(lib, oracle, name, over):
+    """The workload's Q and smoothed K, quantized by the oracle, scored on the tensor cores."""
+    w = WORKLOADS[name].with_(**over)
+    q, k, _ = make_inputs(w, device="cpu")
+    sums = oracle.k_channel_sums(np16(k), w.B, w.Hkv, w.N, w.d)
+    mean = np.array([oracle.lib().oracle_mean_from_sum(int(s), w.N) for s in sums.ravel()],
+                    dtype=np.float32).reshape(w.B * w.Hkv, w.d)
+    qn = oracle.quant_nvfp4(q.reshape(w.B * w.H, w.N, w.d).numpy())
+    kn = oracle.quant_nvfp4(k.reshape(w.B * w.Hkv, w.N, w.d).numpy(), mean=mean)
+    gq, gk = _upload(qn), _upload(kn)
+    nt = -(-w.N // 128)
+    for b, h in {(0, 0), (w.B - 1, w.H - 1)}:
+        got = lib.qattn_debug_qk_nvfp4(gq, gk, w.B, w.H, w.Hkv, w.N, w.d, b, h, 0, nt, 0, nt)
+        S, M = oracle.qk_nvfp4(*qn, *kn, w.H, w.Hkv, b, h, 0, nt * 128, 0, nt * 128)
+        _check_scores(got.cpu().numpy(), S, M, f"{name} b{b} h{h}")
+
+
+def test_qk_nvfp4_full_size_tiles(lib, oracle):
+    """32K-token Q and smoothed K quantized on the GPU (the codes checked equal to the oracle's
+    for the slices used), FP4 score tiles at the corners and the middle of the score matrix."""
+    w = WORKLOADS["llama8b_32k"]
+    q, k, _ = make_inputs(w, device="cuda")
+    h, g = w.H - 1, (w.H - 1) // (w.H // w.Hkv)
+    sums = oracle.k_channel_sums(np16(k[:, g:g + 1]), 1, 1, w.N, w.d)
+    mean1 = np.array([oracle.lib().oracle_mean_from_sum(int(s), w.N) for s in sums.ravel()],
+                     dtype=np.float32)
+    mean = torch.zeros(w.B * w.Hkv, w.d, dtype=torch.float32, device="cuda")
+    mean[g] = torch.from_numpy(mean1).cuda()
+    gq = lib.qattn_quant_nvfp4(q.reshape(w.H, w.N, w.d))
+    gk = lib.qattn_quant_nvfp4(k.reshape(w.Hkv, w.N, w.d), mean)
+    qn = oracle.quant_nvfp4(np16(q[0, h:h + 1]).view(np.float16))
+    kn = oracle.quant_nvfp4(np16(k[0, g:g + 1]).view(np.float16), mean=mean1[None])
+    for mine, ref, s in ((gq, qn, h), (gk, kn, g)):
+        for a, r in zip(mine, ref):
+            assert np.array_equal(a[s:s + 1].cpu().numpy(), r)
+    nt = w.N // 128
+    for qt, kt in {(0, 0), (nt - 1, nt - 1), (nt - 1, 0), (nt // 2, nt // 3)}:
+        got = lib.qattn_debug_qk_nvfp4(gq, gk, w.B, w.H, w.Hkv, w.N, w.d, 0, h, qt, 1, kt, 1)
+        S, M = oracle.qk_nvfp4(qn[0], qn[1], qn[2], kn[0], kn[1], kn[2], 1, 1, 0, 0,
+                               qt * 128, 128, kt * 128, 128)
+        _check_scores(got.cpu().numpy(), S, M, f"full qt{qt} kt{kt}")

@@ -206,3 +206,39 @@ def test_nvfp4_random_blocks_against_independent_encoders(oracle):
     assert np.all(err[unsat] <= 1.0001 * np.broadcast_to(sc[..., None], q.shape)[unsat])
     # the block holding the slice maximum has the largest scale and a code of magnitude 6
     assert scales[0, 3, 0] == 0x7E and (got[0, 3, 0, 5] & 7) == 7
+
+
+def test_qk_nvfp4_exact_on_power_of_two_scales(oracle):
+    """With slice maxima 2688 * 2^k the slice scales g are powers of two, every decoded value is
+    a short dyadic rational and the float64 product is exact: it must equal the score summed with
+    Python fractions from the codes and scale bytes (format tables, not the oracle's decoder)."""
+    from fractions import Fraction
+    rng = np.random.default_rng(21)
+    d, N = 64, 40
+    q = (rng.standard_normal((2, N, d)) * 2).astype(np.float16)
+    k = (rng.standard_normal((1, N, d)) * 2).astype(np.float16)
+    q[0, 0, 0] = 2688 * 2.0 ** -8        # 10.5: slice maxima set g = 2^-8 and 2^-7
+    q[1, 3, 7] = -2688 * 2.0 ** -7
+    k[0, 5, 9] = 2688 * 2.0 ** -7
+    qc, qs, qg = oracle.quant_nvfp4(q)
+    kc, ks, kg = oracle.quant_nvfp4(k)
+    assert list(qg) == [2.0 ** -8, 2.0 ** -7] and list(kg) == [2.0 ** -7]
+    S, M = oracle.qk_nvfp4(qc, qs, qg, kc, ks, kg, H=2, Hkv=1, b=0, h=1, r0=0, nr=8, c0=30, nc=16)
+    e4 = torch.arange(127, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mag = [Fraction(v).limit_denominator(4) for v in E2M1_MAG]
+
+    def dec(codes, scales, s, r, c):
+        byte = int(codes[s, r, c // 2])
+        nib = (byte >> 4) if c % 2 else (byte & 15)
+        v = mag[nib & 7] * (-1 if nib & 8 else 1)
+        return v * Fraction(float(e4[scales[s, r, c // 16]]))
+
+    for i in range(8):
+        for j in range(16):
+            kr = 30 + j
+            if kr >= N:
+                assert S[i, j] == 0 and M[i, j] == 0
+                continue
+            want = sum(dec(qc, qs, 1, i, c) * dec(kc, ks, 0, kr, c) for c in range(d))
+            want *= Fraction(2.0 ** -7) * Fraction(2.0 ** -7)
+            assert Fraction(S[i, j]) == want
