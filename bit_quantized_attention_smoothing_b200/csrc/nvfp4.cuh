@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(256) nvfp4_quant_rows_kernel(
 
 // Blocks along the rows, written transposed: CTA (bx, by, s) quantizes rows 64 bx .. 64 bx + 63
 // of channels 64 by .. 64 by + 63 of slice s.  Rows R .. Rp - 1 are zero padding (Rp = R rounded
-// up to 16).  codes [S][C][Rp/2], scales [S][C][Rp/16].  256 threads; C % 16 == 0.
+// up to 128).  codes [S][C][Rp/2], scales [S][C][Rp/16].  256 threads; C % 16 == 0.
 __global__ void __launch_bounds__(256) nvfp4_quant_cols_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ mean, int R, int C, int Rp,
     const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes,

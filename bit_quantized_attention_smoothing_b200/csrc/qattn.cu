@@ -790,7 +790,7 @@ qattn_status qattn_quant_nvfp4(const void* x, const float* mean, int S, int R, i
   nvfp4_amax_kernel<<<dim3(static_cast<unsigned>(gx), S), 256, 0, st>>>(xh, mean, R, C, amax_bits);
   if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
   if (along_rows) {
-    const int Rp = (R + 15) / 16 * 16;
+    const int Rp = (R + 127) / 128 * 128;
     const dim3 grid((Rp + kNvfp4Tile - 1) / kNvfp4Tile, (C + kNvfp4Tile - 1) / kNvfp4Tile, S);
     nvfp4_quant_cols_kernel<<<grid, 256, 0, st>>>(xh, mean, R, C, Rp, amax_bits, codes, scales);
   } else {

@@ -262,14 +262,14 @@ def qattn_quant_nvfp4(x, mean=None, along_rows=False, stream=None):
     Returns (codes, scales, gscale): uint8 codes with two E2M1 codes per byte, uint8 E4M3 block
     scales, float32 [S] slice scales.  along_rows=False: 16-blocks along C, codes [S, R, C/2],
     scales [S, R, C/16]; along_rows=True: 16-blocks along R, transposed and zero-padded to
-    Rp = 16 * ceil(R / 16): codes [S, C, Rp/2], scales [S, C, Rp/16]."""
+    Rp = 128 * ceil(R / 128): codes [S, C, Rp/2], scales [S, C, Rp/16]."""
     assert x.dim() == 3 and x.dtype == torch.float16, "x: fp16 [S, R, C]"
     S, R, C = x.shape
     if mean is not None:
         assert mean.dtype == torch.float32 and tuple(mean.shape) == (S, C), "mean: float32 [S, C]"
     dev = x.device
     if along_rows:
-        Rp = -(-R // 16) * 16
+        Rp = -(-R // 128) * 128
         codes = torch.empty(S, C, Rp // 2, dtype=torch.uint8, device=dev)
         scales = torch.empty(S, C, Rp // 16, dtype=torch.uint8, device=dev)
     else:

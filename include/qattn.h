@@ -230,8 +230,9 @@ qattn_status qattn_forward_host(const void* q_host, const void* k_host, const vo
  *   along_rows == 0: blocks of 16 consecutive channels of a row (Q and K along d);
  *     codes uint8 [S][R][C/2], scales uint8 [S][R][C/16].
  *   along_rows != 0: blocks of 16 consecutive rows of a channel, written transposed (V along the
- *     tokens, the contraction dimension of P V); rows R .. Rp-1, Rp = R rounded up to 16, are
- *     zero padding; codes uint8 [S][C][Rp/2], scales uint8 [S][C][Rp/16].
+ *     tokens, the contraction dimension of P V); rows R .. Rp-1, Rp = R rounded up to 128 (one
+ *     key tile, so that every row of codes and of scales starts 16-byte aligned), are zero
+ *     padding; codes uint8 [S][C][Rp/2], scales uint8 [S][C][Rp/16].
  *   gscale: float [S], the g of each slice (also used as scratch during the call).
  * Requirements: C % 16 == 0, S <= 65535, R * C <= 2^31; all pointers device, 16-byte aligned.
  * Errors: INVALID_ARG for non-positive sizes or a NULL buffer (mean may be NULL), UNSUPPORTED

@@ -84,6 +84,9 @@ def lib():
         L.oracle_ue4m3_encode.restype = ctypes.c_uint8
         L.oracle_quant_nvfp4.argtypes = [P, P, i, i, i, i, P, P, P]
         L.oracle_quant_nvfp4.restype = i
+        L.oracle_attention_nvfp4.argtypes = [P, P, P, P, P, P, P, P, P, i, i, i, i, i, i, i, P, P,
+                                             ctypes.c_long, P, P]
+        L.oracle_attention_nvfp4.restype = i
         _lib = L
     return _lib
 
@@ -301,10 +304,10 @@ def quant_nvfp4(x, mean=None, along_rows=False):
     Returns (codes uint8, scales uint8, gscale float32 [S]); codes hold two E2M1 codes per byte
     (lower index in the low nibble).  along_rows=False: 16-blocks along C, codes [S, R, C/2],
     scales [S, R, C/16].  along_rows=True: 16-blocks along R, transposed, R padded with zeros to
-    Rp = 16 * ceil(R / 16): codes [S, C, Rp/2], scales [S, C, Rp/16]."""
+    Rp = 128 * ceil(R / 128): codes [S, C, Rp/2], scales [S, C, Rp/16]."""
     x = _bits16(x)
     S, R, C = x.shape
-    Rp = -(-R // 16) * 16
+    Rp = -(-R // 128) * 128
     if along_rows:
         codes = np.zeros((S, C, Rp // 2), dtype=np.uint8)
         scales = np.zeros((S, C, Rp // 16), dtype=np.uint8)
@@ -351,3 +354,26 @@ def qk_nvfp4(q_codes, q_scales, q_g, k_codes, k_scales, k_g, H, Hkv, b, h, r0, n
     Q = rows(q_codes, q_scales, q_g, bh, r0, nr)
     K = rows(k_codes, k_scales, k_g, bg, c0, nc)
     return Q @ K.T, np.abs(Q) @ np.abs(K).T
+
+
+def attention_nvfp4(qn, kn, vn, B, H, Hkv, N, d, causal, rows=None):
+    """Rows of the FP4-path attention (every key tile in FP4; the C file states the readings).
+
+    qn, kn: (codes, scales, gscale) along the channels over B*H and B*Hkv slices; vn: the same for
+    V along the tokens (transposed).  Returns (out float64 [nrows, d], slack float64 [nrows])."""
+    row_bh, row_i = all_rows(B, H, N) if rows is None else rows
+    row_bh = np.ascontiguousarray(row_bh, dtype=np.int64)
+    row_i = np.ascontiguousarray(row_i, dtype=np.int64)
+    out = np.zeros((row_bh.size, d), dtype=np.float64)
+    slack = np.zeros(row_bh.size, dtype=np.float64)
+    c = lambda a, t: _ptr(np.ascontiguousarray(a, dtype=t))
+    Np = vn[0].shape[2] * 2
+    rc = lib().oracle_attention_nvfp4(
+        c(qn[0], np.uint8), c(qn[1], np.uint8), c(qn[2], np.float32),
+        c(kn[0], np.uint8), c(kn[1], np.uint8), c(kn[2], np.float32),
+        c(vn[0], np.uint8), c(vn[1], np.uint8), c(vn[2], np.float32),
+        B, H, Hkv, N, Np, d, 1 if causal else 0, _ptr(row_bh), _ptr(row_i), row_bh.size,
+        _ptr(out), _ptr(slack))
+    if rc != 0:
+        raise ValueError("oracle_attention_nvfp4: bad argument")
+    return out, slack

@@ -547,14 +547,14 @@ static void nvfp4_block(const float* x, float g, uint8_t* codes16, uint8_t* scal
  * along_rows == 0: blocks of 16 consecutive channels of one row (C % 16 == 0);
  *   codes [S][R][C/2] bytes, scales [S][R][C/16].
  * along_rows == 1: blocks of 16 consecutive rows of one channel, written transposed; rows
- *   R .. Rp-1 (Rp = R rounded up to 16) are zero padding;
+ *   R .. Rp-1 (Rp = R rounded up to 128, one key tile) are zero padding;
  *   codes [S][C][Rp/2] bytes, scales [S][C][Rp/16].
  * gscale [S]: g of each slice.  Returns 0, or -1 on a bad argument. */
 int oracle_quant_nvfp4(const uint16_t* x, const float* mean, int S, int R, int C, int along_rows,
                        uint8_t* codes, uint8_t* scales, float* gscale) {
     if (S < 1 || R < 1 || C < 1) return -1;
     if (!along_rows && C % 16 != 0) return -1;
-    int Rp = (R + 15) / 16 * 16;
+    int Rp = (R + 127) / 128 * 128;
     float* xs = (float*)malloc(sizeof(float) * (size_t)R * C);
     float blk[16];
     uint8_t c16[16];
@@ -590,5 +590,148 @@ int oracle_quant_nvfp4(const uint16_t* x, const float* mean, int S, int R, int C
         }
     }
     free(xs);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------------------
+ * Attention on the FP4 path (ThriftAttention page, method section: "FP4 path" computes the blocks
+ * in NVFP4; "online merge" combines blocks with FlashAttention-2's online softmax; the FP4 path's
+ * probability blocks use a two-level quantization adapted from SageAttention3, whose details the
+ * page does not give).  Every key tile here is on the FP4 path (no promotion).  Readings:
+ *   - Q (per query head) and smoothed K (per kv head) are NVFP4 along the channels, V NVFP4 along
+ *     the tokens (transposed, Np tokens per channel row); decoded values as oracle_quant_nvfp4;
+ *   - scores x_j = S_ij * log2(e) / sqrt(d) in binary64 from the decoded Q and K;
+ *   - key tiles of 128 in order; per tile m' = max(m, max_j x_j), corr = 2^(m - m'),
+ *     p_j = 2^(x_j - m') rounded to binary32;
+ *   - two-level quantization of the tile's P row: level 1, a per-row binary32 scale
+ *     gP = max_j p_j / 2688 that maps the row into the E2M1 x E4M3 range; level 2, NVFP4 blocks of
+ *     16 keys with gP as the global scale (the same binary32 steps as oracle_quant_nvfp4);
+ *   - l = l * corr + sum_j p^_j over the dequantized p^ (the values the P V product uses);
+ *     acc = acc * corr + sum_j p^_j v^_j;  out = acc / l.
+ * The GPU's scores carry f32 accumulation and its exponentials binary32 rounding, so an FP4
+ * decision taken within a relative 2^-16 of a tie may go the other way there.  For each output
+ * row the oracle also returns a slack: the sum, over such decisions, of the largest change that
+ * decision can make to the row's output (code: one E2M1 step times its scale; block scale: the
+ * whole block's p plus two steps per element), times (max |v^| + max |out|) / l.
+ * ---------------------------------------------------------------------------------------------- */
+
+static double nvfp4_value(const uint8_t* codes, const uint8_t* scales, long row, int rowlen, int j,
+                          double g) {
+    uint8_t byte = codes[row * (rowlen / 2) + j / 2];
+    uint8_t nib = (j & 1) ? (byte >> 4) : (byte & 15);
+    return oracle_e2m1_decode(nib) * oracle_ue4m3_decode(scales[row * (rowlen / 16) + j / 16]) * g;
+}
+
+/* E2M1 code of q, and whether a relative perturbation of 2^-16 could change it. */
+static int e2m1_near_tie(float q) {
+    const double d = ldexp(1.0, -16);
+    return oracle_e2m1_encode((float)(q * (1.0 - d))) != oracle_e2m1_encode((float)(q * (1.0 + d)));
+}
+
+static int ue4m3_near_tie(float t) {
+    const double d = ldexp(1.0, -16);
+    return oracle_ue4m3_encode((float)(t * (1.0 - d))) != oracle_ue4m3_encode((float)(t * (1.0 + d)));
+}
+
+/* q_codes [B*H][N][d/2], q_scales [B*H][N][d/16], q_g [B*H]; k_* likewise over B*Hkv;
+ * vt_codes [B*Hkv][d][Np/2], vt_scales [B*Hkv][d][Np/16], v_g [B*Hkv].
+ * Rows (row_bh[r], row_i[r]) for r < nrows; out [nrows][d], slack [nrows].  Returns 0, or -1 on a
+ * bad argument. */
+int oracle_attention_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales, const float* q_g,
+                           const uint8_t* k_codes, const uint8_t* k_scales, const float* k_g,
+                           const uint8_t* vt_codes, const uint8_t* vt_scales, const float* v_g,
+                           int B, int H, int Hkv, int N, int Np, int d, int causal,
+                           const long* row_bh, const long* row_i, long nrows, double* out,
+                           double* slack) {
+    if (B < 1 || H < 1 || Hkv < 1 || N < 1 || H % Hkv || d % 16 || Np < N || Np % 16) return -1;
+    const double sl2 = 1.4426950408889634 / sqrt((double)d);
+    const double rel = ldexp(1.0, -16);
+    double* q = (double*)malloc(sizeof(double) * d);
+    double* acc = (double*)malloc(sizeof(double) * d);
+    double x[128], ph[128], risk[128];
+    float p[128];
+    for (long r = 0; r < nrows; ++r) {
+        const long bh = row_bh[r], i = row_i[r];
+        const long b = bh / H, h = bh % H, bg = b * Hkv + h / (H / Hkv);
+        for (int c = 0; c < d; ++c) q[c] = nvfp4_value(q_codes, q_scales, bh * N + i, d, c, q_g[bh]);
+        const long last = causal ? i : N - 1;
+        /* l, acc: the online softmax; rv, rp: the risk sums against |v| and against |out|,
+         * rescaled with l */
+        double m = -INFINITY, l = 0.0, rv = 0.0, rp = 0.0;
+        for (int c = 0; c < d; ++c) acc[c] = 0.0;
+        for (long t0 = 0; t0 <= last; t0 += 128) {
+            const int n = (int)((last - t0 + 1) < 128 ? (last - t0 + 1) : 128);   /* visible keys */
+            double tmax = -INFINITY;
+            for (int j = 0; j < n; ++j) {
+                double sdot = 0.0;
+                for (int c = 0; c < d; ++c)
+                    sdot += q[c] * nvfp4_value(k_codes, k_scales, bg * N + t0 + j, d, c, k_g[bg]);
+                x[j] = sdot * sl2;
+                if (x[j] > tmax) tmax = x[j];
+            }
+            const double mn = m > tmax ? m : tmax;
+            const double corr = exp2(m - mn);
+            float pmax = 0.0f;
+            for (int j = 0; j < 128; ++j) {
+                p[j] = j < n ? (float)exp2(x[j] - mn) : 0.0f;
+                if (p[j] > pmax) pmax = p[j];
+                risk[j] = 0.0;
+                ph[j] = 0.0;
+            }
+            /* level 1: the row's binary32 scale; level 2: NVFP4 blocks of 16 keys */
+            const float gp = pmax / 2688.0f;
+            for (int blk = 0; blk < 8; ++blk) {
+                float bmax = 0.0f;
+                for (int e = 0; e < 16; ++e)
+                    if (p[blk * 16 + e] > bmax) bmax = p[blk * 16 + e];
+                if (!(gp > 0.0f)) continue;
+                const float sixg = 6.0f * gp;
+                const float t = bmax / sixg;
+                const uint8_t sb = oracle_ue4m3_encode(t);
+                const float sc = sb ? (float)oracle_ue4m3_decode(sb) * gp : 0.0f;
+                for (int e = 0; e < 16 && sb; ++e) {
+                    const int j = blk * 16 + e;
+                    const float qq = p[j] / sc;
+                    ph[j] = oracle_e2m1_decode(oracle_e2m1_encode(qq)) * (double)sc;
+                    if (e2m1_near_tie(qq)) {
+                        double lo = oracle_e2m1_decode(oracle_e2m1_encode((float)(qq * (1.0 - rel))));
+                        double hi = oracle_e2m1_decode(oracle_e2m1_encode((float)(qq * (1.0 + rel))));
+                        risk[j] += fabs(hi - lo) * (double)sc;
+                    }
+                }
+                if (ue4m3_near_tie(t)) {
+                    /* the scale may round to a neighbour (one E4M3 step, or 0): every p^ of the
+                     * block may move by up to its own size plus two code steps */
+                    const double big = 2.0 * 2.0 * (double)bmax / 6.0 + 1e-300;
+                    for (int e = 0; e < 16; ++e) risk[blk * 16 + e] += p[blk * 16 + e] + big;
+                }
+            }
+            l *= corr;
+            rv *= corr;
+            rp *= corr;
+            for (int c = 0; c < d; ++c) acc[c] *= corr;
+            for (int j = 0; j < n; ++j) {
+                l += ph[j];
+                double vm = 0.0;
+                for (int c = 0; c < d; ++c) {
+                    const double v = nvfp4_value(vt_codes, vt_scales, bg * d + c, Np, (int)(t0 + j),
+                                                 v_g[bg]);
+                    acc[c] += ph[j] * v;
+                    if (fabs(v) > vm) vm = fabs(v);
+                }
+                rv += risk[j] * vm;
+                rp += risk[j];
+            }
+            m = mn;
+        }
+        double omax = 0.0;
+        for (int c = 0; c < d; ++c) {
+            out[r * d + c] = acc[c] / l;
+            if (fabs(out[r * d + c]) > omax) omax = fabs(out[r * d + c]);
+        }
+        slack[r] = (rv + rp * omax) / l;
+    }
+    free(q);
+    free(acc);
     return 0;
 }

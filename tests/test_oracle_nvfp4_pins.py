@@ -116,7 +116,7 @@ def _unpack(codes):
 @pytest.mark.parametrize("along_rows", [False, True])
 def test_nvfp4_grid_values_come_back_exactly(oracle, along_rows):
     rng = np.random.default_rng(13 + along_rows)
-    S, R, C = 2, 48, 64
+    S, R, C = (2, 128, 64) if along_rows else (2, 48, 64)   # transposed rows pad to 128
     x, want = _grid_slices(rng, S, R, C, along_rows)
     codes, scales, g = oracle.quant_nvfp4(x, along_rows=along_rows)
     got = _unpack(codes).reshape(want.shape)
@@ -138,7 +138,7 @@ def test_nvfp4_transposed_equals_rows_of_the_transpose(oracle):
     S, R, C = 3, 37, 24                                    # ragged R, C not a multiple of 16
     x = (rng.standard_normal((S, R, C)) * np.exp(rng.standard_normal((S, 1, C)))).astype(np.float16)
     codes, scales, g = oracle.quant_nvfp4(x, along_rows=True)
-    Rp = 48
+    Rp = 128
     xt = np.zeros((S, C, Rp), dtype=np.float16)
     xt[:, :, :R] = x.transpose(0, 2, 1)
     c2, s2, g2 = oracle.quant_nvfp4(xt, along_rows=False)
@@ -242,3 +242,83 @@ def test_qk_nvfp4_exact_on_power_of_two_scales(oracle):
             want = sum(dec(qc, qs, 1, i, c) * dec(kc, ks, 0, kr, c) for c in range(d))
             want *= Fraction(2.0 ** -7) * Fraction(2.0 ** -7)
             assert Fraction(S[i, j]) == want
+
+
+# ---- the FP4-path attention (every key tile in FP4, two-level P quantization) ----
+
+def _onehot_operands(B, H, Hkv, N, d, rng):
+    """NVFP4 operands built from codes: query i and key j each hold one channel (i % d, j % d)
+    with E2M1 value 6 and block scale 448, so S_ij = (6 * 448)^2 when the channels agree and 0
+    otherwise; with slice scales 1 the gap is ~10^6 log2 units and every row's softmax is the
+    plain average of V over its visible keys j == i (mod d).  V: random codes and scales."""
+    def onehot(S):
+        codes = np.zeros((S, N, d // 2), dtype=np.uint8)
+        scales = np.zeros((S, N, d // 16), dtype=np.uint8)
+        for n in range(N):
+            c = n % d
+            codes[:, n, c // 2] = 7 << (4 * (c % 2))
+            scales[:, n, c // 16] = 0x7E
+        return codes, scales, np.ones(S, dtype=np.float32)
+    Np = -(-N // 128) * 128
+    vc = rng.integers(0, 256, size=(B * Hkv, d, Np // 2), dtype=np.uint8)
+    vs = rng.integers(0x30, 0x40, size=(B * Hkv, d, Np // 16), dtype=np.uint8)
+    vc[:, :, N // 2:] = 0                                   # padding tokens hold code 0
+    vg = rng.uniform(0.5, 2.0, size=B * Hkv).astype(np.float32)
+    return onehot(B * H), onehot(B * Hkv), (vc, vs, vg)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_nvfp4_one_hot_scores_average_v(oracle, causal):
+    rng = np.random.default_rng(30 + causal)
+    B, H, Hkv, N, d = 1, 2, 1, 300, 64
+    qn, kn, vn = _onehot_operands(B, H, Hkv, N, d, rng)
+    out, slack = oracle.attention_nvfp4(qn, kn, vn, B, H, Hkv, N, d, causal)
+    vdec = oracle.nvfp4_dequant(*vn)[0]                      # [d, Np]: V^T decoded
+    for bh in range(B * H):
+        for i in range(N):
+            keys = [j for j in range(N) if j % d == i % d and (not causal or j <= i)]
+            want = vdec[:, keys].mean(axis=1)
+            np.testing.assert_allclose(out[bh * N + i], want, rtol=1e-12, atol=1e-12)
+    assert np.all(slack == 0)
+
+
+def test_attention_nvfp4_row0_and_v_scale(oracle):
+    """Causal row 0 sees key 0 alone and returns its decoded V; doubling V's slice scale doubles
+    every output exactly."""
+    rng = np.random.default_rng(33)
+    B, H, Hkv, N, d = 1, 1, 1, 200, 128
+    q = rng.standard_normal((1, N, d)).astype(np.float16)
+    k = rng.standard_normal((1, N, d)).astype(np.float16)
+    v = rng.standard_normal((1, N, d)).astype(np.float16)
+    qn, kn, vn = oracle.quant_nvfp4(q), oracle.quant_nvfp4(k), oracle.quant_nvfp4(v, along_rows=True)
+    out, _ = oracle.attention_nvfp4(qn, kn, vn, B, H, Hkv, N, d, True)
+    np.testing.assert_array_equal(out[0], oracle.nvfp4_dequant(*vn)[0][:, 0])
+    vn2 = (vn[0], vn[1], vn[2] * 2)
+    out2, _ = oracle.attention_nvfp4(qn, kn, vn2, B, H, Hkv, N, d, True)
+    np.testing.assert_array_equal(out2, 2 * out)
+
+
+def test_attention_nvfp4_close_to_full_precision(oracle):
+    """The FP4 path stays close to float64 attention of the decoded operands (the only further
+    error is the FP4 rounding of P), and the two-level quantization keeps P's small entries."""
+    rng = np.random.default_rng(34)
+    B, H, Hkv, N, d = 1, 2, 1, 700, 128
+    q = rng.standard_normal((B * H, N, d)).astype(np.float16)
+    k = rng.standard_normal((B * Hkv, N, d)).astype(np.float16)
+    v = rng.standard_normal((B * Hkv, N, d)).astype(np.float16)
+    qn, kn, vn = oracle.quant_nvfp4(q), oracle.quant_nvfp4(k), oracle.quant_nvfp4(v, along_rows=True)
+    out, slack = oracle.attention_nvfp4(qn, kn, vn, B, H, Hkv, N, d, True)
+    Q = oracle.nvfp4_dequant(*qn)
+    K = oracle.nvfp4_dequant(*kn)
+    V = oracle.nvfp4_dequant(*vn)[:, :, :N].transpose(0, 2, 1)
+    cos = []
+    for h in range(H):
+        s = Q[h] @ K[0].T / np.sqrt(d)
+        s = np.where(np.tril(np.ones((N, N), bool)), s, -np.inf)
+        p = np.exp(s - s.max(1, keepdims=True))
+        ref = (p / p.sum(1, keepdims=True)) @ V[0]
+        o = out[h * N:(h + 1) * N]
+        cos.append(float((o * ref).sum() / np.linalg.norm(o) / np.linalg.norm(ref)))
+        assert np.abs(o - ref).mean() < 0.02
+    assert min(cos) > 0.995, cos
+    assert np.median(slack) == 0
