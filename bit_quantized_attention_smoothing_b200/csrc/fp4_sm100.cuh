@@ -19,6 +19,8 @@
 
 #include <cstdint>
 
+#include "attn_sm100.cuh"  // pack_half2
+#include "nvfp4.cuh"       // E2M1 / E4M3 conversions
 #include "sm100_ptx.cuh"
 
 namespace qattn {
@@ -177,6 +179,305 @@ __global__ void __launch_bounds__(128, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace qattn
+
+namespace qattn {
+
+// ------------------------------------------------------------------------------------------------
+// Attention on the FP4 path (ThriftAttention page, method section): every key tile in FP4, the
+// blocks merged by the online softmax ("online merge"), the probability blocks quantized in two
+// levels for the FP4 P V product (a per-row binary32 scale gP = max p / 2688, then NVFP4 blocks of
+// 16 keys with UE4M3 scales).  Operands: Q and smoothed K NVFP4 along the channels, V NVFP4 along
+// the tokens (transposed, rows of Np = ceil(N / 128) * 128 tokens).
+//
+// One CTA of 4 warps per 128-row query tile; thread t owns query row 128 qt + t, which is TMEM lane
+// t.  Per key tile: the warps put K's and V's block scales into tensor memory, one thread loads the
+// E2M1 K and V tiles by TMA and issues the FP4 Q K^T; every thread reads its row of S, takes the
+// online maximum, quantizes its P row (E2M1 codes into the swizzled shared-memory operand, UE4M3
+// scales through shared memory into tensor memory), and one thread issues the FP4 P V into a
+// tensor-memory tile that the threads fold into their fp32 output rows.  The steps run one after
+// another (no pipelining across tiles).  Every wait is bounded and each outcome is agreed by the
+// whole CTA (__syncthreads_and), so a wait that runs out ends every thread's loop together.
+// ------------------------------------------------------------------------------------------------
+
+template <int D>
+struct Fp4AttnCfg {
+  static constexpr int kQK = 128 * (D / 2);  // E2M1 Q or K tile: 128 rows of D/2 bytes
+  static constexpr int kVt = D * 64;         // E2M1 V^T tile: D channel rows of 128 keys
+  static constexpr int kP = 128 * 64;        // E2M1 P tile: 128 rows of 128 keys
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kQK;
+  static constexpr int kOffV = 2 * kQK;
+  static constexpr int kOffP = 2 * kQK + kVt;
+  static constexpr int kOffSfp = kOffP + kP;      // uint32 [2][128]: P scale words by K step
+  static constexpr int kOffBar = kOffSfp + 1024;
+  static constexpr int kSmemUsed = kOffBar + 64 + 1024;
+  static constexpr uint32_t kSwQK = D == 128 ? kSwizzle64B : kSwizzle32B;
+  static constexpr uint32_t kSboQK = 8 * (D / 2);
+  static constexpr int kStepsQK = D / 64;         // K = 64 per instruction
+  static constexpr int kSfvCols = D / 32;         // V scale columns per K step (N = D)
+  // tensor-memory columns: S, the P V tile, then the four scale-factor areas
+  static constexpr uint32_t kColS = 0, kColO = 128, kColSfq = 256, kColSfk = 264, kColSfp = 272,
+                            kColSfv = 280;
+};
+
+// Sum of twice the E2M1 magnitudes of the eight codes in w (values 0, .5, 1, 1.5, 2, 3, 4, 6 are
+// 0, 1, 2, 3, 4, 6, 8, 12 when doubled: one nibble each in the table 0xC8643210).
+__device__ __forceinline__ uint32_t e2m1x8_twice_sum(uint32_t w) {
+  uint32_t s = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) s += (0xC8643210u >> (4 * ((w >> (4 * i)) & 7u))) & 15u;
+  return s;
+}
+
+__device__ __forceinline__ void tmem_st32x2(uint32_t taddr, uint32_t a, uint32_t b) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(a),
+               "r"(b)
+               : "memory");
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(128, 1)
+    attn_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_vt, const uint8_t* __restrict__ q_sf,
+                      const uint8_t* __restrict__ k_sf, const uint8_t* __restrict__ vt_sf,
+                      const float* __restrict__ q_g, const float* __restrict__ k_g,
+                      const float* __restrict__ v_g, __half* __restrict__ out, int H, int Hkv,
+                      int N, int Np, float sl2) {
+  using Cfg = Fp4AttnCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sq = smem + Cfg::kOffQ;
+  uint8_t* sk = smem + Cfg::kOffK;
+  uint8_t* sv = smem + Cfg::kOffV;
+  uint8_t* sp = smem + Cfg::kOffP;
+  uint32_t* sfp = reinterpret_cast<uint32_t*>(smem + Cfg::kOffSfp);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* s_done = bars + 2;
+  uint64_t* o_done = bars + 3;
+  uint32_t* tbase = reinterpret_cast<uint32_t*>(bars + 4);
+  volatile int* abort = reinterpret_cast<volatile int*>(bars + 5);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int qt = CAUSAL ? static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x)
+                        : static_cast<int>(blockIdx.x);
+  const int bh = blockIdx.y;
+  const int b = bh / H, h = bh % H;
+  const int bg = b * Hkv + h / (H / Hkv);
+  const int row = qt * 128 + tid;
+  const int nkt = CAUSAL ? qt + 1 : (N + 127) / 128;
+
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tbase, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tbase;
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  const uint8_t* ksf = k_sf + static_cast<size_t>(bg) * N * (D / 16);
+  const uint8_t* vsf = vt_sf + static_cast<size_t>(bg) * D * (Np / 16);
+  {
+    const uint8_t* qsf = q_sf + static_cast<size_t>(bh) * N * (D / 16);
+#pragma unroll
+    for (int kc = 0; kc < Cfg::kStepsQK; ++kc) {
+      uint32_t w[4];
+      load_sf_words(qsf, D, N, qt * 128, kc, w);
+      tmem_st32x4(lane_base + Cfg::kColSfq + 4 * kc, w[0], w[1], w[2], w[3]);
+    }
+  }
+  if (tid == 0) {
+    mbar_arrive_expect_tx(q_full, Cfg::kQK);
+    tma_load_3d(sq, &tm_q, q_full, 0, qt * 128, bh);
+  }
+  const float gqk = __ldg(q_g + bh) * __ldg(k_g + bg) * sl2;  // S to log2 units
+  const float gv = __ldg(v_g + bg);
+  float m = -INFINITY, l = 0.0f;
+  float o[D];
+#pragma unroll
+  for (int c = 0; c < D; ++c) o[c] = 0.0f;
+  bool ok = true;
+
+  for (int kt = 0; kt < nkt; ++kt) {
+    const uint32_t ph = static_cast<uint32_t>(kt & 1);
+    // (a) K's and V's block scales into this warp's sub-partition
+#pragma unroll
+    for (int kc = 0; kc < Cfg::kStepsQK; ++kc) {
+      uint32_t w[4];
+      load_sf_words(ksf, D, N, kt * 128, kc, w);
+      tmem_st32x4(lane_base + Cfg::kColSfk + 4 * kc, w[0], w[1], w[2], w[3]);
+    }
+#pragma unroll
+    for (int kc = 0; kc < 2; ++kc) {
+      uint32_t w[4];
+#pragma unroll
+      for (int r1 = 0; r1 < Cfg::kSfvCols; ++r1)
+        w[r1] = __ldg(reinterpret_cast<const uint32_t*>(
+            vsf + static_cast<size_t>(lane + 32 * r1) * (Np / 16) + kt * 8 + 4 * kc));
+      if constexpr (D == 128)
+        tmem_st32x4(lane_base + Cfg::kColSfv + 4 * kc, w[0], w[1], w[2], w[3]);
+      else
+        tmem_st32x2(lane_base + Cfg::kColSfv + 2 * kc, w[0], w[1]);
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+    // (b) K and V^T tiles, then S = Q K^T (FP4, block-scaled)
+    if (tid == 0) {
+      tc_fence_after();
+      mbar_arrive_expect_tx(kv_full, Cfg::kQK + Cfg::kVt);
+      tma_load_3d(sk, &tm_k, kv_full, 0, kt * 128, bg);
+      tma_load_3d(sv, &tm_vt, kv_full, kt * 64, 0, bg);
+      const bool loaded = (kt > 0 || mbar_wait(q_full, 0, abort)) && mbar_wait(kv_full, ph, abort);
+      if (loaded) {
+        tc_fence_after();
+        constexpr uint32_t id = idesc_nvf4(128, 128);
+#pragma unroll
+        for (int kc = 0; kc < Cfg::kStepsQK; ++kc) {
+          const uint64_t ad = smem_desc(smem_u32(sq) + kc * 32, 16, Cfg::kSboQK, Cfg::kSwQK);
+          const uint64_t bd = smem_desc(smem_u32(sk) + kc * 32, 16, Cfg::kSboQK, Cfg::kSwQK);
+          mma_nvf4_ss(tmem + Cfg::kColS, ad, bd, id, tmem + Cfg::kColSfq + 4 * kc,
+                      tmem + Cfg::kColSfk + 4 * kc, kc > 0 ? 1u : 0u);
+        }
+        mma_commit(s_done);
+      }
+    }
+    ok = __syncthreads_and(mbar_wait(s_done, ph, abort));
+    if (!ok) break;
+    tc_fence_after();
+    // (c) this row's online softmax step and its two-level FP4 quantization
+    const int kbase = kt * 128;
+    float tmax = -INFINITY;
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t v[32];
+      tmem_ld32(lane_base + Cfg::kColS + 32 * cc, v);
+      tmem_ld_wait(v);
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        const int key = kbase + 32 * cc + t;
+        const bool valid = key < N && (!CAUSAL || key <= row);
+        if (valid) tmax = fmaxf(tmax, __uint_as_float(v[t]) * gqk);
+      }
+    }
+    const float m_new = fmaxf(m, tmax);
+    const float corr = exp2f(m - m_new);
+    const float gp = __fdiv_rn(exp2f(tmax - m_new), kNvfp4Div);
+    const float sixg = __fmul_rn(6.0f, gp);
+    float lsum = 0.0f;
+    uint32_t sfw0 = 0, sfw1 = 0;
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t v[32];
+      tmem_ld32(lane_base + Cfg::kColS + 32 * cc, v);
+      tmem_ld_wait(v);
+      float p[32];
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        const int key = kbase + 32 * cc + t;
+        const bool valid = key < N && (!CAUSAL || key <= row);
+        p[t] = valid ? exp2f(__uint_as_float(v[t]) * gqk - m_new) : 0.0f;
+      }
+      uint32_t cw[4];
+#pragma unroll
+      for (int hb = 0; hb < 2; ++hb) {
+        float* pb = p + 16 * hb;
+        float bmax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, pb[i]);
+        const uint32_t s = gp > 0.0f ? ue4m3_byte(__fdiv_rn(bmax, sixg)) : 0u;
+        cw[2 * hb] = 0u;
+        cw[2 * hb + 1] = 0u;
+        if (s != 0u) {
+          const float sc = __fmul_rn(ue4m3_value(s), gp);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pb[i] = __fdiv_rn(pb[i], sc);
+          cw[2 * hb] = e2m1x8(pb);
+          cw[2 * hb + 1] = e2m1x8(pb + 8);
+          lsum += 0.5f * sc *
+                  static_cast<float>(e2m1x8_twice_sum(cw[2 * hb]) + e2m1x8_twice_sum(cw[2 * hb + 1]));
+        }
+        const int blk = 2 * cc + hb;  // 16-key block 0..7 of the tile
+        if (blk < 4) sfw0 |= s << (8 * blk);
+        else sfw1 |= s << (8 * (blk - 4));
+      }
+      // 16 bytes (keys 32 cc .. 32 cc + 31) into the 64-byte-swizzled row of the P operand
+      st_shared_v4(smem_u32(sp) + tid * 64 + ((cc ^ ((tid >> 1) & 3)) << 4), cw[0], cw[1], cw[2],
+                   cw[3]);
+    }
+    l = l * corr + lsum;
+    sfp[tid] = sfw0;
+    sfp[128 + tid] = sfw1;
+    fence_proxy_async_smem();
+    __syncthreads();
+    // (d) P's scales: row r0 + 32 r1 in column r1 of lane r0, in every sub-partition
+#pragma unroll
+    for (int kc = 0; kc < 2; ++kc)
+      tmem_st32x4(lane_base + Cfg::kColSfp + 4 * kc, sfp[128 * kc + lane], sfp[128 * kc + lane + 32],
+                  sfp[128 * kc + lane + 64], sfp[128 * kc + lane + 96]);
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t id = idesc_nvf4(128, D);
+#pragma unroll
+      for (int kc = 0; kc < 2; ++kc) {
+        const uint64_t ad = smem_desc(smem_u32(sp) + kc * 32, 16, 512, kSwizzle64B);
+        const uint64_t bd = smem_desc(smem_u32(sv) + kc * 32, 16, 512, kSwizzle64B);
+        mma_nvf4_ss(tmem + Cfg::kColO, ad, bd, id, tmem + Cfg::kColSfp + 4 * kc,
+                    tmem + Cfg::kColSfv + Cfg::kSfvCols * kc, kc > 0 ? 1u : 0u);
+      }
+      mma_commit(o_done);
+    }
+    ok = __syncthreads_and(mbar_wait(o_done, ph, abort));
+    if (!ok) break;
+    tc_fence_after();
+    // (e) fold the tile's P V into the output row: O = O * corr + (P^ V^) * gP * gV
+    const float f = gp * gv;
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t v[32];
+      tmem_ld32(lane_base + Cfg::kColO + 32 * cc, v);
+      tmem_ld_wait(v);
+#pragma unroll
+      for (int t = 0; t < 32; ++t) o[32 * cc + t] = o[32 * cc + t] * corr + __uint_as_float(v[t]) * f;
+    }
+    m = m_new;
+  }
+  if (ok && row < N) {
+    const float inv = 1.0f / l;
+    uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + row) * D);
+#pragma unroll
+    for (int c = 0; c < D; c += 8) {
+      uint4 w;
+      w.x = pack_half2(o[c] * inv, o[c + 1] * inv);
+      w.y = pack_half2(o[c + 2] * inv, o[c + 3] * inv);
+      w.z = pack_half2(o[c + 4] * inv, o[c + 5] * inv);
+      w.w = pack_half2(o[c + 6] * inv, o[c + 7] * inv);
+      dst[c / 8] = w;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 

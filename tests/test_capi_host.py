@@ -141,3 +141,14 @@ def test_debug_qk_nvfp4_argument_checks():
     assert L.qattn_debug_qk_nvfp4(*a, 1, 4, 2, 256, 128, 0, 4, 0, 1, 0, 1, None) == 1    # head
     assert L.qattn_debug_qk_nvfp4(*a, 1, 4, 2, 256, 96, 0, 0, 0, 1, 0, 1, None) == 2     # d
     assert L.qattn_debug_qk_nvfp4(P(17), *a[1:], 1, 4, 2, 256, 128, 0, 0, 0, 1, 0, 1, None) == 3
+
+
+def test_attn_nvfp4_argument_checks():
+    L = Q.load()
+    a = tuple(P(16 * (i + 1)) for i in range(10))
+    assert L.qattn_attn_nvfp4(None, *a[1:], 1, 4, 2, 256, 128, 1, None) == 1
+    assert L.qattn_attn_nvfp4(*a, 1, 4, 3, 256, 128, 1, None) == 1         # H % Hkv
+    assert L.qattn_attn_nvfp4(*a, 1, 4, 2, 0, 128, 1, None) == 1           # N
+    assert L.qattn_attn_nvfp4(*a, 1, 4, 2, 256, 96, 1, None) == 2          # d
+    assert L.qattn_attn_nvfp4(*a, 300, 256, 2, 256, 128, 1, None) == 2    # B * H > 65535
+    assert L.qattn_attn_nvfp4(*a[:9], P(24), 1, 4, 2, 256, 128, 1, None) == 3

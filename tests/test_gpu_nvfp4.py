@@ -224,3 +224,118 @@ def test_qk_nvfp4_full_size_tiles(lib, oracle):
         S, M = oracle.qk_nvfp4(qn[0], qn[1], qn[2], kn[0], kn[1], kn[2], 1, 1, 0, 0,
                                qt * 128, 128, kt * 128, 128)
         _check_scores(got.cpu().numpy(), S, M, f"full qt{qt} kt{kt}")
+
+
+# ---- FP4-path attention (every key tile in FP4, two-level P, online merge) ----
+#
+# Against the oracle's FP4-path attention on the same NVFP4 operands.  The GPU's scores carry f32
+# accumulation and its exponentials binary32 rounding; elsewhere the arithmetic is the oracle's
+# (binary32 quantization steps), so outside FP4 decisions taken within 2^-16 of a tie the output
+# agrees to the fp16 output rounding: max-abs 2e-3 (plus half the fp16 spacing where |O| >= 4) and
+# mean-abs 2e-4, as the INT8 path.  A row holding such near-tie decisions may differ by the
+# oracle's per-row slack on top.
+
+def _nvfp4_operands(oracle, w, q, k, v):
+    sums = oracle.k_channel_sums(np16(k), w.B, w.Hkv, w.N, w.d)
+    mean = np.array([oracle.lib().oracle_mean_from_sum(int(s), w.N) for s in sums.ravel()],
+                    dtype=np.float32).reshape(w.B * w.Hkv, w.d)
+    qn = oracle.quant_nvfp4(np16(q).reshape(w.B * w.H, w.N, w.d))
+    kn = oracle.quant_nvfp4(np16(k).reshape(w.B * w.Hkv, w.N, w.d), mean=mean)
+    vn = oracle.quant_nvfp4(np16(v).reshape(w.B * w.Hkv, w.N, w.d), along_rows=True)
+    return qn, kn, vn
+
+
+def _check_fp4_out(got_rows, ref, slack, what):
+    g = got_rows.astype(np.float64)
+    err = np.abs(g - ref)
+    half_ulp = np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64) / 2
+    allow = 2e-3 + np.where(np.abs(ref) >= 4, half_ulp, 0) + slack[:, None]
+    n_slack = int((slack > 0).sum())
+    print(what, f"max-abs {err.max():.3e} mean-abs {err.mean():.3e} rows with slack {n_slack}"
+          f" worst excess {(err - allow).max():.3e}")
+    assert np.all(err <= allow), what
+    assert err.mean() <= 2e-4, what
+
+
+FP4_CASES = [
+    ("tiny", {"N": 300}),
+    ("tiny", {"N": 129, "causal": True}),
+    ("llama8b_32k", {"H": 4, "Hkv": 2, "N": 700}),
+    ("llama8b_32k", {"B": 2, "H": 2, "Hkv": 1, "N": 200, "causal": False}),
+    ("wide64", {"B": 1, "H": 3, "Hkv": 1, "N": 513, "causal": True}),
+    ("long128k", {"H": 2, "Hkv": 1, "N": 1, "causal": True}),
+]
+
+
+@pytest.mark.parametrize("name,over", FP4_CASES,
+                         ids=[f"{n}-" + "-".join(f"{k}{v}" for k, v in o.items()) for n, o in FP4_CASES])
+def test_attn_nvfp4_against_oracle(lib, oracle, name, over):
+    w = WORKLOADS[name].with_(**over)
+    q, k, v = make_inputs(w, device="cpu")
+    qn, kn, vn = _nvfp4_operands(oracle, w, q, k, v)
+    out = lib.qattn_attn_nvfp4(_upload(qn), _upload(kn), _upload(vn), w.B, w.H, w.Hkv, w.N, w.d,
+                               causal=w.causal)
+    assert lib.qattn_check_device_status() == 0
+    ref, slack = oracle.attention_nvfp4(qn, kn, vn, w.B, w.H, w.Hkv, w.N, w.d, w.causal)
+    _check_fp4_out(out.float().cpu().numpy().reshape(-1, w.d), ref, slack, name)
+
+
+@pytest.mark.parametrize("d,causal", [(64, False), (128, True)])
+def test_attn_nvfp4_one_hot_scores(lib, oracle, d, causal):
+    """Scores built from codes so that each row's softmax is the plain mean of V over its
+    visible keys j == i (mod d) (closed form, several key tiles)."""
+    rng = np.random.default_rng(50 + d)
+    B, H, Hkv, N = 1, 2, 1, 400
+
+    def onehot(S):
+        codes = np.zeros((S, N, d // 2), dtype=np.uint8)
+        scales = np.zeros((S, N, d // 16), dtype=np.uint8)
+        for n in range(N):
+            c = n % d
+            codes[:, n, c // 2] = 7 << (4 * (c % 2))
+            scales[:, n, c // 16] = 0x7E
+        return codes, scales, np.ones(S, dtype=np.float32)
+
+    Np = 512
+    vc = rng.integers(0, 256, size=(B * Hkv, d, Np // 2), dtype=np.uint8)
+    vs = rng.integers(0x30, 0x40, size=(B * Hkv, d, Np // 16), dtype=np.uint8)
+    vn = (vc, vs, np.array([0.75], dtype=np.float32))
+    qn, kn = onehot(B * H), onehot(B * Hkv)
+    out = lib.qattn_attn_nvfp4(_upload(qn), _upload(kn), _upload(vn), B, H, Hkv, N, d,
+                               causal=causal).float().cpu().numpy()
+    vdec = oracle.nvfp4_dequant(*vn)[0]
+    for h in range(H):
+        for i in range(N):
+            keys = [j for j in range(N) if j % d == i % d and (not causal or j <= i)]
+            want = vdec[:, keys].mean(axis=1)
+            assert np.abs(out[0, h, i] - want).max() <= 1e-3 + np.abs(want).max() * 2 ** -11
+
+
+def test_attn_nvfp4_full_size_sampled_rows(lib, oracle):
+    """32K-token workload, operands quantized on the GPU (slices used here checked equal to the
+    oracle's), FP4-path attention of all 32 heads; sampled rows of one head against the oracle."""
+    w = WORKLOADS["llama8b_32k"]
+    q, k, v = make_inputs(w, device="cuda")
+    h = 5
+    g = h // (w.H // w.Hkv)
+    sums = oracle.k_channel_sums(np16(k[:, g:g + 1]), 1, 1, w.N, w.d)
+    mean1 = np.array([oracle.lib().oracle_mean_from_sum(int(s), w.N) for s in sums.ravel()],
+                     dtype=np.float32)
+    mean = torch.zeros(w.Hkv, w.d, dtype=torch.float32, device="cuda")
+    mean[g] = torch.from_numpy(mean1).cuda()
+    gq = lib.qattn_quant_nvfp4(q.reshape(w.H, w.N, w.d))
+    gk = lib.qattn_quant_nvfp4(k.reshape(w.Hkv, w.N, w.d), mean)
+    gv = lib.qattn_quant_nvfp4(v.reshape(w.Hkv, w.N, w.d), along_rows=True)
+    out = lib.qattn_attn_nvfp4(gq, gk, gv, w.B, w.H, w.Hkv, w.N, w.d, causal=True)
+    assert lib.qattn_check_device_status() == 0
+    qn = oracle.quant_nvfp4(np16(q[0, h:h + 1]).view(np.float16))
+    kn = oracle.quant_nvfp4(np16(k[0, g:g + 1]).view(np.float16), mean=mean1[None])
+    vn = oracle.quant_nvfp4(np16(v[0, g:g + 1]).view(np.float16), along_rows=True)
+    for mine, ref, s in ((gq, qn, h), (gk, kn, g), (gv, vn, g)):
+        for a, r in zip(mine, ref):
+            assert np.array_equal(a[s:s + 1].cpu().numpy(), r)
+    rows_i = np.array([0, 1, 127, 128, 4095, 20000, w.N - 129, w.N - 1], dtype=np.int64)
+    ref, slack = oracle.attention_nvfp4(qn, kn, vn, 1, 1, 1, w.N, w.d, True,
+                                        rows=(np.zeros_like(rows_i), rows_i))
+    got = out[0, h, torch.from_numpy(rows_i).cuda()].float().cpu().numpy()
+    _check_fp4_out(got, ref, slack, "llama8b_32k full")
