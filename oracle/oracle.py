@@ -84,8 +84,8 @@ def lib():
         L.oracle_ue4m3_encode.restype = ctypes.c_uint8
         L.oracle_quant_nvfp4.argtypes = [P, P, i, i, i, i, P, P, P]
         L.oracle_quant_nvfp4.restype = i
-        L.oracle_attention_nvfp4.argtypes = [P, P, P, P, P, P, P, P, P, i, i, i, i, i, i, i, P, P,
-                                             ctypes.c_long, P, P]
+        L.oracle_attention_nvfp4.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                             i, i, i, i, i, i, i, P, P, ctypes.c_long, P, P]
         L.oracle_attention_nvfp4.restype = i
         _lib = L
     return _lib
@@ -356,11 +356,14 @@ def qk_nvfp4(q_codes, q_scales, q_g, k_codes, k_scales, k_g, H, Hkv, b, h, r0, n
     return Q @ K.T, np.abs(Q) @ np.abs(K).T
 
 
-def attention_nvfp4(qn, kn, vn, B, H, Hkv, N, d, causal, rows=None):
-    """Rows of the FP4-path attention (every key tile in FP4; the C file states the readings).
+def attention_nvfp4(qn, kn, vn, B, H, Hkv, N, d, causal, rows=None, promote=None, q16=None,
+                    k16=None, v16=None, k_mean=None):
+    """Rows of the FP4-path attention (the C file states the readings).
 
     qn, kn: (codes, scales, gscale) along the channels over B*H and B*Hkv slices; vn: the same for
-    V along the tokens (transposed).  Returns (out float64 [nrows, d], slack float64 [nrows])."""
+    V along the tokens (transposed).  promote: uint8 [B*H, ceil(N/256), ceil(N/128)] marking the
+    key tiles computed in FP16 from q16, k16, v16 (fp16) with the smoothed keys (k_mean float32
+    [B*Hkv, d]); None = every tile in FP4.  Returns (out float64 [nrows, d], slack [nrows])."""
     row_bh, row_i = all_rows(B, H, N) if rows is None else rows
     row_bh = np.ascontiguousarray(row_bh, dtype=np.int64)
     row_i = np.ascontiguousarray(row_i, dtype=np.int64)
@@ -372,6 +375,11 @@ def attention_nvfp4(qn, kn, vn, B, H, Hkv, N, d, causal, rows=None):
         c(qn[0], np.uint8), c(qn[1], np.uint8), c(qn[2], np.float32),
         c(kn[0], np.uint8), c(kn[1], np.uint8), c(kn[2], np.float32),
         c(vn[0], np.uint8), c(vn[1], np.uint8), c(vn[2], np.float32),
+        None if promote is None else _ptr(_bits16(q16)),
+        None if promote is None else _ptr(_bits16(k16)),
+        None if promote is None else _ptr(_bits16(v16)),
+        None if promote is None else c(k_mean, np.float32),
+        None if promote is None else c(promote, np.uint8),
         B, H, Hkv, N, Np, d, 1 if causal else 0, _ptr(row_bh), _ptr(row_i), row_bh.size,
         _ptr(out), _ptr(slack))
     if rc != 0:

@@ -635,17 +635,27 @@ static int ue4m3_near_tie(float t) {
 
 /* q_codes [B*H][N][d/2], q_scales [B*H][N][d/16], q_g [B*H]; k_* likewise over B*Hkv;
  * vt_codes [B*Hkv][d][Np/2], vt_scales [B*Hkv][d][Np/16], v_g [B*Hkv].
+ * Promotion (the FP16 path of the same page's method section: the top-k query-key block pairs are
+ * computed in FP16; NULL promote = none): promote [B*H][ceil(N/256)][ceil(N/128)] marks the key
+ * tiles of each 256-row query block that run in FP16, from fp16 q [B*H][N][d], k and v
+ * [B*Hkv][N][d]; their scores use the smoothed keys, x_j = sum_c q_c (k_jc - k_mean_c) log2(e) /
+ * sqrt(d) (k_mean [B*Hkv][d], the mean the FP4 K was smoothed with), p_j is rounded to binary32
+ * and then to fp16, and l and P V take those fp16 values and fp16 V.
  * Rows (row_bh[r], row_i[r]) for r < nrows; out [nrows][d], slack [nrows].  Returns 0, or -1 on a
  * bad argument. */
 int oracle_attention_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales, const float* q_g,
                            const uint8_t* k_codes, const uint8_t* k_scales, const float* k_g,
                            const uint8_t* vt_codes, const uint8_t* vt_scales, const float* v_g,
+                           const uint16_t* q16, const uint16_t* k16, const uint16_t* v16,
+                           const float* k_mean, const uint8_t* promote,
                            int B, int H, int Hkv, int N, int Np, int d, int causal,
                            const long* row_bh, const long* row_i, long nrows, double* out,
                            double* slack) {
     if (B < 1 || H < 1 || Hkv < 1 || N < 1 || H % Hkv || d % 16 || Np < N || Np % 16) return -1;
+    if (promote && (!q16 || !k16 || !v16 || !k_mean)) return -1;
     const double sl2 = 1.4426950408889634 / sqrt((double)d);
     const double rel = ldexp(1.0, -16);
+    const long nsb = (N + 255) / 256, nkt = (N + 127) / 128;
     double* q = (double*)malloc(sizeof(double) * d);
     double* acc = (double*)malloc(sizeof(double) * d);
     double x[128], ph[128], risk[128];
@@ -661,6 +671,34 @@ int oracle_attention_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales, cons
         for (int c = 0; c < d; ++c) acc[c] = 0.0;
         for (long t0 = 0; t0 <= last; t0 += 128) {
             const int n = (int)((last - t0 + 1) < 128 ? (last - t0 + 1) : 128);   /* visible keys */
+            if (promote && promote[(bh * nsb + i / 256) * nkt + t0 / 128]) {
+                /* FP16 path: smoothed scores from the fp16 operands, fp16 P, fp16 V */
+                double tmx = -INFINITY;
+                for (int j = 0; j < n; ++j) {
+                    double sdot = 0.0;
+                    for (int c = 0; c < d; ++c)
+                        sdot += oracle_f16_to_f64(q16[(bh * N + i) * (long)d + c]) *
+                                (oracle_f16_to_f64(k16[(bg * N + t0 + j) * (long)d + c]) -
+                                 (double)k_mean[bg * d + c]);
+                    x[j] = sdot * sl2;
+                    if (x[j] > tmx) tmx = x[j];
+                }
+                const double mn = m > tmx ? m : tmx;
+                const double corr = exp2(m - mn);
+                l *= corr;
+                rv *= corr;
+                rp *= corr;
+                for (int c = 0; c < d; ++c) acc[c] *= corr;
+                for (int j = 0; j < n; ++j) {
+                    const float pf = (float)exp2(x[j] - mn);
+                    const double p16 = oracle_f16_to_f64(oracle_f64_to_f16((double)pf));
+                    l += p16;
+                    for (int c = 0; c < d; ++c)
+                        acc[c] += p16 * oracle_f16_to_f64(v16[(bg * N + t0 + j) * (long)d + c]);
+                }
+                m = mn;
+                continue;
+            }
             double tmax = -INFINITY;
             for (int j = 0; j < n; ++j) {
                 double sdot = 0.0;
