@@ -19,8 +19,9 @@
 
 #include <cstdint>
 
-#include "attn_sm100.cuh"  // pack_half2
+#include "attn_sm100.cuh"  // pack_half2, add_half2_f32
 #include "nvfp4.cuh"       // E2M1 / E4M3 conversions
+#include "quant.cuh"       // half_bits_to_float
 #include "sm100_ptx.cuh"
 
 namespace qattn {
@@ -187,20 +188,24 @@ __global__ void __launch_bounds__(128, 1)
 namespace qattn {
 
 // ------------------------------------------------------------------------------------------------
-// Attention on the FP4 path (ThriftAttention page, method section): every key tile in FP4, the
-// blocks merged by the online softmax ("online merge"), the probability blocks quantized in two
-// levels for the FP4 P V product (a per-row binary32 scale gP = max p / 2688, then NVFP4 blocks of
-// 16 keys with UE4M3 scales).  Operands: Q and smoothed K NVFP4 along the channels, V NVFP4 along
-// the tokens (transposed, rows of Np = ceil(N / 128) * 128 tokens).
+// Attention on the FP4 path with FP16 promotion (ThriftAttention page, method section: the top-k
+// query-key block pairs computed in FP16, the rest in FP4, both merged by one online softmax; the
+// FP4 probability blocks quantized in two levels).  FP4 tiles: Q and smoothed K NVFP4 along the
+// channels, V NVFP4 along the tokens (transposed, rows of Np = ceil(N / 128) * 128 tokens), P
+// quantized per row in two levels (binary32 row scale gP = max p / 2688, then NVFP4 blocks of 16
+// keys with UE4M3 scales).  Promoted tiles (the key tiles listed for the CTA's 256-row query
+// block): fp16 Q K^T on the f16 tensor cores with q . mean subtracted (the FP16 scores see the
+// same smoothed keys as the FP4 ones), P rounded to fp16 into tensor memory, fp16 V.
 //
 // One CTA of 4 warps per 128-row query tile; thread t owns query row 128 qt + t, which is TMEM lane
-// t.  Per key tile: the warps put K's and V's block scales into tensor memory, one thread loads the
-// E2M1 K and V tiles by TMA and issues the FP4 Q K^T; every thread reads its row of S, takes the
-// online maximum, quantizes its P row (E2M1 codes into the swizzled shared-memory operand, UE4M3
-// scales through shared memory into tensor memory), and one thread issues the FP4 P V into a
-// tensor-memory tile that the threads fold into their fp32 output rows.  The steps run one after
-// another (no pipelining across tiles).  Every wait is bounded and each outcome is agreed by the
-// whole CTA (__syncthreads_and), so a wait that runs out ends every thread's loop together.
+// t.  Per key tile: (a) FP4 tiles: the warps put K's and V's block scales into tensor memory;
+// (b) one thread loads the tile's operands by TMA and issues Q K^T; (c) every thread reads its row
+// of S, takes the online maximum and writes its P row (FP4: codes into the swizzled shared-memory
+// operand, scales through shared memory into every sub-partition; FP16: pairs into tensor memory);
+// (d) one thread issues P V into a tensor-memory tile; (e) the threads fold it into their fp32
+// output rows.  The FP16 query tile is loaded only by CTAs with promoted tiles.  The steps run one
+// after another (no pipelining across tiles).  Every wait is bounded and each outcome is agreed by
+// the whole CTA (__syncthreads_and), so a wait that runs out ends every thread's loop together.
 // ------------------------------------------------------------------------------------------------
 
 template <int D>
@@ -208,20 +213,25 @@ struct Fp4AttnCfg {
   static constexpr int kQK = 128 * (D / 2);  // E2M1 Q or K tile: 128 rows of D/2 bytes
   static constexpr int kVt = D * 64;         // E2M1 V^T tile: D channel rows of 128 keys
   static constexpr int kP = 128 * 64;        // E2M1 P tile: 128 rows of 128 keys
+  static constexpr int kT16 = 128 * D * 2;   // fp16 tile of 128 rows (D/64 boxes of 64 columns)
+  static constexpr int kBox16 = 128 * 128;   // one 64-column fp16 box: 128 rows of 128 bytes
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kQK;
   static constexpr int kOffV = 2 * kQK;
   static constexpr int kOffP = 2 * kQK + kVt;
   static constexpr int kOffSfp = kOffP + kP;      // uint32 [2][128]: P scale words by K step
-  static constexpr int kOffBar = kOffSfp + 1024;
+  static constexpr int kOffQ16 = kOffSfp + 1024;
+  static constexpr int kOffK16 = kOffQ16 + kT16;
+  static constexpr int kOffV16 = kOffK16 + kT16;
+  static constexpr int kOffBar = kOffV16 + kT16;
   static constexpr int kSmemUsed = kOffBar + 64 + 1024;
   static constexpr uint32_t kSwQK = D == 128 ? kSwizzle64B : kSwizzle32B;
   static constexpr uint32_t kSboQK = 8 * (D / 2);
-  static constexpr int kStepsQK = D / 64;         // K = 64 per instruction
+  static constexpr int kStepsQK = D / 64;         // K = 64 per FP4 instruction
   static constexpr int kSfvCols = D / 32;         // V scale columns per K step (N = D)
-  // tensor-memory columns: S, the P V tile, then the four scale-factor areas
+  // tensor-memory columns: S, the P V tile, the four scale-factor areas, fp16 P (64 columns)
   static constexpr uint32_t kColS = 0, kColO = 128, kColSfq = 256, kColSfk = 264, kColSfp = 272,
-                            kColSfv = 280;
+                            kColSfv = 280, kColP16 = 288;
 };
 
 // Sum of twice the E2M1 magnitudes of the eight codes in w (values 0, .5, 1, 1.5, 2, 3, 4, 6 are
@@ -239,14 +249,53 @@ __device__ __forceinline__ void tmem_st32x2(uint32_t taddr, uint32_t a, uint32_t
                : "memory");
 }
 
+__device__ __forceinline__ void tmem_st32x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// Instruction descriptor of kind::f16 with fp16 A and B, both K-major, f32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_f16_f32_kk(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Single-thread forms of the f16 MMAs (A from shared memory, or from tensor memory).
+__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem), "l"(adesc),
+      "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(128, 1)
     attn_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_vt, const uint8_t* __restrict__ q_sf,
+                      const __grid_constant__ CUtensorMap tm_vt,
+                      const __grid_constant__ CUtensorMap tm_q16,
+                      const __grid_constant__ CUtensorMap tm_k16,
+                      const __grid_constant__ CUtensorMap tm_v16, const uint8_t* __restrict__ q_sf,
                       const uint8_t* __restrict__ k_sf, const uint8_t* __restrict__ vt_sf,
                       const float* __restrict__ q_g, const float* __restrict__ k_g,
-                      const float* __restrict__ v_g, __half* __restrict__ out, int H, int Hkv,
+                      const float* __restrict__ v_g, const uint16_t* __restrict__ q16,
+                      const float* __restrict__ k_mean, const int* __restrict__ kv_list,
+                      const int* __restrict__ kv_count, __half* __restrict__ out, int H, int Hkv,
                       int N, int Np, float sl2) {
   using Cfg = Fp4AttnCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -256,14 +305,18 @@ __global__ void __launch_bounds__(128, 1)
   uint8_t* sk = smem + Cfg::kOffK;
   uint8_t* sv = smem + Cfg::kOffV;
   uint8_t* sp = smem + Cfg::kOffP;
+  uint8_t* sq16 = smem + Cfg::kOffQ16;
+  uint8_t* sk16 = smem + Cfg::kOffK16;
+  uint8_t* sv16 = smem + Cfg::kOffV16;
   uint32_t* sfp = reinterpret_cast<uint32_t*>(smem + Cfg::kOffSfp);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kOffBar);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* s_done = bars + 2;
   uint64_t* o_done = bars + 3;
-  uint32_t* tbase = reinterpret_cast<uint32_t*>(bars + 4);
-  volatile int* abort = reinterpret_cast<volatile int*>(bars + 5);
+  uint64_t* q16_full = bars + 4;
+  uint32_t* tbase = reinterpret_cast<uint32_t*>(bars + 5);
+  volatile int* abort = reinterpret_cast<volatile int*>(bars + 6);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -273,10 +326,19 @@ __global__ void __launch_bounds__(128, 1)
   const int b = bh / H, h = bh % H;
   const int bg = b * Hkv + h / (H / Hkv);
   const int row = qt * 128 + tid;
-  const int nkt = CAUSAL ? qt + 1 : (N + 127) / 128;
+  const int ntk = (N + 127) / 128;
+  const int nkt = CAUSAL ? qt + 1 : ntk;
+  // this CTA's promoted key tiles: the list of its 256-row query block (ascending)
+  const int* plist = nullptr;
+  int pcount = 0;
+  if (kv_list != nullptr) {
+    const long long qb = static_cast<long long>(bh) * ((N + 255) / 256) + qt / 2;
+    plist = kv_list + qb * ntk;
+    pcount = __ldg(kv_count + qb);
+  }
 
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < 5; ++i) mbar_init(bars + i, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -303,55 +365,107 @@ __global__ void __launch_bounds__(128, 1)
   if (tid == 0) {
     mbar_arrive_expect_tx(q_full, Cfg::kQK);
     tma_load_3d(sq, &tm_q, q_full, 0, qt * 128, bh);
+    if (pcount > 0) {
+      mbar_arrive_expect_tx(q16_full, Cfg::kT16);
+#pragma unroll
+      for (int x = 0; x < D / 64; ++x)
+        tma_load_3d(sq16 + x * Cfg::kBox16, &tm_q16, q16_full, 64 * x, qt * 128, bh);
+    }
   }
-  const float gqk = __ldg(q_g + bh) * __ldg(k_g + bg) * sl2;  // S to log2 units
+  // c = q . mean for this row (FP16 scores minus c see the smoothed keys)
+  float cq = 0.0f;
+  if (pcount > 0 && row < N) {
+    const uint4* qr = reinterpret_cast<const uint4*>(q16 + (static_cast<size_t>(bh) * N + row) * D);
+    const float* mr = k_mean + static_cast<size_t>(bg) * D;
+#pragma unroll 4
+    for (int c8 = 0; c8 < D / 8; ++c8) {
+      const uint4 v = __ldg(qr + c8);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        cq = fmaf(half_bits_to_float(w[e] & 0xFFFFu), __ldg(mr + 8 * c8 + 2 * e), cq);
+        cq = fmaf(half_bits_to_float(w[e] >> 16), __ldg(mr + 8 * c8 + 2 * e + 1), cq);
+      }
+    }
+  }
+  const float gqk = __ldg(q_g + bh) * __ldg(k_g + bg) * sl2;  // FP4 S to log2 units
   const float gv = __ldg(v_g + bg);
   float m = -INFINITY, l = 0.0f;
   float o[D];
 #pragma unroll
   for (int c = 0; c < D; ++c) o[c] = 0.0f;
   bool ok = true;
+  bool q16_ready = false;
+  int pi = 0;
 
   for (int kt = 0; kt < nkt; ++kt) {
     const uint32_t ph = static_cast<uint32_t>(kt & 1);
-    // (a) K's and V's block scales into this warp's sub-partition
+    while (pi < pcount && __ldg(plist + pi) < kt) ++pi;
+    const bool promoted = pi < pcount && __ldg(plist + pi) == kt;
+    // (a) FP4 tiles: K's and V's block scales into this warp's sub-partition
+    if (!promoted) {
 #pragma unroll
-    for (int kc = 0; kc < Cfg::kStepsQK; ++kc) {
-      uint32_t w[4];
-      load_sf_words(ksf, D, N, kt * 128, kc, w);
-      tmem_st32x4(lane_base + Cfg::kColSfk + 4 * kc, w[0], w[1], w[2], w[3]);
-    }
+      for (int kc = 0; kc < Cfg::kStepsQK; ++kc) {
+        uint32_t w[4];
+        load_sf_words(ksf, D, N, kt * 128, kc, w);
+        tmem_st32x4(lane_base + Cfg::kColSfk + 4 * kc, w[0], w[1], w[2], w[3]);
+      }
 #pragma unroll
-    for (int kc = 0; kc < 2; ++kc) {
-      uint32_t w[4];
+      for (int kc = 0; kc < 2; ++kc) {
+        uint32_t w[4];
 #pragma unroll
-      for (int r1 = 0; r1 < Cfg::kSfvCols; ++r1)
-        w[r1] = __ldg(reinterpret_cast<const uint32_t*>(
-            vsf + static_cast<size_t>(lane + 32 * r1) * (Np / 16) + kt * 8 + 4 * kc));
-      if constexpr (D == 128)
-        tmem_st32x4(lane_base + Cfg::kColSfv + 4 * kc, w[0], w[1], w[2], w[3]);
-      else
-        tmem_st32x2(lane_base + Cfg::kColSfv + 2 * kc, w[0], w[1]);
+        for (int r1 = 0; r1 < Cfg::kSfvCols; ++r1)
+          w[r1] = __ldg(reinterpret_cast<const uint32_t*>(
+              vsf + static_cast<size_t>(lane + 32 * r1) * (Np / 16) + kt * 8 + 4 * kc));
+        if constexpr (D == 128)
+          tmem_st32x4(lane_base + Cfg::kColSfv + 4 * kc, w[0], w[1], w[2], w[3]);
+        else
+          tmem_st32x2(lane_base + Cfg::kColSfv + 2 * kc, w[0], w[1]);
+      }
     }
     tmem_st_wait();
     tc_fence_before();
     __syncthreads();
-    // (b) K and V^T tiles, then S = Q K^T (FP4, block-scaled)
+    // (b) the tile's operands, then S = Q K^T
     if (tid == 0) {
       tc_fence_after();
-      mbar_arrive_expect_tx(kv_full, Cfg::kQK + Cfg::kVt);
-      tma_load_3d(sk, &tm_k, kv_full, 0, kt * 128, bg);
-      tma_load_3d(sv, &tm_vt, kv_full, kt * 64, 0, bg);
-      const bool loaded = (kt > 0 || mbar_wait(q_full, 0, abort)) && mbar_wait(kv_full, ph, abort);
+      bool loaded;
+      if (promoted) {
+        mbar_arrive_expect_tx(kv_full, 2 * Cfg::kT16);
+#pragma unroll
+        for (int x = 0; x < D / 64; ++x) {
+          tma_load_3d(sk16 + x * Cfg::kBox16, &tm_k16, kv_full, 64 * x, kt * 128, bg);
+          tma_load_3d(sv16 + x * Cfg::kBox16, &tm_v16, kv_full, 64 * x, kt * 128, bg);
+        }
+        loaded = (q16_ready || mbar_wait(q16_full, 0, abort)) && mbar_wait(kv_full, ph, abort);
+        q16_ready = true;
+      } else {
+        mbar_arrive_expect_tx(kv_full, Cfg::kQK + Cfg::kVt);
+        tma_load_3d(sk, &tm_k, kv_full, 0, kt * 128, bg);
+        tma_load_3d(sv, &tm_vt, kv_full, kt * 64, 0, bg);
+        loaded = (kt > 0 || mbar_wait(q_full, 0, abort)) && mbar_wait(kv_full, ph, abort);
+      }
+      if (kt == 0 && promoted && loaded) loaded = mbar_wait(q_full, 0, abort);
       if (loaded) {
         tc_fence_after();
-        constexpr uint32_t id = idesc_nvf4(128, 128);
+        if (promoted) {
+          constexpr uint32_t id = idesc_f16_f32_kk(128, 128);
 #pragma unroll
-        for (int kc = 0; kc < Cfg::kStepsQK; ++kc) {
-          const uint64_t ad = smem_desc(smem_u32(sq) + kc * 32, 16, Cfg::kSboQK, Cfg::kSwQK);
-          const uint64_t bd = smem_desc(smem_u32(sk) + kc * 32, 16, Cfg::kSboQK, Cfg::kSwQK);
-          mma_nvf4_ss(tmem + Cfg::kColS, ad, bd, id, tmem + Cfg::kColSfq + 4 * kc,
-                      tmem + Cfg::kColSfk + 4 * kc, kc > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk / 4) * Cfg::kBox16 + (kk % 4) * 32;
+            const uint64_t ad = smem_desc(smem_u32(sq16) + off, 16, 1024, kSwizzle128B);
+            const uint64_t bd = smem_desc(smem_u32(sk16) + off, 16, 1024, kSwizzle128B);
+            mma_f16_ss(tmem + Cfg::kColS, ad, bd, id, kk > 0 ? 1u : 0u);
+          }
+        } else {
+          constexpr uint32_t id = idesc_nvf4(128, 128);
+#pragma unroll
+          for (int kc = 0; kc < Cfg::kStepsQK; ++kc) {
+            const uint64_t ad = smem_desc(smem_u32(sq) + kc * 32, 16, Cfg::kSboQK, Cfg::kSwQK);
+            const uint64_t bd = smem_desc(smem_u32(sk) + kc * 32, 16, Cfg::kSboQK, Cfg::kSwQK);
+            mma_nvf4_ss(tmem + Cfg::kColS, ad, bd, id, tmem + Cfg::kColSfq + 4 * kc,
+                        tmem + Cfg::kColSfk + 4 * kc, kc > 0 ? 1u : 0u);
+          }
         }
         mma_commit(s_done);
       }
@@ -359,8 +473,10 @@ __global__ void __launch_bounds__(128, 1)
     ok = __syncthreads_and(mbar_wait(s_done, ph, abort));
     if (!ok) break;
     tc_fence_after();
-    // (c) this row's online softmax step and its two-level FP4 quantization
+    // (c) this row's online softmax step
     const int kbase = kt * 128;
+    const float xs = promoted ? sl2 : gqk;   // x = (S - xo) * xs, log2 units
+    const float xo = promoted ? cq : 0.0f;
     float tmax = -INFINITY;
 #pragma unroll 1
     for (int cc = 0; cc < 4; ++cc) {
@@ -371,84 +487,123 @@ __global__ void __launch_bounds__(128, 1)
       for (int t = 0; t < 32; ++t) {
         const int key = kbase + 32 * cc + t;
         const bool valid = key < N && (!CAUSAL || key <= row);
-        if (valid) tmax = fmaxf(tmax, __uint_as_float(v[t]) * gqk);
+        if (valid) tmax = fmaxf(tmax, (__uint_as_float(v[t]) - xo) * xs);
       }
     }
     const float m_new = fmaxf(m, tmax);
     const float corr = exp2f(m - m_new);
-    const float gp = __fdiv_rn(exp2f(tmax - m_new), kNvfp4Div);
-    const float sixg = __fmul_rn(6.0f, gp);
+    float f;      // factor of the tile's P V accumulator
     float lsum = 0.0f;
-    uint32_t sfw0 = 0, sfw1 = 0;
+    if (promoted) {
+      // fp16 P pairs (keys 2c, 2c + 1 in column c) into tensor memory; l takes the rounded P
 #pragma unroll 1
-    for (int cc = 0; cc < 4; ++cc) {
-      uint32_t v[32];
-      tmem_ld32(lane_base + Cfg::kColS + 32 * cc, v);
-      tmem_ld_wait(v);
-      float p[32];
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(lane_base + Cfg::kColS + 32 * cc, v);
+        tmem_ld_wait(v);
+        uint32_t pk[16];
 #pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        const int key = kbase + 32 * cc + t;
-        const bool valid = key < N && (!CAUSAL || key <= row);
-        p[t] = valid ? exp2f(__uint_as_float(v[t]) * gqk - m_new) : 0.0f;
-      }
-      uint32_t cw[4];
-#pragma unroll
-      for (int hb = 0; hb < 2; ++hb) {
-        float* pb = p + 16 * hb;
-        float bmax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, pb[i]);
-        const uint32_t s = gp > 0.0f ? ue4m3_byte(__fdiv_rn(bmax, sixg)) : 0u;
-        cw[2 * hb] = 0u;
-        cw[2 * hb + 1] = 0u;
-        if (s != 0u) {
-          const float sc = __fmul_rn(ue4m3_value(s), gp);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) pb[i] = __fdiv_rn(pb[i], sc);
-          cw[2 * hb] = e2m1x8(pb);
-          cw[2 * hb + 1] = e2m1x8(pb + 8);
-          lsum += 0.5f * sc *
-                  static_cast<float>(e2m1x8_twice_sum(cw[2 * hb]) + e2m1x8_twice_sum(cw[2 * hb + 1]));
+        for (int t = 0; t < 32; t += 2) {
+          const int key = kbase + 32 * cc + t;
+          const bool v0 = key < N && (!CAUSAL || key <= row);
+          const bool v1 = key + 1 < N && (!CAUSAL || key + 1 <= row);
+          const float p0 = v0 ? exp2f((__uint_as_float(v[t]) - xo) * xs - m_new) : 0.0f;
+          const float p1 = v1 ? exp2f((__uint_as_float(v[t + 1]) - xo) * xs - m_new) : 0.0f;
+          pk[t / 2] = pack_half2(p0, p1);
+          lsum = add_half2_f32(lsum, pk[t / 2]);
         }
-        const int blk = 2 * cc + hb;  // 16-key block 0..7 of the tile
-        if (blk < 4) sfw0 |= s << (8 * blk);
-        else sfw1 |= s << (8 * (blk - 4));
+        tmem_st32x16(lane_base + Cfg::kColP16 + 16 * cc, pk);
       }
-      // 16 bytes (keys 32 cc .. 32 cc + 31) into the 64-byte-swizzled row of the P operand
-      st_shared_v4(smem_u32(sp) + tid * 64 + ((cc ^ ((tid >> 1) & 3)) << 4), cw[0], cw[1], cw[2],
-                   cw[3]);
-    }
-    l = l * corr + lsum;
-    sfp[tid] = sfw0;
-    sfp[128 + tid] = sfw1;
-    fence_proxy_async_smem();
-    __syncthreads();
-    // (d) P's scales: row r0 + 32 r1 in column r1 of lane r0, in every sub-partition
+      l = l * corr + lsum;
+      f = 1.0f;
+      tmem_st_wait();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t id = idesc_f16_f32_bmn(128, D);
+        const uint64_t dv = smem_desc(smem_u32(sv16), Cfg::kBox16, 1024, kSwizzle128B);
 #pragma unroll
-    for (int kc = 0; kc < 2; ++kc)
-      tmem_st32x4(lane_base + Cfg::kColSfp + 4 * kc, sfp[128 * kc + lane], sfp[128 * kc + lane + 32],
-                  sfp[128 * kc + lane + 64], sfp[128 * kc + lane + 96]);
-    tmem_st_wait();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t id = idesc_nvf4(128, D);
-#pragma unroll
-      for (int kc = 0; kc < 2; ++kc) {
-        const uint64_t ad = smem_desc(smem_u32(sp) + kc * 32, 16, 512, kSwizzle64B);
-        const uint64_t bd = smem_desc(smem_u32(sv) + kc * 32, 16, 512, kSwizzle64B);
-        mma_nvf4_ss(tmem + Cfg::kColO, ad, bd, id, tmem + Cfg::kColSfp + 4 * kc,
-                    tmem + Cfg::kColSfv + Cfg::kSfvCols * kc, kc > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_f16_ts(tmem + Cfg::kColO, tmem + Cfg::kColP16 + 8 * kk, dv + 128 * kk, id,
+                     kk > 0 ? 1u : 0u);
+        mma_commit(o_done);
       }
-      mma_commit(o_done);
+    } else {
+      // two-level FP4 quantization of the P row
+      const float gp = __fdiv_rn(exp2f(tmax - m_new), kNvfp4Div);
+      const float sixg = __fmul_rn(6.0f, gp);
+      uint32_t sfw0 = 0, sfw1 = 0;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(lane_base + Cfg::kColS + 32 * cc, v);
+        tmem_ld_wait(v);
+        float p[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          const int key = kbase + 32 * cc + t;
+          const bool valid = key < N && (!CAUSAL || key <= row);
+          p[t] = valid ? exp2f(__uint_as_float(v[t]) * gqk - m_new) : 0.0f;
+        }
+        uint32_t cw[4];
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+          float* pb = p + 16 * hb;
+          float bmax = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, pb[i]);
+          const uint32_t s = gp > 0.0f ? ue4m3_byte(__fdiv_rn(bmax, sixg)) : 0u;
+          cw[2 * hb] = 0u;
+          cw[2 * hb + 1] = 0u;
+          if (s != 0u) {
+            const float sc = __fmul_rn(ue4m3_value(s), gp);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pb[i] = __fdiv_rn(pb[i], sc);
+            cw[2 * hb] = e2m1x8(pb);
+            cw[2 * hb + 1] = e2m1x8(pb + 8);
+            lsum += 0.5f * sc *
+                    static_cast<float>(e2m1x8_twice_sum(cw[2 * hb]) + e2m1x8_twice_sum(cw[2 * hb + 1]));
+          }
+          const int blk = 2 * cc + hb;  // 16-key block 0..7 of the tile
+          if (blk < 4) sfw0 |= s << (8 * blk);
+          else sfw1 |= s << (8 * (blk - 4));
+        }
+        // 16 bytes (keys 32 cc .. 32 cc + 31) into the 64-byte-swizzled row of the P operand
+        st_shared_v4(smem_u32(sp) + tid * 64 + ((cc ^ ((tid >> 1) & 3)) << 4), cw[0], cw[1], cw[2],
+                     cw[3]);
+      }
+      l = l * corr + lsum;
+      f = gp * gv;
+      sfp[tid] = sfw0;
+      sfp[128 + tid] = sfw1;
+      fence_proxy_async_smem();
+      __syncthreads();
+      // (d) P's scales: row r0 + 32 r1 in column r1 of lane r0, in every sub-partition
+#pragma unroll
+      for (int kc = 0; kc < 2; ++kc)
+        tmem_st32x4(lane_base + Cfg::kColSfp + 4 * kc, sfp[128 * kc + lane],
+                    sfp[128 * kc + lane + 32], sfp[128 * kc + lane + 64], sfp[128 * kc + lane + 96]);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t id = idesc_nvf4(128, D);
+#pragma unroll
+        for (int kc = 0; kc < 2; ++kc) {
+          const uint64_t ad = smem_desc(smem_u32(sp) + kc * 32, 16, 512, kSwizzle64B);
+          const uint64_t bd = smem_desc(smem_u32(sv) + kc * 32, 16, 512, kSwizzle64B);
+          mma_nvf4_ss(tmem + Cfg::kColO, ad, bd, id, tmem + Cfg::kColSfp + 4 * kc,
+                      tmem + Cfg::kColSfv + Cfg::kSfvCols * kc, kc > 0 ? 1u : 0u);
+        }
+        mma_commit(o_done);
+      }
     }
     ok = __syncthreads_and(mbar_wait(o_done, ph, abort));
     if (!ok) break;
     tc_fence_after();
-    // (e) fold the tile's P V into the output row: O = O * corr + (P^ V^) * gP * gV
-    const float f = gp * gv;
+    // (e) fold the tile's P V into the output row: O = O * corr + acc * f
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
       uint32_t v[32];
@@ -459,6 +614,8 @@ __global__ void __launch_bounds__(128, 1)
     }
     m = m_new;
   }
+  // a promoted list with no tile up to the causal diagonal leaves the fp16 Q load unconsumed
+  if (tid == 0 && pcount > 0 && !q16_ready) (void)mbar_wait(q16_full, 0, abort);
   if (ok && row < N) {
     const float inv = 1.0f / l;
     uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + row) * D);

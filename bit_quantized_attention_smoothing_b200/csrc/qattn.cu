@@ -117,21 +117,22 @@ bool make_fp4_vt_map(CUtensorMap* m, const void* base, int d, int Np, long long 
 }
 
 template <int D, bool CAUSAL>
-qattn_status launch_attn_nvfp4(const CUtensorMap& tq, const CUtensorMap& tk,
-                               const CUtensorMap& tv, const uint8_t* q_sf, const uint8_t* k_sf,
+qattn_status launch_attn_nvfp4(const CUtensorMap* maps, const uint8_t* q_sf, const uint8_t* k_sf,
                                const uint8_t* vt_sf, const float* q_g, const float* k_g,
-                               const float* v_g, void* out, int B, int H, int Hkv, int N, int Np,
-                               cudaStream_t st) {
-  // 120 KB of shared memory keeps one CTA (and its 512 tensor-memory columns) per SM.
-  const int smem = 120 * 1024;
-  static_assert(Fp4AttnCfg<D>::kSmemUsed <= 120 * 1024, "shared memory");
+                               const float* v_g, const void* q16, const float* k_mean,
+                               const int* kv_list, const int* kv_count, void* out, int B, int H,
+                               int Hkv, int N, int Np, cudaStream_t st) {
+  // 140 KB of shared memory keeps one CTA (and its 512 tensor-memory columns) per SM.
+  const int smem = 140 * 1024;
+  static_assert(Fp4AttnCfg<D>::kSmemUsed <= 140 * 1024, "shared memory");
   auto kern = attn_nvfp4_kernel<D, CAUSAL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return QATTN_ERR_CUDA;
   const dim3 grid((N + 127) / 128, B * H);
   const float sl2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-  kern<<<grid, 128, smem, st>>>(tq, tk, tv, q_sf, k_sf, vt_sf, q_g, k_g, v_g,
-                                static_cast<__half*>(out), H, Hkv, N, Np, sl2);
+  kern<<<grid, 128, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], q_sf, k_sf,
+                                vt_sf, q_g, k_g, v_g, static_cast<const uint16_t*>(q16), k_mean,
+                                kv_list, kv_count, static_cast<__half*>(out), H, Hkv, N, Np, sl2);
   return launch_status();
 }
 
@@ -743,26 +744,42 @@ qattn_status qattn_debug_qk_int32(const int8_t* q_i8, const int8_t* k_i8, int32_
 qattn_status qattn_attn_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales, const float* q_g,
                               const uint8_t* k_codes, const uint8_t* k_scales, const float* k_g,
                               const uint8_t* vt_codes, const uint8_t* vt_scales, const float* v_g,
-                              void* out, int B, int H, int Hkv, int N, int d, int causal,
-                              qattn_stream_t stream) {
+                              const void* q, const void* k, const void* v, const float* k_mean,
+                              const int* kv_list, const int* kv_count, void* out, int B, int H,
+                              int Hkv, int N, int d, int causal, qattn_stream_t stream) {
   qattn_status s = check_shape(B, H, Hkv, N, d);
   if (s != QATTN_OK) return s;
   s = check_ptrs(q_codes, q_scales, q_g, k_codes, k_scales, k_g, vt_codes, vt_scales, v_g, out);
   if (s != QATTN_OK) return s;
+  const bool promote = kv_list != nullptr;
+  if (promote && (s = check_ptrs(q, k, v, k_mean, kv_list, kv_count)) != QATTN_OK) return s;
   if (static_cast<long long>(B) * H > 65535) return QATTN_ERR_UNSUPPORTED;
   if ((s = device_ok()) != QATTN_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int Np = (N + 127) / 128 * 128;
-  CUtensorMap tq, tk, tv;
-  if (!make_fp4_map(&tq, q_codes, d, N, static_cast<long long>(B) * H) ||
-      !make_fp4_map(&tk, k_codes, d, N, static_cast<long long>(B) * Hkv) ||
-      !make_fp4_vt_map(&tv, vt_codes, d, Np, static_cast<long long>(B) * Hkv))
+  CUtensorMap maps[6];
+  if (!make_fp4_map(&maps[0], q_codes, d, N, static_cast<long long>(B) * H) ||
+      !make_fp4_map(&maps[1], k_codes, d, N, static_cast<long long>(B) * Hkv) ||
+      !make_fp4_vt_map(&maps[2], vt_codes, d, Np, static_cast<long long>(B) * Hkv))
     return QATTN_ERR_CUDA;
+  if (promote) {
+    // fp16 Q, K, V tiles: boxes of 64 columns x 128 rows, 128-byte swizzle
+    if (!make_v_map(&maps[3], q, d, N, static_cast<long long>(B) * H) ||
+        !make_v_map(&maps[4], k, d, N, static_cast<long long>(B) * Hkv) ||
+        !make_v_map(&maps[5], v, d, N, static_cast<long long>(B) * Hkv))
+      return QATTN_ERR_CUDA;
+  } else {
+    maps[3] = maps[4] = maps[5] = maps[0];  // never read without promotion
+  }
+  const uint16_t* q16 = static_cast<const uint16_t*>(q);
+#define QATTN_FP4_ARGS maps, q_scales, k_scales, vt_scales, q_g, k_g, v_g, q16, k_mean, kv_list, \
+                       kv_count, out, B, H, Hkv, N, Np, st
   if (d == 128)
-    return causal ? launch_attn_nvfp4<128, true>(tq, tk, tv, q_scales, k_scales, vt_scales, q_g, k_g, v_g, out, B, H, Hkv, N, Np, st)
-                  : launch_attn_nvfp4<128, false>(tq, tk, tv, q_scales, k_scales, vt_scales, q_g, k_g, v_g, out, B, H, Hkv, N, Np, st);
-  return causal ? launch_attn_nvfp4<64, true>(tq, tk, tv, q_scales, k_scales, vt_scales, q_g, k_g, v_g, out, B, H, Hkv, N, Np, st)
-                : launch_attn_nvfp4<64, false>(tq, tk, tv, q_scales, k_scales, vt_scales, q_g, k_g, v_g, out, B, H, Hkv, N, Np, st);
+    return causal ? launch_attn_nvfp4<128, true>(QATTN_FP4_ARGS)
+                  : launch_attn_nvfp4<128, false>(QATTN_FP4_ARGS);
+  return causal ? launch_attn_nvfp4<64, true>(QATTN_FP4_ARGS)
+                : launch_attn_nvfp4<64, false>(QATTN_FP4_ARGS);
+#undef QATTN_FP4_ARGS
 }
 
 qattn_status qattn_debug_qk_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales,

@@ -97,7 +97,8 @@ def _lib():
         L.qattn_debug_wait_timeout.restype = i
         L.qattn_quant_nvfp4.argtypes = [P, P, i, i, i, i, P, P, P, P]
         L.qattn_quant_nvfp4.restype = i
-        L.qattn_attn_nvfp4.argtypes = [P, P, P, P, P, P, P, P, P, P, i, i, i, i, i, i, P]
+        L.qattn_attn_nvfp4.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                       i, i, i, i, i, i, P]
         L.qattn_attn_nvfp4.restype = i
         L.qattn_debug_qk_nvfp4.argtypes = [P, P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, i, P]
         L.qattn_debug_qk_nvfp4.restype = i
@@ -331,17 +332,22 @@ def qattn_debug_qk_int32(q_i8, k_i8, b, h, qt0, nqt, kt0, nkt, s_out=None, strea
 
 
 def qattn_attn_nvfp4(q_nvfp4, k_nvfp4, vt_nvfp4, B, H, Hkv, N, d, causal=False, out=None,
-                     stream=None):
+                     promote=None, stream=None):
     """FP4-path attention from NVFP4 operands (each the (codes, scales, gscale) triple of
-    qattn_quant_nvfp4: Q and K along the channels, V along the tokens); fp16 out [B, H, N, d]."""
+    qattn_quant_nvfp4: Q and smoothed K along the channels, V along the tokens); fp16 out
+    [B, H, N, d].  promote = (q, k, v, k_mean, kv_list, kv_count): fp16 inputs, the mean K was
+    smoothed with, and qattn_block_select's lists of the key tiles to compute in FP16."""
     qc, qs, qg = q_nvfp4
     kc, ks, kg = k_nvfp4
     vc, vs, vg = vt_nvfp4
     if out is None:
         out = torch.empty(B, H, N, d, dtype=torch.float16, device=qc.device)
+    pq = pk = pv = pm = pl = pc = None
+    if promote is not None:
+        pq, pk, pv, pm, pl, pc = promote
     st = _lib().qattn_attn_nvfp4(_p(qc), _p(qs), _p(qg), _p(kc), _p(ks), _p(kg), _p(vc), _p(vs),
-                                 _p(vg), _p(out), B, H, Hkv, N, d, int(bool(causal)),
-                                 _stream(stream))
+                                 _p(vg), _p(pq), _p(pk), _p(pv), _p(pm), _p(pl), _p(pc), _p(out),
+                                 B, H, Hkv, N, d, int(bool(causal)), _stream(stream))
     _check("qattn_attn_nvfp4", st)
     return out
 

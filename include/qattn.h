@@ -242,20 +242,28 @@ qattn_status qattn_quant_nvfp4(const void* x, const float* mean, int S, int R, i
                                int along_rows, uint8_t* codes, uint8_t* scales, float* gscale,
                                qattn_stream_t stream);
 
-/* Attention on the FP4 path (ThriftAttention page, method section: "FP4 path" and "online
- * merge"; every key tile in FP4, no promotion): S = FP4 Q K^T on the block-scaled tensor cores,
- * the online softmax over key tiles of 128, each tile's P row quantized in two levels (a binary32
- * row scale gP = max p / 2688, then NVFP4 blocks of 16 keys with E4M3 scales, the same binary32
- * steps as qattn_quant_nvfp4), O += P^ V^ on the block-scaled tensor cores with V NVFP4 along the
- * tokens; l sums the dequantized P; out = O / l in fp16 [B][H][N][d].
- * Inputs as qattn_quant_nvfp4 writes them: q_* along the channels over B*H slices, k_* (smoothed
- * K) over B*Hkv slices, vt_* along the rows (transposed, Np = N rounded up to 128) over B*Hkv
- * slices.  Same checks and errors as qattn_attn_quantized; B * H <= 65535. */
+/* Attention on the FP4 path with FP16 promotion (ThriftAttention page, method section: the top-k
+ * query-key block pairs in FP16, the rest in FP4 with NVFP4, merged by one online softmax; the
+ * FP4 probability blocks quantized in two levels).
+ * FP4 tiles: S = FP4 Q K^T on the block-scaled tensor cores; each tile's P row quantized as a
+ * binary32 row scale gP = max p / 2688, then NVFP4 blocks of 16 keys with E4M3 scales (the same
+ * binary32 steps as qattn_quant_nvfp4); O += P^ V^ on the block-scaled tensor cores, V NVFP4
+ * along the tokens.  Promoted tiles (kv_list non-NULL): the key tiles listed for the query tile's
+ * 256-row block (qattn_block_select's lists) run as fp16 q . (k - k_mean) on the f16 tensor cores
+ * (the same smoothed keys as the FP4 tiles), fp16-rounded P, fp16 V.  l sums the P values the
+ * P V product uses; out = O / l in fp16 [B][H][N][d].
+ * Inputs as qattn_quant_nvfp4 writes them: q_* along the channels over B*H slices, k_* (K minus
+ * k_mean) over B*Hkv slices, vt_* along the rows (transposed, Np = N rounded up to 128) over B*Hkv
+ * slices.  With kv_list == NULL every tile runs in FP4 and q, k, v, k_mean, kv_count are not read;
+ * otherwise q [B][H][N][d], k and v [B][Hkv][N][d] are the fp16 inputs, k_mean float [B*Hkv][d],
+ * kv_list / kv_count as qattn_block_select writes them.  Same checks and errors as
+ * qattn_attn_quantized; B * H <= 65535. */
 qattn_status qattn_attn_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales, const float* q_g,
                               const uint8_t* k_codes, const uint8_t* k_scales, const float* k_g,
                               const uint8_t* vt_codes, const uint8_t* vt_scales, const float* v_g,
-                              void* out, int B, int H, int Hkv, int N, int d, int causal,
-                              qattn_stream_t stream);
+                              const void* q, const void* k, const void* v, const float* k_mean,
+                              const int* kv_list, const int* kv_count, void* out, int B, int H,
+                              int Hkv, int N, int d, int causal, qattn_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
  * Checks.

@@ -145,10 +145,16 @@ def test_debug_qk_nvfp4_argument_checks():
 
 def test_attn_nvfp4_argument_checks():
     L = Q.load()
-    a = tuple(P(16 * (i + 1)) for i in range(10))
-    assert L.qattn_attn_nvfp4(None, *a[1:], 1, 4, 2, 256, 128, 1, None) == 1
-    assert L.qattn_attn_nvfp4(*a, 1, 4, 3, 256, 128, 1, None) == 1         # H % Hkv
-    assert L.qattn_attn_nvfp4(*a, 1, 4, 2, 0, 128, 1, None) == 1           # N
-    assert L.qattn_attn_nvfp4(*a, 1, 4, 2, 256, 96, 1, None) == 2          # d
-    assert L.qattn_attn_nvfp4(*a, 300, 256, 2, 256, 128, 1, None) == 2    # B * H > 65535
-    assert L.qattn_attn_nvfp4(*a[:9], P(24), 1, 4, 2, 256, 128, 1, None) == 3
+    a = tuple(P(16 * (i + 1)) for i in range(9))
+    none6 = (None,) * 6
+    prom = tuple(P(256 + 16 * i) for i in range(6))
+    o = P(1024)
+    assert L.qattn_attn_nvfp4(None, *a[1:], *none6, o, 1, 4, 2, 256, 128, 1, None) == 1
+    assert L.qattn_attn_nvfp4(*a, *none6, o, 1, 4, 3, 256, 128, 1, None) == 1         # H % Hkv
+    assert L.qattn_attn_nvfp4(*a, *none6, o, 1, 4, 2, 0, 128, 1, None) == 1           # N
+    assert L.qattn_attn_nvfp4(*a, *none6, o, 1, 4, 2, 256, 96, 1, None) == 2          # d
+    assert L.qattn_attn_nvfp4(*a, *none6, o, 300, 256, 2, 256, 128, 1, None) == 2    # B * H
+    assert L.qattn_attn_nvfp4(*a, *none6, P(24), 1, 4, 2, 256, 128, 1, None) == 3     # out
+    # promotion: lists given, an fp16 operand or the mean missing / misaligned
+    assert L.qattn_attn_nvfp4(*a, None, *prom[1:], o, 1, 4, 2, 256, 128, 1, None) == 1
+    assert L.qattn_attn_nvfp4(*a, *prom[:3], P(20), *prom[4:], o, 1, 4, 2, 256, 128, 1, None) == 3

@@ -339,3 +339,87 @@ def test_attn_nvfp4_full_size_sampled_rows(lib, oracle):
                                         rows=(np.zeros_like(rows_i), rows_i))
     got = out[0, h, torch.from_numpy(rows_i).cuda()].float().cpu().numpy()
     _check_fp4_out(got, ref, slack, "llama8b_32k full")
+
+
+# ---- FP16 promotion of the selected key tiles (the ThriftAttention page's method) ----
+
+def _lists_equal(gl, gc, ol, oc):
+    gl, gc = gl.cpu().numpy(), gc.cpu().numpy()
+    assert np.array_equal(gc, oc)
+    for bh in range(oc.shape[0]):
+        for i in range(oc.shape[1]):
+            assert np.array_equal(gl[bh, i, :oc[bh, i]], ol[bh, i, :oc[bh, i]])
+
+
+PROMO_CASES = [
+    ("tiny", {"N": 300}, 1),
+    ("llama8b_32k", {"H": 4, "Hkv": 2, "N": 700}, 1),
+    ("llama8b_32k", {"B": 2, "H": 2, "Hkv": 1, "N": 600, "causal": False}, 2),
+    ("wide64", {"B": 1, "H": 3, "Hkv": 1, "N": 513, "causal": True}, 0),
+    ("prefill4k", {"B": 1, "H": 2, "Hkv": 2, "N": 640}, 100),          # every tile promoted
+]
+
+
+@pytest.mark.parametrize("name,over,topk", PROMO_CASES,
+                         ids=[f"{n}-" + "-".join(f"{k}{v}" for k, v in o.items()) + f"-top{t}"
+                              for n, o, t in PROMO_CASES])
+def test_attn_nvfp4_promoted_against_oracle(lib, oracle, name, over, topk):
+    """Key tiles chosen by the block-mean top-k (lists bit-exact against the oracle's) run in
+    FP16, the others in FP4, merged by one online softmax."""
+    w = WORKLOADS[name].with_(**over)
+    q, k, v = make_inputs(w, device="cpu")
+    qn, kn, vn = _nvfp4_operands(oracle, w, q, k, v)
+    sums = oracle.k_channel_sums(np16(k), w.B, w.Hkv, w.N, w.d)
+    mean = np.array([oracle.lib().oracle_mean_from_sum(int(s), w.N) for s in sums.ravel()],
+                    dtype=np.float32).reshape(w.B * w.Hkv, w.d)
+    qg, kg, vg = q.cuda(), k.cuda(), v.cuda()
+    gl, gc = lib.qattn_block_select(qg, kg, topk, causal=w.causal)
+    ol, oc = oracle.block_select(np16(q), np16(k), w.B, w.H, w.Hkv, w.N, w.d, w.causal, topk)
+    _lists_equal(gl, gc, ol, oc)
+    out = lib.qattn_attn_nvfp4(_upload(qn), _upload(kn), _upload(vn), w.B, w.H, w.Hkv, w.N, w.d,
+                               causal=w.causal,
+                               promote=(qg, kg, vg, torch.from_numpy(mean).cuda(), gl, gc))
+    assert lib.qattn_check_device_status() == 0
+    mask = oracle.tile_mask(ol, oc, w.N)
+    ref, slack = oracle.attention_nvfp4(qn, kn, vn, w.B, w.H, w.Hkv, w.N, w.d, w.causal,
+                                        promote=mask, q16=np16(q), k16=np16(k), v16=np16(v),
+                                        k_mean=mean)
+    _check_fp4_out(out.float().cpu().numpy().reshape(-1, w.d), ref, slack, f"{name} top{topk}")
+
+
+def test_attn_nvfp4_promoted_full_size_sampled_rows(lib, oracle):
+    """32K tokens, top-16 key tiles per 256-row block in FP16 (plus the diagonals), the rest in
+    FP4; lists, quantization and the mean from the GPU path (lists and the used slices checked
+    against the oracle), sampled rows of one head against the oracle."""
+    w = WORKLOADS["llama8b_32k"]
+    topk = 16
+    q, k, v = make_inputs(w, device="cuda")
+    h = 9
+    g = h // (w.H // w.Hkv)
+    sums = oracle.k_channel_sums(np16(k), 1, w.Hkv, w.N, w.d)
+    mean = np.array([oracle.lib().oracle_mean_from_sum(int(s), w.N) for s in sums.ravel()],
+                    dtype=np.float32).reshape(w.Hkv, w.d)
+    meang = torch.from_numpy(mean).cuda()
+    gq = lib.qattn_quant_nvfp4(q.reshape(w.H, w.N, w.d))
+    gk = lib.qattn_quant_nvfp4(k.reshape(w.Hkv, w.N, w.d), meang)
+    gv = lib.qattn_quant_nvfp4(v.reshape(w.Hkv, w.N, w.d), along_rows=True)
+    gl, gc = lib.qattn_block_select(q, k, topk, causal=True)
+    out = lib.qattn_attn_nvfp4(gq, gk, gv, w.B, w.H, w.Hkv, w.N, w.d, causal=True,
+                               promote=(q, k, v, meang, gl, gc))
+    assert lib.qattn_check_device_status() == 0
+    ol, oc = oracle.block_select(np16(q), np16(k), w.B, w.H, w.Hkv, w.N, w.d, True, topk)
+    _lists_equal(gl, gc, ol, oc)
+    qh, kh, vh = np16(q[0, h:h + 1]), np16(k[0, g:g + 1]), np16(v[0, g:g + 1])
+    qn = oracle.quant_nvfp4(qh.view(np.float16))
+    kn = oracle.quant_nvfp4(kh.view(np.float16), mean=mean[g:g + 1])
+    vn = oracle.quant_nvfp4(vh.view(np.float16), along_rows=True)
+    for mine, ref, s in ((gq, qn, h), (gk, kn, g), (gv, vn, g)):
+        for a, r in zip(mine, ref):
+            assert np.array_equal(a[s:s + 1].cpu().numpy(), r)
+    mask = oracle.tile_mask(ol[h:h + 1], oc[h:h + 1], w.N)
+    rows_i = np.array([0, 1, 255, 256, 5000, 20000, w.N - 129, w.N - 1], dtype=np.int64)
+    ref, slack = oracle.attention_nvfp4(qn, kn, vn, 1, 1, 1, w.N, w.d, True,
+                                        rows=(np.zeros_like(rows_i), rows_i), promote=mask,
+                                        q16=qh, k16=kh, v16=vh, k_mean=mean[g:g + 1])
+    got = out[0, h, torch.from_numpy(rows_i).cuda()].float().cpu().numpy()
+    _check_fp4_out(got, ref, slack, "llama8b_32k promoted full")
