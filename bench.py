@@ -52,6 +52,10 @@ def parse_args(argv=None):
     p.add_argument("--sparse-topk", type=int, default=-1,
                    help="block-sparse mode: key tiles per 256-row query block chosen by the "
                         "block-mean score (top-k plus the causal diagonals); -1 = dense")
+    p.add_argument("--fp4-topk", type=int, default=None,
+                   help="FP4-path mode (NVFP4 operands, two-level FP4 P): the key tiles chosen "
+                        "per 256-row query block (top-k plus the causal diagonals) run in FP16; "
+                        "-1 = every tile in FP4; omitted = the INT8 path")
     return p.parse_args(argv)
 
 
@@ -402,6 +406,241 @@ def run_ours(args):
     return line
 
 
+
+# ------------------------------------------------------------------------------------------------
+# FP4-path mode (--fp4-topk)
+# ------------------------------------------------------------------------------------------------
+
+def oracle_fp4_sample_run(w, q, k, v, topk, target_s):
+    """Times the oracle's FP4 path on a sample: channel mean, NVFP4 quantization of kv head 0 and
+    its first query head (full N), the selection for that head when promoting, then query rows
+    spread over the sequence, the count grown until the run takes about target_s."""
+    from oracle import oracle as O
+    O.build()
+    qs = q[0:1, 0:1].contiguous().cpu().numpy().view(np.uint16)
+    ks = k[0:1, 0:1].contiguous().cpu().numpy().view(np.uint16)
+    vs = v[0:1, 0:1].contiguous().cpu().numpy().view(np.uint16)
+
+    def prep():
+        sums = O.k_channel_sums(ks, 1, 1, w.N, w.d)
+        mean = np.array([O.lib().oracle_mean_from_sum(int(x), w.N) for x in sums.ravel()],
+                        dtype=np.float32).reshape(1, w.d)
+        qn = O.quant_nvfp4(qs.reshape(1, w.N, w.d))
+        kn = O.quant_nvfp4(ks.reshape(1, w.N, w.d), mean=mean)
+        vn = O.quant_nvfp4(vs.reshape(1, w.N, w.d), along_rows=True)
+        mask = None
+        if topk >= 0:
+            lst, cnt = O.block_select(qs, ks, 1, 1, 1, w.N, w.d, w.causal, topk)
+            mask = O.tile_mask(lst, cnt, w.N)
+        return mean, qn, kn, vn, mask
+
+    def run(nrows, pre):
+        mean, qn, kn, vn, mask = pre
+        i = np.linspace(0, w.N - 1, nrows).astype(np.int64)
+        O.attention_nvfp4(qn, kn, vn, 1, 1, 1, w.N, w.d, w.causal, rows=(np.zeros_like(i), i),
+                          promote=mask, q16=qs, k16=ks, v16=vs, k_mean=mean)
+        return i
+
+    t0 = time.perf_counter()
+    pre = prep()
+    t_prep = time.perf_counter() - t0
+    nrows = 2
+    while True:
+        t1 = time.perf_counter()
+        run(nrows, pre)
+        dt = time.perf_counter() - t1
+        if dt >= 0.4 * max(target_s - t_prep, 0.5) or nrows >= w.N:
+            break
+        nrows = int(min(w.N, nrows * min(64.0, max(2.0, 0.8 * max(target_s - t_prep, 0.5) / max(dt, 1e-3)))))
+    t0 = time.perf_counter()
+    i = run(nrows, prep())
+    dt = time.perf_counter() - t0
+    pairs = float(np.sum(i + 1)) if w.causal else float(len(i)) * w.N
+    return {"value": 4.0 * w.d * pairs / dt / 1e12, "unit": "TOPS", "cores": 1, "kind": "oracle",
+            "seconds": round(dt, 3),
+            "sample": (f"kv head 0 and query head 0 of batch 0: channel mean, NVFP4 quantization "
+                       f"of Q, K and V over all N={w.N} tokens"
+                       f"{', the key-tile selection' if topk >= 0 else ''}, then {len(i)} query "
+                       f"rows spread over the sequence ({pairs:.3g} visible pairs, 4*d ops each), "
+                       f"single-threaded")}
+
+
+def run_fp4(args):
+    import torch
+    import torch.distributed as dist
+    from bit_quantized_attention_smoothing_b200 import qattn as Q
+    from bit_quantized_attention_smoothing_b200.workloads import WORKLOADS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = WORKLOADS[args.workload]
+    topk = args.fp4_topk
+    Q.load()
+    q, k, v = make_inputs(w, device="cuda")
+    B, H, Hkv, N, d = w.B, w.H, w.Hkv, w.N, w.d
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        Q.qattn_forward_nvfp4(q, k, v, topk, out, w.causal, stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if Q.qattn_check_device_status(stream) != 0:
+        raise RuntimeError("device status reports a timed-out wait during warm-up")
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(K):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    total_ms = e0.elapsed_time(e1)
+    if Q.qattn_check_device_status(stream) != 0:
+        raise RuntimeError("device status reports a timed-out wait in the timed region")
+    total_ms_max = max_over_ranks(total_ms, world, q.device)
+    ops = w.ops
+    value = weak_scaling_tops(ops, K, world, total_ms_max)
+
+    # the attention kernel alone, on operands the product path prepares (separate loop)
+    mean = torch.empty(B * Hkv, d, dtype=torch.float32, device=q.device)
+    nqb, nkb = -(-N // 128), -(-N // 64)
+    q_i8 = torch.empty(B, H, N, d, dtype=torch.int8, device=q.device)
+    k_i8 = torch.empty(B, Hkv, N, d, dtype=torch.int8, device=q.device)
+    q_s = torch.empty(B, H, nqb, dtype=torch.float32, device=q.device)
+    k_s = torch.empty(B, Hkv, nkb, dtype=torch.float32, device=q.device)
+    ws = torch.empty(Q.qattn_smooth_quant_workspace(B, Hkv, d), dtype=torch.uint8, device=q.device)
+    Q.qattn_smooth_quant(q, k, q_i8, q_s, k_i8, k_s, mean, ws, stream)
+    del q_i8, k_i8
+    qn = Q.qattn_quant_nvfp4(q.reshape(B * H, N, d))
+    kn = Q.qattn_quant_nvfp4(k.reshape(B * Hkv, N, d), mean)
+    vn = Q.qattn_quant_nvfp4(v.reshape(B * Hkv, N, d), along_rows=True)
+    prom = None
+    density_fp16 = 0.0
+    if topk >= 0:
+        kl, kc = Q.qattn_block_select(q, k, topk, w.causal)
+        prom = (q, k, v, mean, kl, kc)
+        cnt = kc.cpu().numpy().astype(np.int64)
+        lst = kl.cpu().numpy()
+        nqt = -(-N // 128)
+        allp = fp16p = 0
+        for bh in range(B * H):
+            for i in range(cnt.shape[1]):
+                for tile in (2 * i, 2 * i + 1):
+                    if tile >= nqt:
+                        continue
+                    lim = tile if w.causal else nqt - 1
+                    allp += lim + 1
+                    fp16p += int((lst[bh, i, :cnt[bh, i]] <= lim).sum())
+        density_fp16 = fp16p / allp
+    ka = max(3, min(K, 10))
+    for _ in range(2):
+        Q.qattn_attn_nvfp4(qn, kn, vn, B, H, Hkv, N, d, w.causal, out, prom, stream)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a0.record(stream)
+    for _ in range(ka):
+        Q.qattn_attn_nvfp4(qn, kn, vn, B, H, Hkv, N, d, w.causal, out, prom, stream)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    attn_ms = a0.elapsed_time(a1) / ka
+
+    # end to end: pinned host q, k, v copied in, the one-call forward, out copied back
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        Q.qattn_forward_nvfp4(qd, kd, vd, topk, out, w.causal, stream)
+        oh.copy_(out, non_blocking=True)
+
+    e2e_step()
+    ke = max(1, args.e2e_steps)
+    barrier()
+    torch.cuda.synchronize()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(ke):
+        e2e_step()
+    x1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1), world, q.device)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    peaks, peak_src = load_peaks()
+    bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    fp4_peak = 4.0 * bf16   # nominal dense FP4:BF16 ratio 9:2.25
+    # ceiling of the kernel's mix: the FP4 pairs at the FP4 rate, the promoted ones at FP16
+    peak = 1.0 / ((1.0 - density_fp16) / fp4_peak + density_fp16 / bf16)
+    achieved = ops / (attn_ms / 1e3) / 1e12
+    launches = 12 + (4 if topk >= 0 else 0)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": round(total_ms_max / K, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e2m1 x e2m1 (ue4m3 block scales) -> f32 for Q K^T and P V"
+                 + ("; f16 x f16 -> f32 for the promoted tiles" if topk >= 0 else ""),
+        "data": "synthetic",
+        "path": "fp4",
+        "config": {"workload": w.name, "B": B, "H": H, "Hkv": Hkv, "N": N, "d": d,
+                   "causal": w.causal, "fp4_topk": topk,
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "l2": "inputs larger than L2, no flush"},
+        "fp16_pair_fraction": round(density_fp16, 4),
+        "attn_ms": round(attn_ms, 4),
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "attn_nvfp4_kernel",
+            "achieved": round(achieved, 2),
+            "peak": round(peak, 1),
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": None,
+            "peak_source": (f"{peak_src} bf16 GEMM burst {bf16:.1f} TF/s; FP4 = 4x (nominal "
+                            f"dense ratio); the promoted fraction of the pairs at the bf16 rate "
+                            f"({'of measured' if peak_src == 'measured' else 'of fallback'})"),
+        },
+        "e2e": {"value": round(weak_scaling_tops(ops, ke, world, e2e_ms), 2), "unit": "TOPS",
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (qh, kh, vh)),
+                "d2h_bytes_per_step": oh.numel() * oh.element_size(), "steps": ke,
+                "api": "pinned host copies + qattn_forward_nvfp4 + copy back"},
+        "gpu_launches": launches * K,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_fp4_sample_run(w, q, k, v, topk, args.cpu_seconds)
+    return line
+
 # ------------------------------------------------------------------------------------------------
 # reference arm: the oracle, timed on the host cores
 # ------------------------------------------------------------------------------------------------
@@ -450,7 +689,12 @@ def run_reference(args):
 
 def main(argv=None):
     args = parse_args(argv)
-    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if args.impl == "reference":
+        line = run_reference(args)
+    elif args.fp4_topk is not None:
+        line = run_fp4(args)
+    else:
+        line = run_ours(args)
     if line is not None:
         print(json.dumps(line), flush=True)
 

@@ -215,6 +215,15 @@ __global__ void __launch_bounds__(256) nvfp4_quant_cols_kernel(
   }
 }
 
+// mean[i] = (float)((double)sums[i] / (N * 2^24)): the smoothing mean from the exact channel sums
+// of K * 2^24, one binary64 division and one rounding to binary32 (as the INT8 path's quantizer).
+__global__ void k_mean_from_sums_kernel(const long long* __restrict__ sums, int N, int n,
+                                        float* __restrict__ mean) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n)
+    mean[i] = __double2float_rn(__ddiv_rn(__ll2double_rn(sums[i]), static_cast<double>(N) * 16777216.0));
+}
+
 // gscale[s] = amax / 2688 in place (gscale holds the maxima as floats on entry).
 __global__ void nvfp4_finalize_kernel(float* __restrict__ gscale, int S) {
   const int s = blockIdx.x * blockDim.x + threadIdx.x;

@@ -294,6 +294,73 @@ qattn_status dispatch_smooth_quant(const void* q, const void* k, int B, int H, i
   return run_smooth_quant<64>(q, k, B, H, Hkv, N, q_i8, q_scale, k_i8, k_scale, k_mean, sums, st);
 }
 
+// NVFP4 quantization launches (arguments already checked): zeroed slice maxima, maxima,
+// quantization along the channels or transposed along the rows, slice scales.
+qattn_status dispatch_quant_nvfp4(const void* x, const float* mean, int S, int R, int C,
+                                  int along_rows, uint8_t* codes, uint8_t* scales, float* gscale,
+                                  cudaStream_t st) {
+  const uint16_t* xh = static_cast<const uint16_t*>(x);
+  unsigned* amax_bits = reinterpret_cast<unsigned*>(gscale);
+  if (cudaMemsetAsync(gscale, 0, sizeof(float) * static_cast<size_t>(S), st) != cudaSuccess)
+    return QATTN_ERR_CUDA;
+  // slice maxima: about 16 resident CTAs per SM over all slices, at least 4 vectors a thread
+  const long long nvec = static_cast<long long>(R) * C / 8;
+  long long gx = (nvec + 1023) / 1024;
+  const long long cap = (148LL * 16 + S - 1) / S;
+  if (gx > cap) gx = cap;
+  if (gx < 1) gx = 1;
+  nvfp4_amax_kernel<<<dim3(static_cast<unsigned>(gx), S), 256, 0, st>>>(xh, mean, R, C, amax_bits);
+  if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
+  if (along_rows) {
+    const int Rp = (R + 127) / 128 * 128;
+    const dim3 grid((Rp + kNvfp4Tile - 1) / kNvfp4Tile, (C + kNvfp4Tile - 1) / kNvfp4Tile, S);
+    nvfp4_quant_cols_kernel<<<grid, 256, 0, st>>>(xh, mean, R, C, Rp, amax_bits, codes, scales);
+  } else {
+    const long long total = static_cast<long long>(S) * R * (C / 16);
+    long long blocks = (total + 255) / 256;
+    if (blocks > 148LL * 32) blocks = 148LL * 32;
+    nvfp4_quant_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(xh, mean, R, C, total,
+                                                                          amax_bits, codes, scales);
+  }
+  if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
+  nvfp4_finalize_kernel<<<(S + 255) / 256, 256, 0, st>>>(gscale, S);
+  return launch_status();
+}
+
+// FP4-path attention launch (arguments already checked).
+qattn_status dispatch_attn_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales, const float* q_g,
+                                 const uint8_t* k_codes, const uint8_t* k_scales, const float* k_g,
+                                 const uint8_t* vt_codes, const uint8_t* vt_scales,
+                                 const float* v_g, const void* q, const void* k, const void* v,
+                                 const float* k_mean, const int* kv_list, const int* kv_count,
+                                 void* out, int B, int H, int Hkv, int N, int d, int causal,
+                                 cudaStream_t st) {
+  const int Np = (N + 127) / 128 * 128;
+  CUtensorMap maps[6];
+  if (!make_fp4_map(&maps[0], q_codes, d, N, static_cast<long long>(B) * H) ||
+      !make_fp4_map(&maps[1], k_codes, d, N, static_cast<long long>(B) * Hkv) ||
+      !make_fp4_vt_map(&maps[2], vt_codes, d, Np, static_cast<long long>(B) * Hkv))
+    return QATTN_ERR_CUDA;
+  if (kv_list != nullptr) {
+    // fp16 Q, K, V tiles: boxes of 64 columns x 128 rows, 128-byte swizzle
+    if (!make_v_map(&maps[3], q, d, N, static_cast<long long>(B) * H) ||
+        !make_v_map(&maps[4], k, d, N, static_cast<long long>(B) * Hkv) ||
+        !make_v_map(&maps[5], v, d, N, static_cast<long long>(B) * Hkv))
+      return QATTN_ERR_CUDA;
+  } else {
+    maps[3] = maps[4] = maps[5] = maps[0];  // never read without promotion
+  }
+  const uint16_t* q16 = static_cast<const uint16_t*>(q);
+#define QATTN_FP4_ARGS maps, q_scales, k_scales, vt_scales, q_g, k_g, v_g, q16, k_mean, kv_list, \
+                       kv_count, out, B, H, Hkv, N, Np, st
+  if (d == 128)
+    return causal ? launch_attn_nvfp4<128, true>(QATTN_FP4_ARGS)
+                  : launch_attn_nvfp4<128, false>(QATTN_FP4_ARGS);
+  return causal ? launch_attn_nvfp4<64, true>(QATTN_FP4_ARGS)
+                : launch_attn_nvfp4<64, false>(QATTN_FP4_ARGS);
+#undef QATTN_FP4_ARGS
+}
+
 // ---------------------------------------------------------------------------------------------
 // Per-device memory pools for the allocating entry points
 // ---------------------------------------------------------------------------------------------
@@ -751,35 +818,78 @@ qattn_status qattn_attn_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales, c
   if (s != QATTN_OK) return s;
   s = check_ptrs(q_codes, q_scales, q_g, k_codes, k_scales, k_g, vt_codes, vt_scales, v_g, out);
   if (s != QATTN_OK) return s;
-  const bool promote = kv_list != nullptr;
-  if (promote && (s = check_ptrs(q, k, v, k_mean, kv_list, kv_count)) != QATTN_OK) return s;
+  if (kv_list != nullptr && (s = check_ptrs(q, k, v, k_mean, kv_list, kv_count)) != QATTN_OK)
+    return s;
   if (static_cast<long long>(B) * H > 65535) return QATTN_ERR_UNSUPPORTED;
   if ((s = device_ok()) != QATTN_OK) return s;
+  return dispatch_attn_nvfp4(q_codes, q_scales, q_g, k_codes, k_scales, k_g, vt_codes, vt_scales,
+                             v_g, q, k, v, k_mean, kv_list, kv_count, out, B, H, Hkv, N, d, causal,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+qattn_status qattn_forward_nvfp4(const void* q, const void* k, const void* v, void* out, int B,
+                                 int H, int Hkv, int N, int d, int causal, int topk,
+                                 qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q, k, v, out);
+  if (s != QATTN_OK) return s;
+  // topk -1: every tile in FP4; topk >= 0: the selected tiles in FP16 (non-causal topk 0 would
+  // promote nothing and is the same as -1, so it is accepted)
+  if (topk < -1) return QATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 65535) return QATTN_ERR_UNSUPPORTED;
+  if (topk >= 0 && (N + kSelKRows - 1) / kSelKRows > kSelMaxTiles) return QATTN_ERR_UNSUPPORTED;
+  if ((s = device_ok()) != QATTN_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int Np = (N + 127) / 128 * 128;
-  CUtensorMap maps[6];
-  if (!make_fp4_map(&maps[0], q_codes, d, N, static_cast<long long>(B) * H) ||
-      !make_fp4_map(&maps[1], k_codes, d, N, static_cast<long long>(B) * Hkv) ||
-      !make_fp4_vt_map(&maps[2], vt_codes, d, Np, static_cast<long long>(B) * Hkv))
-    return QATTN_ERR_CUDA;
-  if (promote) {
-    // fp16 Q, K, V tiles: boxes of 64 columns x 128 rows, 128-byte swizzle
-    if (!make_v_map(&maps[3], q, d, N, static_cast<long long>(B) * H) ||
-        !make_v_map(&maps[4], k, d, N, static_cast<long long>(B) * Hkv) ||
-        !make_v_map(&maps[5], v, d, N, static_cast<long long>(B) * Hkv))
-      return QATTN_ERR_CUDA;
-  } else {
-    maps[3] = maps[4] = maps[5] = maps[0];  // never read without promotion
+  // one stream-ordered workspace: channel sums and mean, the three NVFP4 operands, and (with
+  // promotion) the selection's scratch and tile lists
+  const size_t BH = static_cast<size_t>(B) * H, BG = static_cast<size_t>(B) * Hkv;
+  const size_t Np = (static_cast<size_t>(N) + 127) / 128 * 128;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes); return o; };
+  const size_t o_sums = take(sizeof(long long) * BG * d), o_mean = take(sizeof(float) * BG * d);
+  const size_t o_qc = take(BH * N * d / 2), o_qs = take(BH * N * d / 16), o_qg = take(4 * BH);
+  const size_t o_kc = take(BG * N * d / 2), o_ks = take(BG * N * d / 16), o_kg = take(4 * BG);
+  const size_t o_vc = take(BG * d * Np / 2), o_vs = take(BG * d * Np / 16), o_vg = take(4 * BG);
+  const SelLayout S = sel_layout(B, H, Hkv, N, d);
+  const size_t o_sel = topk >= 0 ? take(S.total) : 0;
+  const size_t o_list = topk >= 0 ? take(sizeof(int) * BH * S.nsb * S.nkt) : 0;
+  const size_t o_count = topk >= 0 ? take(sizeof(int) * BH * S.nsb) : 0;
+  void* ws = nullptr;
+  if ((s = pool_alloc(&ws, off, st)) != QATTN_OK) return s;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  long long* sums = reinterpret_cast<long long*>(w + o_sums);
+  float* mean = reinterpret_cast<float*>(w + o_mean);
+  int* kv_list = topk >= 0 ? reinterpret_cast<int*>(w + o_list) : nullptr;
+  int* kv_count = topk >= 0 ? reinterpret_cast<int*>(w + o_count) : nullptr;
+  if (cudaMemsetAsync(sums, 0, sizeof(long long) * BG * d, st) != cudaSuccess) s = QATTN_ERR_CUDA;
+  if (s == QATTN_OK) {
+    const dim3 g1(static_cast<unsigned>(BG), (N + kSumRowsPerCta - 1) / kSumRowsPerCta);
+    if (d == 128) k_channel_sums_kernel<128><<<g1, 256, 0, st>>>(static_cast<const uint16_t*>(k), N, sums);
+    else k_channel_sums_kernel<64><<<g1, 256, 0, st>>>(static_cast<const uint16_t*>(k), N, sums);
+    const int n = static_cast<int>(BG) * d;
+    k_mean_from_sums_kernel<<<(n + 255) / 256, 256, 0, st>>>(sums, N, n, mean);
+    s = launch_status();
   }
-  const uint16_t* q16 = static_cast<const uint16_t*>(q);
-#define QATTN_FP4_ARGS maps, q_scales, k_scales, vt_scales, q_g, k_g, v_g, q16, k_mean, kv_list, \
-                       kv_count, out, B, H, Hkv, N, Np, st
-  if (d == 128)
-    return causal ? launch_attn_nvfp4<128, true>(QATTN_FP4_ARGS)
-                  : launch_attn_nvfp4<128, false>(QATTN_FP4_ARGS);
-  return causal ? launch_attn_nvfp4<64, true>(QATTN_FP4_ARGS)
-                : launch_attn_nvfp4<64, false>(QATTN_FP4_ARGS);
-#undef QATTN_FP4_ARGS
+  if (s == QATTN_OK)
+    s = dispatch_quant_nvfp4(q, nullptr, static_cast<int>(BH), N, d, 0, w + o_qc, w + o_qs,
+                             reinterpret_cast<float*>(w + o_qg), st);
+  if (s == QATTN_OK)
+    s = dispatch_quant_nvfp4(k, mean, static_cast<int>(BG), N, d, 0, w + o_kc, w + o_ks,
+                             reinterpret_cast<float*>(w + o_kg), st);
+  if (s == QATTN_OK)
+    s = dispatch_quant_nvfp4(v, nullptr, static_cast<int>(BG), N, d, 1, w + o_vc, w + o_vs,
+                             reinterpret_cast<float*>(w + o_vg), st);
+  if (s == QATTN_OK && topk >= 0)
+    s = d == 128 ? run_block_select<128>(q, k, B, H, Hkv, N, causal, topk, kv_list, kv_count, w + o_sel, st)
+                 : run_block_select<64>(q, k, B, H, Hkv, N, causal, topk, kv_list, kv_count, w + o_sel, st);
+  if (s == QATTN_OK)
+    s = dispatch_attn_nvfp4(w + o_qc, w + o_qs, reinterpret_cast<float*>(w + o_qg), w + o_kc,
+                            w + o_ks, reinterpret_cast<float*>(w + o_kg), w + o_vc, w + o_vs,
+                            reinterpret_cast<float*>(w + o_vg), q, k, v, mean, kv_list, kv_count,
+                            out, B, H, Hkv, N, d, causal, st);
+  if (cudaFreeAsync(ws, st) != cudaSuccess && s == QATTN_OK) s = QATTN_ERR_CUDA;
+  return s;
 }
 
 qattn_status qattn_debug_qk_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales,
@@ -843,33 +953,8 @@ qattn_status qattn_quant_nvfp4(const void* x, const float* mean, int S, int R, i
   if (s != QATTN_OK) return s;
   if (mean && !aligned16(mean)) return QATTN_ERR_MISALIGNED;
   if ((s = device_ok()) != QATTN_OK) return s;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const uint16_t* xh = static_cast<const uint16_t*>(x);
-  unsigned* amax_bits = reinterpret_cast<unsigned*>(gscale);
-  if (cudaMemsetAsync(gscale, 0, sizeof(float) * static_cast<size_t>(S), st) != cudaSuccess)
-    return QATTN_ERR_CUDA;
-  // slice maxima: about 16 resident CTAs per SM over all slices, at least 4 vectors a thread
-  const long long nvec = static_cast<long long>(R) * C / 8;
-  long long gx = (nvec + 1023) / 1024;
-  const long long cap = (148LL * 16 + S - 1) / S;
-  if (gx > cap) gx = cap;
-  if (gx < 1) gx = 1;
-  nvfp4_amax_kernel<<<dim3(static_cast<unsigned>(gx), S), 256, 0, st>>>(xh, mean, R, C, amax_bits);
-  if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
-  if (along_rows) {
-    const int Rp = (R + 127) / 128 * 128;
-    const dim3 grid((Rp + kNvfp4Tile - 1) / kNvfp4Tile, (C + kNvfp4Tile - 1) / kNvfp4Tile, S);
-    nvfp4_quant_cols_kernel<<<grid, 256, 0, st>>>(xh, mean, R, C, Rp, amax_bits, codes, scales);
-  } else {
-    const long long total = static_cast<long long>(S) * R * (C / 16);
-    long long blocks = (total + 255) / 256;
-    if (blocks > 148LL * 32) blocks = 148LL * 32;
-    nvfp4_quant_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(xh, mean, R, C, total,
-                                                                          amax_bits, codes, scales);
-  }
-  if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
-  nvfp4_finalize_kernel<<<(S + 255) / 256, 256, 0, st>>>(gscale, S);
-  return launch_status();
+  return dispatch_quant_nvfp4(x, mean, S, R, C, along_rows, codes, scales, gscale,
+                              reinterpret_cast<cudaStream_t>(stream));
 }
 
 qattn_status qattn_check_device_status(qattn_stream_t stream) {

@@ -32,7 +32,7 @@ EXPORTS = [
     "qattn_forward_sparse",
     "qattn_forward_workspace", "qattn_forward_ws", "qattn_forward",
     "qattn_forward_host", "qattn_debug_qk_int32", "qattn_debug_wait_timeout",
-    "qattn_quant_nvfp4", "qattn_attn_nvfp4", "qattn_debug_qk_nvfp4", "qattn_check_device_status",
+    "qattn_quant_nvfp4", "qattn_attn_nvfp4", "qattn_forward_nvfp4", "qattn_debug_qk_nvfp4", "qattn_check_device_status",
 ]
 
 
@@ -100,6 +100,8 @@ def _lib():
         L.qattn_attn_nvfp4.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
                                        i, i, i, i, i, i, P]
         L.qattn_attn_nvfp4.restype = i
+        L.qattn_forward_nvfp4.argtypes = [P, P, P, P, i, i, i, i, i, i, i, P]
+        L.qattn_forward_nvfp4.restype = i
         L.qattn_debug_qk_nvfp4.argtypes = [P, P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, i, P]
         L.qattn_debug_qk_nvfp4.restype = i
         L.qattn_check_device_status.argtypes = [P]
@@ -349,6 +351,17 @@ def qattn_attn_nvfp4(q_nvfp4, k_nvfp4, vt_nvfp4, B, H, Hkv, N, d, causal=False, 
                                  _p(vg), _p(pq), _p(pk), _p(pv), _p(pm), _p(pl), _p(pc), _p(out),
                                  B, H, Hkv, N, d, int(bool(causal)), _stream(stream))
     _check("qattn_attn_nvfp4", st)
+    return out
+
+
+def qattn_forward_nvfp4(q, k, v, topk=-1, out=None, causal=False, stream=None):
+    """The FP4-path forward in one call (smoothing, NVFP4 operands, optional top-k FP16
+    promotion, attention); fp16 in, fp16 out."""
+    B, H, Hkv, N, d = _dims(q, k)
+    out = torch.empty(B, H, N, d, dtype=torch.float16, device=q.device) if out is None else out
+    st = _lib().qattn_forward_nvfp4(_p(q), _p(k), _p(v), _p(out), B, H, Hkv, N, d,
+                                    int(bool(causal)), int(topk), _stream(stream))
+    _check("qattn_forward_nvfp4", st)
     return out
 
 

@@ -265,6 +265,17 @@ qattn_status qattn_attn_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales, c
                               const int* kv_list, const int* kv_count, void* out, int B, int H,
                               int Hkv, int N, int d, int causal, qattn_stream_t stream);
 
+/* The FP4-path forward in one call, fp16 in, fp16 out: K's channel mean (exact sums, as
+ * qattn_smooth_quant), NVFP4 quantization of Q, of K minus the mean and of V along the tokens
+ * (qattn_quant_nvfp4), with topk >= 0 the key-tile selection (qattn_block_select's rule) whose
+ * tiles run in FP16, then qattn_attn_nvfp4.  topk == -1: every tile in FP4.  Results equal those
+ * of the separate calls.  The workspace comes stream-ordered from the library's per-device pool.
+ * Errors: topk < -1 QATTN_ERR_INVALID_ARG; with topk >= 0, N > 131072 QATTN_ERR_UNSUPPORTED;
+ * otherwise as qattn_attn_nvfp4. */
+qattn_status qattn_forward_nvfp4(const void* q, const void* k, const void* v, void* out, int B,
+                                 int H, int Hkv, int N, int d, int causal, int topk,
+                                 qattn_stream_t stream);
+
 /* ------------------------------------------------------------------------------------------
  * Checks.
  * ------------------------------------------------------------------------------------------ */

@@ -158,3 +158,16 @@ def test_attn_nvfp4_argument_checks():
     # promotion: lists given, an fp16 operand or the mean missing / misaligned
     assert L.qattn_attn_nvfp4(*a, None, *prom[1:], o, 1, 4, 2, 256, 128, 1, None) == 1
     assert L.qattn_attn_nvfp4(*a, *prom[:3], P(20), *prom[4:], o, 1, 4, 2, 256, 128, 1, None) == 3
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((None, P(32), P(48), P(64), 1, 4, 2, 256, 128, 1, 4, None), 1),     # null pointer
+    ((P(16), P(32), P(48), P(64), 1, 4, 3, 256, 128, 1, 4, None), 1),    # H % Hkv != 0
+    ((P(16), P(32), P(48), P(64), 1, 4, 2, 256, 128, 1, -2, None), 1),   # topk < -1
+    ((P(16), P(32), P(48), P(64), 1, 4, 2, 256, 96, 1, 4, None), 2),     # d
+    ((P(16), P(32), P(48), P(64), 1, 4, 2, 131073, 128, 1, 4, None), 2), # selection limit
+    ((P(16), P(33), P(48), P(64), 1, 4, 2, 256, 128, 1, -1, None), 3),   # misaligned
+])
+def test_forward_nvfp4_argument_checks(args, expect):
+    L = Q.load()
+    assert L.qattn_forward_nvfp4(*args) == expect

@@ -423,3 +423,29 @@ def test_attn_nvfp4_promoted_full_size_sampled_rows(lib, oracle):
                                         q16=qh, k16=kh, v16=vh, k_mean=mean[g:g + 1])
     got = out[0, h, torch.from_numpy(rows_i).cuda()].float().cpu().numpy()
     _check_fp4_out(got, ref, slack, "llama8b_32k promoted full")
+
+
+@pytest.mark.parametrize("name,over,topk", [("llama8b_32k", {"H": 4, "Hkv": 2, "N": 700}, 2),
+                                            ("tiny", {"N": 300}, -1),
+                                            ("wide64", {"B": 2, "H": 2, "Hkv": 1, "N": 400,
+                                                        "causal": True}, 0)])
+def test_forward_nvfp4_one_call_equals_the_separate_calls(lib, oracle, name, over, topk):
+    """qattn_forward_nvfp4 = channel mean + three quantizations + selection + attention, bit for
+    bit; its mean is the oracle's exact channel mean."""
+    w = WORKLOADS[name].with_(**over)
+    q, k, v = (t.cuda() for t in make_inputs(w, device="cpu"))
+    one = lib.qattn_forward_nvfp4(q, k, v, topk, causal=w.causal)
+    sums = oracle.k_channel_sums(np16(k), w.B, w.Hkv, w.N, w.d)
+    mean = torch.from_numpy(np.array([oracle.lib().oracle_mean_from_sum(int(s), w.N)
+                                      for s in sums.ravel()], dtype=np.float32)
+                            .reshape(w.B * w.Hkv, w.d)).cuda()
+    qn = lib.qattn_quant_nvfp4(q.reshape(w.B * w.H, w.N, w.d))
+    kn = lib.qattn_quant_nvfp4(k.reshape(w.B * w.Hkv, w.N, w.d), mean)
+    vn = lib.qattn_quant_nvfp4(v.reshape(w.B * w.Hkv, w.N, w.d), along_rows=True)
+    prom = None
+    if topk >= 0:
+        gl, gc = lib.qattn_block_select(q, k, topk, causal=w.causal)
+        prom = (q, k, v, mean, gl, gc)
+    sep = lib.qattn_attn_nvfp4(qn, kn, vn, w.B, w.H, w.Hkv, w.N, w.d, causal=w.causal, promote=prom)
+    assert lib.qattn_check_device_status() == 0
+    assert torch.equal(one.view(torch.int16), sep.view(torch.int16))
