@@ -384,3 +384,19 @@ def test_attention_nvfp4_mixed_tiles_use_one_softmax(oracle):
     wrong, _ = oracle.attention_nvfp4(qn, kn, vn, 1, H, 1, N, d, True, promote=half, q16=q, k16=k,
                                       v16=v, k_mean=np.zeros_like(mean))
     assert np.abs(wrong - ref).mean() > 2 * e_fp4
+
+
+def test_nvfp4_hand_derived_example(oracle):
+    """tests/golden/nvfp4_two_blocks.json: two 16-value blocks whose codes, scale bytes and packed
+    bytes were derived by hand from the format definitions (derivation inside the file)."""
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "nvfp4_two_blocks.json")
+    doc = json.load(open(path))
+    x = np.array(doc["input"]["values"], dtype=np.float16).reshape(doc["input"]["shape"])
+    codes, scales, g = oracle.quant_nvfp4(x)
+    exp = doc["expected"]
+    assert list(codes.ravel()) == exp["code_bytes"]
+    assert list(scales.ravel()) == exp["scale_bytes"]
+    assert g[0] == np.float32(7) / np.float32(2688)
+    assert list(_unpack(codes).ravel()) == exp["codes_per_element"]
