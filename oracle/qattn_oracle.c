@@ -4,6 +4,11 @@
  * ("SAGEATTENTION: accurate 8-bit attention for plug-and-play inference acceleration",
  * aibr.jp/archives/102657).
  *
+ * The file also holds, each in its own section further down, the oracle's parts for the
+ * ThriftAttention page ("ThriftAttention: Selective Mixed Precision for Long-Context FP4
+ * Attention", gist.science/ja/paper/2605.23081, method section): the block-mean key-tile
+ * selection, NVFP4 quantization, and the FP4-path attention with FP16 promotion.
+ *
  * TEST INFRASTRUCTURE ONLY.  Only the test suite, the package's smoke check and the CPU-baseline leg
  * of the benchmark may load this library.  The product path (the CUDA library) never calls it and
  * shares no code, header, table or helper with it.

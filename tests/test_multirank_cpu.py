@@ -90,3 +90,12 @@ def test_reference_arm_prints_on_rank_zero_only():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["config"]["workload"] == "tiny" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_bench_modes_parse():
+    """The FP4-path mode is selected by --fp4-topk (-1: all FP4); omitted, the INT8 path."""
+    import bench
+    assert bench.parse_args([]).fp4_topk is None
+    assert bench.parse_args(["--fp4-topk", "16"]).fp4_topk == 16
+    assert bench.parse_args(["--fp4-topk", "-1"]).fp4_topk == -1
+    assert bench.parse_args(["--sparse-topk", "8"]).sparse_topk == 8
