@@ -171,3 +171,15 @@ def test_attn_nvfp4_argument_checks():
 def test_forward_nvfp4_argument_checks(args, expect):
     L = Q.load()
     assert L.qattn_forward_nvfp4(*args) == expect
+
+
+def test_binding_argument_counts_match_the_header():
+    """Every declaration in include/qattn.h has as many parameters as the binding passes."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    L = Q.load()
+    decls = re.findall(r"\b(qattn_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", text)
+    assert len(decls) >= len(Q.EXPORTS) - 1
+    for name, params in decls:
+        params = params.strip()
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        assert len(getattr(L, name).argtypes) == n, name
