@@ -1,13 +1,16 @@
-"""NVFP4 quantization on the GPU against the oracle (FP4 path of the ThriftAttention page, method
-section; the format per NVIDIA's definition: E2M1 codes, E4M3 scale per 16 values, binary32
-scale per slice).
+"""The FP4 path of the ThriftAttention page (method section) on the GPU against the oracle.
 
-Codes, block scales and slice scales are integer / bit-pattern results of the same binary32
-operations on both sides, so every byte and every float is compared exactly: small ragged cases
-of both block directions with and without a channel mean, the degenerate cases (all-zero slice,
-blocks whose scale rounds to 0, fp16 subnormals, a single row), the workload generator's Q, K
-(smoothed with the oracle's channel means) and V, and at full size (Q, K, V of the 32K-token
-Llama-8B-shaped workload, the launch shapes a full-size FP4 path would use) sampled slices.
+- NVFP4 quantization (E2M1 codes, E4M3 scale per 16 values, binary32 scale per slice; the format
+  per NVIDIA's definition): codes, block scales and slice scales are results of the same binary32
+  operations on both sides, so every byte and float is compared exactly.  Covered: small ragged
+  cases of both block directions with and without a channel mean, the degenerate cases (all-zero
+  slice, blocks whose scale rounds to 0, fp16 subnormals, a single row), the workload generator's
+  Q, smoothed K and V, and sampled slices at 32K tokens.
+- FP4 score tiles on the block-scaled tensor cores: within 2^-20 of the magnitude sum.
+- The FP4-path attention (two-level FP4 P, online merge), with and without FP16 promotion of the
+  block-mean top-k key tiles: within the INT8 path's output bar of the oracle (plus the oracle's
+  per-row slack for FP4 decisions within 2^-16 of a tie), a one-hot closed form, sampled rows at
+  32K tokens; the one-call forward equals the separate calls bit for bit.
 """
 import numpy as np
 import pytest
