@@ -1,7 +1,8 @@
-// fp4_sm100.cuh -- FP4 scores on the block-scaled tensor cores: the Q K^T product of the FP4 path
-// of the ThriftAttention page ("ThriftAttention: Selective Mixed Precision for Long-Context FP4
-// Attention", gist.science/ja/paper/2605.23081, method section, "FP4 path": blocks computed in
-// FP4 with the NVFP4 micro-scaling format on Blackwell's native FP4 tensor cores).
+// fp4_sm100.cuh -- the FP4 path of the ThriftAttention page ("ThriftAttention: Selective Mixed
+// Precision for Long-Context FP4 Attention", gist.science/ja/paper/2605.23081, method section,
+// "FP4 path": blocks computed in FP4 with the NVFP4 micro-scaling format on Blackwell's native FP4
+// tensor cores) on the block-scaled tensor cores: FP4 score tiles (qk_nvfp4_kernel) and the
+// attention with FP16 promotion of selected key tiles (attn_nvfp4_kernel, further down).
 //
 // Operands are NVFP4 as qattn_quant_nvfp4 writes them along the channels: E2M1 codes packed two
 // per byte (rows of d/2 bytes) and one E4M3 scale byte per 16 channels (rows of d/16 bytes).
