@@ -7,7 +7,9 @@ tcgen05 attention kernel, all through the C ABI (qattn_smooth_quant then qattn_a
 the two halves of qattn_forward_ws, timed separately with CUDA events on the launching stream).
 
 Metric: TOPS = 4*B*H*N^2*d / t, halved for causal; also reported as a fraction of the B200 INT8
-tensor peak (the measured bf16 GEMM peak x 2, the nominal INT8:BF16 ratio).
+tensor peak, measured in the same run with an int8 cuBLAS GEMM (torch._int_mm, 8192^3), beside the
+datasheet's 4.5 POPS.  The long-context workload (long128k) is timed after the main one and
+reported in the same line under "workloads".
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 Multi-GPU (weak scaling, one full workload per rank, no data-path collective):
@@ -49,6 +51,13 @@ def parse_args(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="target CPU time of the oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--extra-workloads", default="long128k",
+                   help="comma-separated workloads timed after the main one and reported under "
+                        "'workloads' in the same JSON line (empty: none)")
+    p.add_argument("--extra-steps", type=int, default=10)
+    p.add_argument("--no-gemm-peaks", dest="gemm_peaks", action="store_false",
+                   help="skip the int8/fp16 GEMM peak measurement (roofline then uses "
+                        "MEASURED_PEAKS.json's bf16 figure and the nominal INT8 ratio)")
     p.add_argument("--sparse-topk", type=int, default=-1,
                    help="block-sparse mode: key tiles per 256-row query block chosen by the "
                         "block-mean score (top-k plus the causal diagonals); -1 = dense")
@@ -230,28 +239,75 @@ def weak_scaling_tops(ops_per_step: float, steps: int, world: int, max_ms: float
     return world * ops_per_step * steps / (max_ms / 1e3) / 1e12
 
 
-def run_ours(args):
+def measure_gemm_peaks(device, seconds=2.0):
+    """Tensor-core GEMM peaks on this GPU through torch (cuBLAS): int8 x int8 -> int32
+    (torch._int_mm) and fp16 x fp16 -> fp16, both 8192^3 (2 * 8192^3 operations), as a burst (best
+    of 10 single calls, CUDA events) and sustained (back-to-back calls for `seconds`).  Returns a
+    dict in TOPS; a GEMM that torch cannot run on this device is left out."""
     import torch
-    import torch.distributed as dist
-    from bit_quantized_attention_smoothing_b200 import qattn as Q
-    from bit_quantized_attention_smoothing_b200.workloads import WORKLOADS, make_inputs
+    n = 8192
+    ops = 2.0 * n ** 3
+    out = {}
+    gen = torch.Generator(device=device).manual_seed(5)
+    for name, make, fn in (
+            # B column-major (a transposed view), so both operands are K-contiguous
+            ("int8", lambda: torch.randint(-127, 128, (n, n), generator=gen, device=device, dtype=torch.int8),
+             lambda a, b: torch._int_mm(a, b.t())),
+            ("fp16", lambda: torch.randn(n, n, generator=gen, device=device, dtype=torch.float16),
+             lambda a, b: a @ b)):
+        try:
+            a, b = make(), make()
+            for _ in range(3):
+                fn(a, b)
+            torch.cuda.synchronize(device)
+            best = float("inf")
+            for _ in range(10):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn(a, b)
+                e1.record()
+                e1.synchronize()
+                best = min(best, e0.elapsed_time(e1))
+            reps = max(10, int(seconds * 1e3 / best))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                fn(a, b)
+            e1.record()
+            e1.synchronize()
+            out[name] = {"burst": ops / (best / 1e3) / 1e12,
+                         "sustained": ops * reps / (e0.elapsed_time(e1) / 1e3) / 1e12}
+            del a, b
+        except (RuntimeError, TypeError) as exc:   # no such GEMM for this device
+            out[name + "_error"] = str(exc).splitlines()[0][:160]
+    torch.cuda.empty_cache()
+    return out
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+def tensor_peaks(measured):
+    """(P8, P16, source text): the INT8 and FP16 dense peaks for the roofline (burst figures: the
+    attention kernel is timed as its own launches and stays at the maximum SM clock)."""
+    peaks, peak_src = load_peaks()
+    tag = "of measured" if peak_src == "measured" else "of fallback"
+    bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    if "fp16" in measured:
+        p16, s16 = measured["fp16"]["burst"], "fp16 GEMM measured in this run (torch, cuBLAS, 8192^3)"
+    else:
+        p16, s16 = bf16, f"bf16 GEMM burst {bf16:.1f} TF/s ({tag}; fp16 has the same nominal rate)"
+    if "int8" in measured:
+        p8, s8 = measured["int8"]["burst"], "int8 GEMM measured in this run (torch._int_mm, cuBLAS, 8192^3)"
+    else:
+        p8, s8 = 2.0 * bf16, f"2 x bf16 GEMM burst ({tag}; nominal INT8:BF16 ratio 4.5:2.25)"
+    return p8, p16, f"P8: {s8}; P16: {s16}"
 
-    w = WORKLOADS[args.workload]
-    Q.load()
-    q, k, v = make_inputs(w, device="cuda")
+
+def run_workload(Q, w, args, steps, warmup, e2e_steps, stream, world, barrier, clock_dev):
+    """Times the dense (or block-sparse) INT8 path on workload w: `steps` steps on device-resident
+    inputs (smoothing + quantization, then attention, CUDA events around each half), then
+    `e2e_steps` calls of qattn_forward_host on pinned host buffers.  Returns a dict of
+    measurements (the slowest rank's times)."""
+    import torch
+    q, k, v = make_inputs_cuda(w)
     B, H, Hkv, N, d = w.B, w.H, w.Hkv, w.N, w.d
     nqb, nkb = -(-N // 128), -(-N // 64)
     dev = q.device
@@ -261,10 +317,10 @@ def run_ours(args):
     k_s = torch.empty(B, Hkv, nkb, dtype=torch.float32, device=dev)
     ws = torch.empty(Q.qattn_smooth_quant_workspace(B, Hkv, d), dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
-    stream = torch.cuda.current_stream()
     working_set = sum(t.numel() * t.element_size() for t in (q, k, v, q_i8, k_i8, out))
 
     sparse = args.sparse_topk >= 0
+    density = 1.0
     if sparse:
         # block-sparse mode: the selection runs with the pre-processing, every step
         kl, kc = Q.qattn_block_select(q, k, args.sparse_topk, w.causal, stream=stream)
@@ -296,19 +352,18 @@ def run_ours(args):
         else:
             Q.qattn_attn_quantized(q_i8, q_s, k_i8, k_s, v, out, w.causal, stream)
 
-    for _ in range(max(3, args.warmup)):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     if Q.qattn_check_device_status(stream) != 0:
         raise RuntimeError("device status reports a timed-out wait during warm-up")
 
-    K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        for i in range(K):
+    with ClockSampler(clock_dev) as clk:
+        for i in range(steps):
             ev[i][0].record(stream)
             step(ev[i][1])
             ev[i][2].record(stream)
@@ -319,16 +374,13 @@ def run_ours(args):
     quant_ms = [e[0].elapsed_time(e[1]) for e in ev]
     if Q.qattn_check_device_status(stream) != 0:
         raise RuntimeError("device status reports a timed-out wait in the timed region")
-
     total_ms_max = max_over_ranks(total_ms, world, dev)
-    ops = w.ops
-    value = weak_scaling_tops(ops, K, world, total_ms_max)
 
     # end to end through the C ABI on host buffers (H2D of q, k, v and D2H of out inside)
     qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
     oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
     Q.qattn_forward_host(qh, kh, vh, oh, w.causal, stream)  # warm-up (pool, tensor maps)
-    ke = max(1, args.e2e_steps)
+    ke = max(1, e2e_steps)
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -338,50 +390,35 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    e2e_value = weak_scaling_tops(ops, ke, world, e2e_ms)
-    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
-    d2h = oh.numel() * oh.element_size()
+    return {
+        "q": q, "k": k, "v": v, "working_set": working_set, "sparse": sparse, "density": density,
+        "total_ms_max": total_ms_max, "attn_ms": statistics.mean(attn_ms),
+        "quant_ms": statistics.mean(quant_ms), "clocks": clk.summary(), "e2e_ms": e2e_ms,
+        "e2e_steps": ke, "h2d": sum(t.numel() * t.element_size() for t in (qh, kh, vh)),
+        "d2h": oh.numel() * oh.element_size(),
+        "launches_per_step": 3 + (4 if sparse else 0),
+    }
 
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank != 0:
-        return None
 
-    peaks, peak_src = load_peaks()
-    bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    int8_peak = 2.0 * bf16                       # nominal INT8:BF16 dense ratio 4.5:2.25
-    mixed_peak = 2.0 / (1.0 / int8_peak + 1.0 / bf16)   # half the ops INT8, half FP16
-    attn_avg_ms = statistics.mean(attn_ms)
+def make_inputs_cuda(w):
+    from bit_quantized_attention_smoothing_b200.workloads import make_inputs
+    return make_inputs(w, device="cuda")
+
+
+def workload_line(w, r, steps, world, p8, p16, peak_src):
+    """The measured numbers of one workload: value, roofline of the attention kernel, e2e."""
+    ops = w.ops
+    value = weak_scaling_tops(ops, steps, world, r["total_ms_max"])
+    mixed_peak = 2.0 / (1.0 / p8 + 1.0 / p16)   # half the metric's ops INT8, half FP16
     # the roofline counts the work the kernel does: in block-sparse mode only the computed tiles
-    achieved = (ops * density if sparse else ops) / (attn_avg_ms / 1e3) / 1e12
-    clocks = clk.summary()
-    line = {
-        "metric": METRIC,
+    achieved = ops * r["density"] / (r["attn_ms"] / 1e3) / 1e12
+    return {
         "value": round(value, 2),
-        "unit": "TOPS",
-        "n_gpus": world,
-        "steps": K,
-        "warmup": max(3, args.warmup),
-        "ms_per_step": round(total_ms_max / K, 4),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "s8xs8->s32 (QK^T), f16xf16->f32 (PV)",
-        "data": "synthetic",
-        "config": {"workload": w.name, "B": B, "H": H, "Hkv": Hkv, "N": N, "d": d,
-                   "causal": w.causal, "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
-                   "l2": f"inputs larger than L2: working set {working_set / 2**20:.0f} MiB "
-                         f"vs 126 MiB L2, no flush"},
-        "value_frac_of_int8_peak": round(value / int8_peak, 4),
-        "attn_ms": round(attn_avg_ms, 4),
-        "quant_ms": round(statistics.mean(quant_ms), 4),
-        **({"sparse": {"topk": args.sparse_topk, "density": round(density, 4),
-                       "selection": "per 256-row query block: causal diagonal tiles plus the "
-                                    "topk 128-key tiles by block-mean score",
-                       "note": "value counts the metric's dense operation count; "
-                               "roofline.achieved counts the computed tiles only"}}
-           if sparse else {}),
+        "ms_per_step": round(r["total_ms_max"] / steps, 4),
+        "steps": steps,
+        "value_frac_of_int8_peak": round(value / p8, 4),
+        "attn_ms": round(r["attn_ms"], 4),
+        "quant_ms": round(r["quant_ms"], 4),
         "roofline": {
             "bound": "tensor",
             "kernel": "attn_fwd_kernel",
@@ -390,19 +427,116 @@ def run_ours(args):
             "unit": "TFLOP/s",
             "frac": round(achieved / mixed_peak, 4),
             "traffic": profiled_traffic(w.name),
-            "peak_source": (f"{peak_src} bf16 GEMM burst {bf16:.1f} TF/s; INT8 = 2x; mixed "
-                            f"INT8/FP16 ceiling 2/(1/P8+1/P16) since half the ops run at each "
-                            f"rate ({'of measured' if peak_src == 'measured' else 'of fallback'})"),
-            "frac_of_int8_peak": round(achieved / int8_peak, 4),
+            "peak_source": ("mixed INT8/FP16 ceiling 2/(1/P8+1/P16), since half the metric's "
+                            "operations run at each rate; " + peak_src),
+            "frac_of_int8_peak": round(achieved / p8, 4),
+            "frac_of_int8_datasheet": round(achieved / 4500.0, 4),
         },
-        "e2e": {"value": round(e2e_value, 2), "unit": "TOPS", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": ke,
+        "e2e": {"value": round(weak_scaling_tops(ops, r["e2e_steps"], world, r["e2e_ms"]), 2),
+                "unit": "TOPS", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                "steps": r["e2e_steps"],
                 "api": "qattn_forward_host (host fp16 buffers; copies, workspace and kernels inside)"},
-        "gpu_launches": 3 * K,
-        "clocks": clocks,
+        "clocks": r["clocks"],
     }
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_sample_run(w, q, k, v, args.cpu_seconds)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from bit_quantized_attention_smoothing_b200 import qattn as Q
+    from bit_quantized_attention_smoothing_b200.workloads import WORKLOADS
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    Q.load()
+    stream = torch.cuda.current_stream()
+    warmup = max(3, args.warmup)
+    w = WORKLOADS[args.workload]
+    r = run_workload(Q, w, args, args.steps, warmup, args.e2e_steps, stream, world, barrier, local)
+    q, k, v = r.pop("q"), r.pop("k"), r.pop("v")
+    cpu_base = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cpu_base = oracle_sample_run(w, q, k, v, args.cpu_seconds)
+    del q, k, v
+    torch.cuda.empty_cache()
+    extra = {}
+    for name in [x for x in args.extra_workloads.split(",") if x and x != w.name]:
+        we = WORKLOADS[name]
+        re_ = run_workload(Q, we, args, args.extra_steps, warmup, max(1, min(args.e2e_steps, 3)),
+                           stream, world, barrier, local)
+        for key in ("q", "k", "v"):
+            re_.pop(key)
+        extra[name] = (we, re_)
+        torch.cuda.empty_cache()
+    measured = measure_gemm_peaks(torch.device("cuda", local)) if args.gemm_peaks else {}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    p8, p16, peak_src = tensor_peaks(measured)
+    main = workload_line(w, r, args.steps, world, p8, p16, peak_src)
+    line = {
+        "metric": METRIC,
+        "value": main["value"],
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": warmup,
+        "ms_per_step": main["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "s8xs8->s32 (QK^T), f16xf16->f32 (PV)",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                   "causal": w.causal, "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "l2": f"inputs larger than L2: working set {r['working_set'] / 2**20:.0f} MiB "
+                         f"vs 126 MiB L2, no flush"},
+        "value_frac_of_int8_peak": main["value_frac_of_int8_peak"],
+        "attn_ms": main["attn_ms"],
+        "quant_ms": main["quant_ms"],
+        **({"sparse": {"topk": args.sparse_topk, "density": round(r["density"], 4),
+                       "selection": "per 256-row query block: causal diagonal tiles plus the "
+                                    "topk 128-key tiles by block-mean score",
+                       "note": "value counts the metric's dense operation count; "
+                               "roofline.achieved counts the computed tiles only"}}
+           if r["sparse"] else {}),
+        "roofline": main["roofline"],
+        "e2e": main["e2e"],
+        "gpu_launches": r["launches_per_step"] * args.steps,
+        "clocks": main["clocks"],
+        "tensor_peaks_tops": {
+            "int8_used": round(p8, 1), "fp16_used": round(p16, 1),
+            "int8_datasheet_dense": 4500.0, "fp16_datasheet_dense": 2250.0,
+            **{f"{kk}_{m}": round(vv[m], 1) for kk, vv in measured.items() if isinstance(vv, dict)
+               for m in ("burst", "sustained")},
+            **{kk: vv for kk, vv in measured.items() if not isinstance(vv, dict)}},
+    }
+    if extra:
+        line["workloads"] = {}
+        for name, (we, re_) in extra.items():
+            wl = workload_line(we, re_, args.extra_steps, world, p8, p16, peak_src)
+            wl["config"] = {"B": we.B, "H": we.H, "Hkv": we.Hkv, "N": we.N, "d": we.d,
+                            "causal": we.causal,
+                            "l2": f"working set {re_['working_set'] / 2**20:.0f} MiB, no flush"}
+            wl["gpu_launches"] = re_["launches_per_step"] * args.extra_steps
+            line["workloads"][name] = wl
+    if cpu_base is not None:
+        line["cpu_baseline"] = cpu_base
     return line
 
 
@@ -679,7 +813,12 @@ def run_reference(args):
         "dtype": "s8xs8->s32, f64",
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "N": w.N, "d": w.d,
-                   "causal": w.causal},
+                   "causal": w.causal,
+                   "parallelism": (f"replicas x{os.environ.get('WORLD_SIZE')}"
+                                   if int(os.environ.get("WORLD_SIZE", "1")) > 1 else "1 GPU"),
+                   "l2": f"inputs larger than L2: working set "
+                         f"{(2 * w.B * (w.H + 2 * w.Hkv) * w.N * w.d + w.B * (w.H + w.Hkv) * w.N * w.d + 2 * w.B * w.H * w.N * w.d) / 2**20:.0f} "
+                         f"MiB vs 126 MiB L2, no flush"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": r["cores"],
                          "kind": "oracle", "sample": r["sample"]},
         "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,

@@ -364,18 +364,27 @@ __device__ __forceinline__ void setmaxnreg_dec56() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
 }
 
+// Score-tile dump of the DUMP instantiation: the CTAs of query head bh, pairs pair0 .. (one per
+// block), store the raw int32 scores each softmax thread loads from tensor memory for query tiles
+// qt0 .. qt0+nqt-1 and key tiles kt0 .. kt0+nkt-1 into s_out [nqt*128][ld] (row-major).
+struct ScoreDump {
+  int32_t* s_out;
+  int ld, bh, pair0, qt0, nqt, kt0, nkt;
+};
+
 // QF16: Q arrives as fp16 (q16) and the softmax warps quantize their own Q tile into shared
 // memory before the first QK^T (per-tile amax, scale = amax / 127, the same rounding as
 // quantize_kernel); otherwise int8 Q and its scales come from the smoothing + quantization pass
-// (tm_q, q_scale).
-template <int D, bool CAUSAL, bool QF16>
+// (tm_q, q_scale).  DUMP: the same kernel, which also writes the int32 score tiles it reads (the
+// exactness check of Q K^T); only its block-to-work mapping differs (see ScoreDump).
+template <int D, bool CAUSAL, bool QF16, bool DUMP = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scale,
                     const uint16_t* __restrict__ q16, const int* __restrict__ kv_list,
                     const int* __restrict__ kv_count,
                     const float* __restrict__ k_scale, __half* __restrict__ out, int B, int H,
-                    int Hkv, int N, float scale_log2) {
+                    int Hkv, int N, float scale_log2, ScoreDump dump) {
   using Cfg = AttnCfg<D>;
   constexpr int ST = Cfg::kStages;
   constexpr int kTmaWarp = kSoftmaxThreads / 32;  // warp 8
@@ -399,9 +408,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // they read is shared by the heads of a kv head and stays in L2).  Non-causal: every CTA reads
   // its head's whole K/V, so the pairs of one head run together and reuse it from L2 (all heads at
   // once would need every head's K/V resident).
-  const int pair = CAUSAL ? npairs - 1 - static_cast<int>(blockIdx.x / BH)
+  const int pair = DUMP ? dump.pair0 + static_cast<int>(blockIdx.x)
+                 : CAUSAL ? npairs - 1 - static_cast<int>(blockIdx.x / BH)
                           : static_cast<int>(blockIdx.x % npairs);
-  const int bh = CAUSAL ? static_cast<int>(blockIdx.x % BH) : static_cast<int>(blockIdx.x / npairs);
+  const int bh = DUMP ? dump.bh
+                 : CAUSAL ? static_cast<int>(blockIdx.x % BH) : static_cast<int>(blockIdx.x / npairs);
   const int b = bh / H;
   const int h = bh % H;
   const int g = h / (H / Hkv);
@@ -489,12 +500,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t dq0 = smem_desc(smem_u32(smem + Cfg::kOffQ), 16, Cfg::kSboQK, Cfg::kSwQK);
       const uint64_t dk0 = smem_desc(smem_u32(smem + Cfg::kOffK), 16, Cfg::kSboQK, Cfg::kSwQK);
       const uint64_t dv0 = smem_desc(smem_u32(smem + Cfg::kOffV), Cfg::kVBox, 1024, kSwizzle128B);
-      bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->q_full, 0, abort) && mbar_wait(&bars->kv_full[0], 0, abort));
+      // a CTA whose lists hold no key tile (n_kv == 0: block-sparse lists with zero entries) has
+      // nothing to multiply; its softmax warps write zero rows
+      bool ok = n_kv > 0 &&
+                __all_sync(0xFFFFFFFFu, mbar_wait(&bars->q_full, 0, abort) && mbar_wait(&bars->kv_full[0], 0, abort));
       tc_fence_after();
       if (ok) {
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
-          if (w == 1 && nw1 == 0) break;
+          if ((w == 0 ? nw0 : nw1) == 0) continue;  // a tile without key tiles waits on no score
           const uint64_t da = dq0 + static_cast<uint64_t>((w * Cfg::kQTile) >> 4);
           mma_i8_ss_warp(tmem + w * 128, da, dk0, idq, 0u);
 #pragma unroll
@@ -603,6 +617,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int c = 0; c < 4; ++c) tmem_ld32(s_tm + c * 32, sr[c]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld_wait(sr[c]);
+        if constexpr (DUMP) {
+          if (t >= dump.qt0 && t < dump.qt0 + dump.nqt && kt >= dump.kt0 && kt < dump.kt0 + dump.nkt) {
+            int4* dst = reinterpret_cast<int4*>(dump.s_out + static_cast<size_t>((t - dump.qt0) * kBM + row) * dump.ld +
+                                                (kt - dump.kt0) * kBN);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; e += 4)
+                dst[c * 8 + e / 4] = make_int4(static_cast<int>(sr[c][e]), static_cast<int>(sr[c][e + 1]),
+                                               static_cast<int>(sr[c][e + 2]), static_cast<int>(sr[c][e + 3]));
+          }
+        }
         int lim = N - 1 - kt * kBN;
         if (CAUSAL && kt == t) lim = min(lim, row);
         const float c0 = sq * ks0 * scale_log2;
@@ -659,6 +685,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
       }
+    } else {
+      // no key tile for this Q tile (an empty block-sparse list): the softmax over no keys is
+      // empty, and its rows are written as zeros
+      const int qrow = (wt == 0 ? tq0 : tq1) * kBM + row;
+      if ((wt == 0 || has1) && qrow < N) {
+        uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + qrow) * D);
+#pragma unroll
+        for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0, 0, 0, 0);
+      }
     }
   }
 
@@ -668,88 +703,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
-  }
-}
-
-// ------------------------------------------------------------------------------------------------
-// int32 score tiles through the same TMA -> tcgen05.mma kind::i8 -> TMEM -> tcgen05.ld path.
-// grid (nqt, nkt), 128 threads; each CTA computes one 128x128 tile of S_int = Q_i8 K_i8^T.
-// ------------------------------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(128, 1)
-    qk_int32_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    int32_t* __restrict__ s_out, int bh, int bg, int qt0, int kt0, int ldo) {
-  using Cfg = AttnCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  uint8_t* sq = smem;
-  uint8_t* sk = smem + Cfg::kQTile;
-  uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + Cfg::kQTile + Cfg::kKTile);
-  uint64_t* bar_mma = bar_ld + 1;
-  uint32_t* tbase = reinterpret_cast<uint32_t*>(bar_ld + 2);
-  volatile int* abort = reinterpret_cast<volatile int*>(bar_ld + 3);
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int qt = qt0 + blockIdx.x;
-  const int kt = kt0 + blockIdx.y;
-  if (threadIdx.x == 0) {
-    mbar_init(bar_ld, 1);
-    mbar_init(bar_mma, 1);
-    *abort = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(tbase, 128);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tbase;
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(bar_ld, Cfg::kQTile + Cfg::kKTile);
-    tma_load_3d(sq, &tm_q, bar_ld, 0, qt * kBM, bh);
-    tma_load_3d(sk, &tm_k, bar_ld, 0, kt * kBN, bg);
-    if (mbar_wait(bar_ld, 0, abort)) {
-      tc_fence_after();
-      constexpr uint32_t idq = idesc_i8_s32(kBM, kBN);
-#pragma unroll
-      for (int kk = 0; kk < D / 32; ++kk) {
-        const uint64_t ad = smem_desc(smem_u32(sq) + kk * 32, 16, Cfg::kSboQK, Cfg::kSwQK);
-        const uint64_t bd = smem_desc(smem_u32(sk) + kk * 32, 16, Cfg::kSboQK, Cfg::kSwQK);
-        mma_i8_ss(tmem, ad, bd, idq, kk > 0 ? 1u : 0u);
-      }
-      mma_commit(bar_mma);
-    }
-  }
-  __syncwarp();
-  const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar_mma, 0, abort));
-  tc_fence_after();
-  if (ok) {
-    // the 16x256b load shape the attention softmax uses: two loads per warp (lanes +0, +16)
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int lane_base = warp * 32 + hh * 16;
-      uint32_t r[64];
-      tmem_ld16x256b_x16(tmem + (static_cast<uint32_t>(lane_base) << 16), r);
-      tmem_ld_wait(r);
-      const int rA = lane_base + (lane >> 2);
-      int32_t* oA = s_out + static_cast<size_t>(blockIdx.x * kBM + rA) * ldo + blockIdx.y * kBN + 2 * (lane & 3);
-      int32_t* oB = oA + static_cast<size_t>(8) * ldo;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        *reinterpret_cast<uint2*>(oA + 8 * i) = make_uint2(r[4 * i + 0], r[4 * i + 1]);
-        *reinterpret_cast<uint2*>(oB + 8 * i) = make_uint2(r[4 * i + 2], r[4 * i + 3]);
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, 128);
   }
 }
 

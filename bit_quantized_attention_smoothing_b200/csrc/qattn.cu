@@ -192,12 +192,14 @@ qattn_status run_smooth_quant(const void* q, const void* k, int B, int H, int Hk
   return launch_status();
 }
 
-// q is int8 (with q_scale) or, for QF16, the fp16 Q that the kernel quantizes itself.
-template <int D, bool CAUSAL, bool QF16>
+// q is int8 (with q_scale) or, for QF16, the fp16 Q that the kernel quantizes itself.  DUMP:
+// the score-dumping instantiation, one CTA per Q-tile pair dump->pair0 .. of head dump->bh.
+template <int D, bool CAUSAL, bool QF16, bool DUMP = false>
 qattn_status run_attn(const void* q, const float* q_scale, const int8_t* k_i8,
                       const float* k_scale, const void* v, void* out, int B, int H, int Hkv,
                       int N, cudaStream_t st, const int* kv_list = nullptr,
-                      const int* kv_count = nullptr) {
+                      const int* kv_count = nullptr, const ScoreDump* dump = nullptr,
+                      int dump_pairs = 0) {
   CUtensorMap tq, tk, tv;
   std::memset(&tq, 0, sizeof(tq));  // unused by the QF16 kernel
   if ((!QF16 && !make_i8_map(&tq, q, D, N, static_cast<long long>(B) * H)) ||
@@ -205,7 +207,7 @@ qattn_status run_attn(const void* q, const float* q_scale, const int8_t* k_i8,
       !make_v_map(&tv, v, D, N, static_cast<long long>(B) * Hkv))
     return QATTN_ERR_CUDA;
   using Cfg = AttnCfg<D>;
-  auto kern = attn_fwd_kernel<D, CAUSAL, QF16>;
+  auto kern = attn_fwd_kernel<D, CAUSAL, QF16, DUMP>;
   // The kernel moves registers between its warpgroups with setmaxnreg; the split adds up only if
   // the launch allocates exactly kAttnLaunchRegs per thread, so never launch it otherwise.
   static int regs_checked = 0;
@@ -219,12 +221,12 @@ qattn_status run_attn(const void* q, const float* q_scale, const int8_t* k_i8,
       cudaSuccess)
     return QATTN_ERR_CUDA;
   const int nqt = (N + kBM - 1) / kBM;
-  const long long grid = static_cast<long long>(B) * H * ((nqt + 1) / 2);
+  const long long grid = DUMP ? dump_pairs : static_cast<long long>(B) * H * ((nqt + 1) / 2);
   if (grid > 0x7FFFFFFFLL) return QATTN_ERR_UNSUPPORTED;
   const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   kern<<<static_cast<unsigned>(grid), kAttnThreads, Cfg::kSmemBytes, st>>>(
       tq, tk, tv, q_scale, QF16 ? static_cast<const uint16_t*>(q) : nullptr, kv_list, kv_count, k_scale,
-      static_cast<__half*>(out), B, H, Hkv, N, scale_log2);
+      static_cast<__half*>(out), B, H, Hkv, N, scale_log2, dump ? *dump : ScoreDump{});
   return launch_status();
 }
 
@@ -534,7 +536,8 @@ qattn_status qattn_block_select(const void* q, const void* k, int B, int H, int 
   if (s != QATTN_OK) return s;
   s = check_ptrs(q, k, kv_list, kv_count);
   if (s != QATTN_OK) return s;
-  if (topk < 0) return QATTN_ERR_INVALID_ARG;
+  // non-causal with topk 0 would list no key tile for any query block
+  if (topk < 0 || (!causal && topk == 0)) return QATTN_ERR_INVALID_ARG;
   if ((N + kSelKRows - 1) / kSelKRows > kSelMaxTiles) return QATTN_ERR_UNSUPPORTED;
   if (ws == nullptr || ws_bytes < sel_layout(B, H, Hkv, N, d).total) return QATTN_ERR_WORKSPACE;
   if (!aligned16(ws)) return QATTN_ERR_MISALIGNED;
@@ -773,39 +776,58 @@ qattn_status qattn_forward_host(const void* q_host, const void* k_host, const vo
 }
 
 qattn_status qattn_debug_qk_int32(const int8_t* q_i8, const int8_t* k_i8, int32_t* s_out, int B,
-                                  int H, int Hkv, int N, int d, int b, int h, int qt0, int nqt,
-                                  int kt0, int nkt, qattn_stream_t stream) {
+                                  int H, int Hkv, int N, int d, int causal, int b, int h, int qt0,
+                                  int nqt, int kt0, int nkt, qattn_stream_t stream) {
   qattn_status s = check_shape(B, H, Hkv, N, d);
   if (s != QATTN_OK) return s;
   s = check_ptrs(q_i8, k_i8, s_out);
   if (s != QATTN_OK) return s;
   const int ntiles = (N + 127) / 128;
   if (b < 0 || b >= B || h < 0 || h >= H || qt0 < 0 || nqt < 1 || kt0 < 0 || nkt < 1 ||
-      qt0 + nqt > ntiles || kt0 + nkt > ntiles || nqt > 65535 || nkt > 65535)
+      qt0 + nqt > ntiles || kt0 + nkt > ntiles)
     return QATTN_ERR_INVALID_ARG;
   if ((s = device_ok()) != QATTN_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  CUtensorMap tq, tk;
-  if (!make_i8_map(&tq, q_i8, d, N, static_cast<long long>(B) * H) ||
-      !make_i8_map(&tk, k_i8, d, N, static_cast<long long>(B) * Hkv))
-    return QATTN_ERR_CUDA;
-  // 64 KB of shared memory per CTA caps residency at 3 CTAs (384 TMEM columns) per SM.
-  const int smem = 64 * 1024;
-  const int bh = b * H + h;
-  const int bg = b * Hkv + h / (H / Hkv);
-  dim3 grid(nqt, nkt);
-  if (d == 128) {
-    if (cudaFuncSetAttribute(qk_int32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-      return QATTN_ERR_CUDA;
-    qk_int32_kernel<128><<<grid, 128, smem, st>>>(tq, tk, s_out, bh, bg, qt0, kt0, nkt * 128);
-  } else {
-    if (cudaFuncSetAttribute(qk_int32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-      return QATTN_ERR_CUDA;
-    qk_int32_kernel<64><<<grid, 128, smem, st>>>(tq, tk, s_out, bh, bg, qt0, kt0, nkt * 128);
+  // The attention kernel itself runs, so it needs V, an output and scales: zero V and zero scales
+  // (every score then dequantizes to 0; the int32 tiles do not depend on them), from the pool.
+  const size_t nqb = (N + 127) / 128, nkb = (N + 63) / 64;
+  const size_t vb = align_up(sizeof(uint16_t) * static_cast<size_t>(B) * Hkv * N * d);
+  const size_t ob = align_up(sizeof(uint16_t) * static_cast<size_t>(B) * H * N * d);
+  const size_t qsb = align_up(sizeof(float) * static_cast<size_t>(B) * H * nqb);
+  const size_t ksb = align_up(sizeof(float) * static_cast<size_t>(B) * Hkv * nkb);
+  void* ws = nullptr;
+  if ((s = pool_alloc(&ws, vb + ob + qsb + ksb, st)) != QATTN_OK) return s;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const size_t s_bytes = sizeof(int32_t) * static_cast<size_t>(nqt) * 128 * nkt * 128;
+  // tiles the causal kernel never computes (key tile above the query tile) read as 0
+  if (cudaMemsetAsync(w, 0, vb, st) != cudaSuccess ||
+      cudaMemsetAsync(w + vb + ob, 0, qsb + ksb, st) != cudaSuccess ||
+      cudaMemsetAsync(s_out, 0, s_bytes, st) != cudaSuccess)
+    s = QATTN_ERR_CUDA;
+  ScoreDump dump;
+  dump.s_out = s_out;
+  dump.ld = nkt * 128;
+  dump.bh = b * H + h;
+  dump.pair0 = qt0 / 2;
+  dump.qt0 = qt0;
+  dump.nqt = nqt;
+  dump.kt0 = kt0;
+  dump.nkt = nkt;
+  const int pairs = (qt0 + nqt - 1) / 2 - qt0 / 2 + 1;
+  const float* qs = reinterpret_cast<const float*>(w + vb + ob);
+  const float* ks = reinterpret_cast<const float*>(w + vb + ob + qsb);
+  if (s == QATTN_OK) {
+#define QATTN_DUMP_ARGS q_i8, qs, k_i8, ks, w, w + vb, B, H, Hkv, N, st, nullptr, nullptr, &dump, pairs
+    if (d == 128)
+      s = causal ? run_attn<128, true, false, true>(QATTN_DUMP_ARGS)
+                 : run_attn<128, false, false, true>(QATTN_DUMP_ARGS);
+    else
+      s = causal ? run_attn<64, true, false, true>(QATTN_DUMP_ARGS)
+                 : run_attn<64, false, false, true>(QATTN_DUMP_ARGS);
+#undef QATTN_DUMP_ARGS
   }
-  return launch_status();
+  if (cudaFreeAsync(ws, st) != cudaSuccess && s == QATTN_OK) s = QATTN_ERR_CUDA;
+  return s;
 }
 
 qattn_status qattn_attn_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales, const float* q_g,

@@ -91,7 +91,7 @@ def _lib():
         L.qattn_forward.restype = i
         L.qattn_forward_host.argtypes = [P, P, P, P, i, i, i, i, i, i, P]
         L.qattn_forward_host.restype = i
-        L.qattn_debug_qk_int32.argtypes = [P, P, P, i, i, i, i, i, i, i, i, i, i, i, P]
+        L.qattn_debug_qk_int32.argtypes = [P, P, P, i, i, i, i, i, i, i, i, i, i, i, i, P]
         L.qattn_debug_qk_int32.restype = i
         L.qattn_debug_wait_timeout.argtypes = [ctypes.c_longlong, P, P]
         L.qattn_debug_wait_timeout.restype = i
@@ -172,8 +172,18 @@ def qattn_smooth_quant(q, k, q_i8=None, q_scale=None, k_i8=None, k_scale=None, k
 def qattn_smooth_quant_noalloc(q, k, q_i8, q_scale, k_i8, k_scale, k_mean=None, stream=None):
     """qattn_smooth_quant without a workspace or any allocation: the caller passes every output
     buffer, and the library's fixed device scratch (B*Hkv*d <= 65536) holds the channel sums.
-    For callers that cannot allocate device memory at call time."""
+    For callers that cannot allocate device memory at call time.  Every buffer is checked for
+    dtype, device and size first: the library writes them without knowing their sizes."""
     B, H, Hkv, N, d = _dims(q, k)
+    nqb, nkb = -(-N // QBLOCK), -(-N // KBLOCK)
+    want = [("q_i8", q_i8, torch.int8, B * H * N * d), ("q_scale", q_scale, torch.float32, B * H * nqb),
+            ("k_i8", k_i8, torch.int8, B * Hkv * N * d), ("k_scale", k_scale, torch.float32, B * Hkv * nkb)]
+    if k_mean is not None:
+        want.append(("k_mean", k_mean, torch.float32, B * Hkv * d))
+    for name, t, dt, n in want:
+        if t.dtype != dt or t.device != q.device or t.numel() != n:
+            raise ValueError(f"{name}: need {dt} with {n} elements on {q.device}, got {t.dtype} "
+                             f"with {t.numel()} on {t.device}")
     st = _lib().qattn_smooth_quant_noalloc(_p(q), _p(k), B, H, Hkv, N, d, _p(q_i8), _p(q_scale),
                                            _p(k_i8), _p(k_scale), _p(k_mean), _stream(stream))
     _check("qattn_smooth_quant_noalloc", st)
@@ -323,12 +333,15 @@ def qattn_forward_host(q, k, v, out=None, causal=False, stream=None):
     return out
 
 
-def qattn_debug_qk_int32(q_i8, k_i8, b, h, qt0, nqt, kt0, nkt, s_out=None, stream=None):
+def qattn_debug_qk_int32(q_i8, k_i8, b, h, qt0, nqt, kt0, nkt, causal=False, s_out=None,
+                         stream=None):
+    """int32 score tiles as the attention kernel (causal or not) loads them from tensor memory:
+    int32 [nqt*128, nkt*128] for query tiles qt0.. and key tiles kt0.. of batch b, head h."""
     B, H, Hkv, N, d = _dims(q_i8, k_i8)
     if s_out is None:
         s_out = torch.empty(nqt * 128, nkt * 128, dtype=torch.int32, device=q_i8.device)
-    st = _lib().qattn_debug_qk_int32(_p(q_i8), _p(k_i8), _p(s_out), B, H, Hkv, N, d, b, h, qt0,
-                                     nqt, kt0, nkt, _stream(stream))
+    st = _lib().qattn_debug_qk_int32(_p(q_i8), _p(k_i8), _p(s_out), B, H, Hkv, N, d,
+                                     int(bool(causal)), b, h, qt0, nqt, kt0, nkt, _stream(stream))
     _check("qattn_debug_qk_int32", st)
     return s_out
 

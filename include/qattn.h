@@ -130,7 +130,8 @@ size_t qattn_block_select_workspace(int B, int H, int Hkv, int N, int d);
  * Writes kv_list [B*H][ceil(N/256)][ceil(N/128)] (entries past the count are not written) and
  * kv_count [B*H][ceil(N/256)], both int32.  ws: at least qattn_block_select_workspace() bytes,
  * clobbered.  Lists are bit-exact functions of the inputs.  N <= 131072 (else
- * QATTN_ERR_UNSUPPORTED). */
+ * QATTN_ERR_UNSUPPORTED); topk < 0, or topk == 0 without causal (no tile for any block):
+ * QATTN_ERR_INVALID_ARG. */
 qattn_status qattn_block_select(const void* q, const void* k, int B, int H, int Hkv, int N, int d,
                                 int causal, int topk, int* kv_list, int* kv_count, void* ws,
                                 size_t ws_bytes, qattn_stream_t stream);
@@ -139,7 +140,8 @@ qattn_status qattn_block_select(const void* q, const void* k, int B, int H, int 
  * the tiles in kv_list[bh][i][0 .. kv_count[bh][i]) (and, when causal, only keys <= their own
  * index); the other tiles are neither loaded nor multiplied.  With every tile listed the result
  * equals qattn_attn_quantized's bit for bit.  Lists as written by qattn_block_select; a causal
- * list must hold its block's diagonal tiles (every row needs a key). */
+ * list must hold its block's diagonal tiles (every row needs a key).  A query tile whose list
+ * holds no tile it may see (kv_count 0) has no key to attend to: its rows are written as zeros. */
 qattn_status qattn_attn_quantized_sparse(const int8_t* q_i8, const float* q_scale,
                                          const int8_t* k_i8, const float* k_scale, const void* v,
                                          void* out, int B, int H, int Hkv, int N, int d,
@@ -280,14 +282,19 @@ qattn_status qattn_forward_nvfp4(const void* q, const void* k, const void* v, vo
  * Checks.
  * ------------------------------------------------------------------------------------------ */
 
-/* int32 score tiles S_int = Q_i8 K_i8^T through the same TMA -> tcgen05.mma kind::i8 -> tensor
- * memory -> tcgen05.ld path the attention kernel uses, without masking: for query tiles
- * qt0 .. qt0+nqt-1 and key tiles kt0 .. kt0+nkt-1 (128 rows each) of batch b, query head h.
- * s_out: device int32 [nqt*128, nkt*128], row-major; rows or columns beyond N are written as the
- * product with zero-filled rows (0). */
+/* int32 score tiles S_int = Q_i8 K_i8^T as the attention kernel itself computes and reads them
+ * (SageAttention page, sec. 3: the integer Q K^T with 32-bit accumulation): the kernel of
+ * qattn_attn_quantized (causal or not) runs for the Q-tile pairs that hold query tiles
+ * qt0 .. qt0+nqt-1 of batch b, query head h, and its softmax threads store the int32 scores they
+ * load from tensor memory for key tiles kt0 .. kt0+nkt-1 (128 rows each) before any masking.  V
+ * and the scales are zeros from the library's pool (the int32 tiles do not depend on them).
+ * s_out: device int32 [nqt*128][nkt*128], row-major; rows or columns beyond N hold the product
+ * with zero-filled rows (0); with causal != 0, tiles whose key tile lies above the query tile are
+ * never computed by the causal kernel and read as 0.  Errors: window outside the tiles of N, or
+ * b, h out of range: QATTN_ERR_INVALID_ARG; otherwise as qattn_attn_quantized. */
 qattn_status qattn_debug_qk_int32(const int8_t* q_i8, const int8_t* k_i8, int32_t* s_out, int B,
-                                  int H, int Hkv, int N, int d, int b, int h, int qt0, int nqt,
-                                  int kt0, int nkt, qattn_stream_t stream);
+                                  int H, int Hkv, int N, int d, int causal, int b, int h, int qt0,
+                                  int nqt, int kt0, int nkt, qattn_stream_t stream);
 
 /* FP4 score tiles through the block-scaled tensor cores: S = gQ gK * sum over the d channels of
  * E2M1(q) E4M3(sq) * E2M1(k) E4M3(sk), i.e. the dot products of the decoded NVFP4 rows, computed

@@ -192,6 +192,53 @@ def attention_quantized(q_i8, q_scale, k_i8, k_scale, v, B, H, Hkv, N, d, causal
     return out
 
 
+def attention_quantized_all(q_i8, q_scale, k_i8, k_scale, v, B, H, Hkv, N, d, causal,
+                            chunk=2048):
+    """Every row of the quantized attention output (float64 [B*H*N, d], rows in (b, h, i) order):
+    the definition attention_quantized evaluates row by row in C, written here with float64
+    library matmuls on the CPU (torch), one query head and up to `chunk` of its rows at a time, so
+    that whole workloads finish in minutes.  Per row i of head (b, h), kv head g = h / (H / Hkv):
+      S_int[i, j] = sum_c q_i8[i, c] k_i8[j, c]  (a float64 matmul of integers: every partial sum
+                    is an integer below 2^53, so it is exact),
+      S[i, j]     = ((S_int[i, j] * sQ[i / 128]) * sK[j / 64]) * (1 / sqrt(d)),
+      keys j > i dropped when causal, P = exp(S - max_j S), O[i] = sum_j P[i, j] V[j] / sum_j P[i, j]
+    (SageAttention page, sec. 3-4: the int32 product, dequantized with the two block scales, then
+    the softmax and P V; the blockwise online softmax equals this plain row softmax up to rounding).
+    Only the summation order of the float64 sums differs from the C loops."""
+    import torch
+    q_i8 = np.ascontiguousarray(q_i8, dtype=np.int8).reshape(B, H, N, d)
+    k_i8 = np.ascontiguousarray(k_i8, dtype=np.int8).reshape(B, Hkv, N, d)
+    q_scale = np.asarray(q_scale, dtype=np.float32).reshape(B, H, -1)
+    k_scale = np.asarray(k_scale, dtype=np.float32).reshape(B, Hkv, -1)
+    vv = _bits16(v).reshape(B, Hkv, N, d)
+    inv_sqrt_d = 1.0 / np.sqrt(float(d))
+    G = H // Hkv
+    out = np.empty((B * H * N, d), dtype=np.float64)
+    for b in range(B):
+        for g in range(Hkv):
+            K = torch.from_numpy(k_i8[b, g].astype(np.float64))
+            V = torch.from_numpy(vv[b, g].view(np.float16).astype(np.float64))
+            sk = torch.from_numpy(np.repeat(k_scale[b, g].astype(np.float64), KBLOCK)[:N])
+            for h in range(g * G, (g + 1) * G):
+                Q = q_i8[b, h]
+                sq = np.repeat(q_scale[b, h].astype(np.float64), QBLOCK)[:N]
+                for r0 in range(0, N, chunk):
+                    r1 = min(N, r0 + chunk)
+                    nk = r1 if causal else N
+                    S = torch.from_numpy(Q[r0:r1].astype(np.float64)) @ K[:nk].T
+                    S = S * torch.from_numpy(sq[r0:r1])[:, None]
+                    S = S * sk[None, :nk]
+                    S = S * inv_sqrt_d
+                    if causal:
+                        later = torch.arange(nk)[None, :] > torch.arange(r0, r1)[:, None]
+                        S.masked_fill_(later, -np.inf)
+                    P = torch.exp(S - S.max(dim=1, keepdim=True).values)
+                    O = (P @ V[:nk]) / P.sum(dim=1, keepdim=True)
+                    row0 = (b * H + h) * N
+                    out[row0 + r0: row0 + r1] = O.numpy()
+    return out
+
+
 SBLOCK = 256  # block-sparse selection: query rows per selection block
 KTILE = 128   # block-sparse selection: keys per key tile
 

@@ -49,7 +49,8 @@ def out_errors(gpu_out_rows, ref64_rows):
     return float(e.max()), float(e.mean())
 
 
-# Output tolerances of the forward against the oracle's unrounded float64 output.
+# Output tolerances of the forward against the oracle's unrounded float64 output: max-abs 2e-3
+# and mean-abs 2e-4, flat, over every compared element.
 MAX_ABS_TOL = 2e-3
 MEAN_ABS_TOL = 2e-4
 
@@ -57,20 +58,17 @@ MEAN_ABS_TOL = 2e-4
 def check_output(gpu_out_rows, ref64_rows):
     """Applies the output tolerance; returns (ok, message).
 
-    mean |O_gpu - O64| <= 2e-4 over all elements, and max |O_gpu - O64| <= 2e-3 for every
-    element with |O64| < 4.  The output is fp16, whose own rounding (half the spacing of the fp16
-    grid) is 1.95e-3 for |O| in [4, 8): there the budget is 2e-3 on top of that half-spacing."""
+    max |O_gpu - O64| <= 2e-3 and mean |O_gpu - O64| <= 2e-4 over all compared elements, O_gpu
+    the fp16 output and O64 the oracle's unrounded float64 output.  The message also reports, for
+    information, the floor the fp16 output type alone sets: max and mean |fp16(O64) - O64|."""
     import numpy as np
     g = gpu_out_rows.astype(np.float64)
     r = np.asarray(ref64_rows, dtype=np.float64)
     e = np.abs(g - r)
-    half_ulp = np.spacing(np.abs(r).astype(np.float16)).astype(np.float64) / 2
-    big = np.abs(r) >= 4.0
-    allow = np.where(big, MAX_ABS_TOL + half_ulp, MAX_ABS_TOL)
-    excess = e - allow
-    i = int(np.argmax(excess))
-    mean = float(e.mean())
-    msg = (f"max-abs {e.max():.3e} (|O|={abs(r.flat[int(np.argmax(e))]):.3f}), worst vs allowance "
-           f"{e.flat[i]:.3e} <= {allow.flat[i]:.3e} at |O|={abs(r.flat[i]):.3f}, mean-abs "
-           f"{mean:.3e}, elements with |O|>=4: {int(big.sum())}")
-    return bool(excess.max() <= 0 and mean <= MEAN_ABS_TOL), msg
+    floor = np.abs(r.astype(np.float16).astype(np.float64) - r)
+    i = int(np.argmax(e))
+    mx, mean = float(e.flat[i]), float(e.mean())
+    msg = (f"max-abs {mx:.3e} at |O|={abs(r.flat[i]):.3f} (fp16 floor there {floor.flat[i]:.3e}), "
+           f"mean-abs {mean:.3e}; fp16 rounding floor max {floor.max():.3e} mean {floor.mean():.3e}; "
+           f"elements {e.size}, over 2e-3: {int((e > MAX_ABS_TOL).sum())}")
+    return bool(mx <= MAX_ABS_TOL and mean <= MEAN_ABS_TOL), msg

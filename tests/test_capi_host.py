@@ -93,9 +93,9 @@ def test_workspace_and_alignment_checks():
     st = L.qattn_smooth_quant(P(16), P(32), 1, 4, 2, 256, 128, P(48), P(64), P(80), P(96), P(20),
                               P(112), 1 << 20, None)
     assert st == 3
-    st = L.qattn_debug_qk_int32(P(16), P(32), P(48), 1, 4, 2, 256, 128, 0, 0, 1, 2, 0, 1, None)
+    st = L.qattn_debug_qk_int32(P(16), P(32), P(48), 1, 4, 2, 256, 128, 0, 0, 0, 1, 2, 0, 1, None)
     assert st == 1
-    st = L.qattn_debug_qk_int32(P(16), P(32), P(48), 1, 4, 2, 256, 128, 0, 4, 0, 1, 0, 1, None)
+    st = L.qattn_debug_qk_int32(P(16), P(32), P(48), 1, 4, 2, 256, 128, 1, 0, 4, 0, 1, 0, 1, None)
     assert st == 1
     assert L.qattn_debug_wait_timeout(1000, None, None) == 1
     assert L.qattn_debug_wait_timeout(-1, P(16), None) == 1
@@ -114,6 +114,34 @@ def test_workspace_and_alignment_checks():
 def test_forward_sparse_argument_checks(args, expect):
     L = Q.load()
     assert L.qattn_forward_sparse(*args) == expect
+
+
+@pytest.mark.parametrize("causal,topk,expect", [(0, 0, 1), (0, -1, 1), (1, -1, 1)])
+def test_block_select_rejects_empty_selections(causal, topk, expect):
+    # non-causal topk 0 would list no key tile for any query block
+    L = Q.load()
+    st = L.qattn_block_select(P(16), P(32), 1, 4, 2, 256, 128, causal, topk, P(48), P(64),
+                              P(4096), 1 << 20, None)
+    assert st == expect
+
+
+@pytest.mark.parametrize("bad", ["q_i8", "q_scale", "k_i8", "k_scale", "k_mean"])
+def test_noalloc_binding_checks_output_buffers(bad):
+    # the allocation-free entry writes caller buffers whose sizes it cannot see: the binding
+    # checks dtype and size before calling it (CPU tensors here, so nothing reaches a device)
+    import torch
+    B, H, Hkv, N, d = 1, 4, 2, 300, 64
+    q = torch.zeros(B, H, N, d, dtype=torch.float16)
+    k = torch.zeros(B, Hkv, N, d, dtype=torch.float16)
+    bufs = {"q_i8": torch.empty(B, H, N, d, dtype=torch.int8),
+            "q_scale": torch.empty(B, H, 3, dtype=torch.float32),
+            "k_i8": torch.empty(B, Hkv, N, d, dtype=torch.int8),
+            "k_scale": torch.empty(B, Hkv, 5, dtype=torch.float32),
+            "k_mean": torch.empty(B, Hkv, d, dtype=torch.float32)}
+    t = bufs[bad]
+    bufs[bad] = torch.empty(t.numel() - 1, dtype=t.dtype) if bad != "k_i8" else t.to(torch.uint8)
+    with pytest.raises(ValueError, match=bad):
+        Q.qattn_smooth_quant_noalloc(q, k, **bufs)
 
 
 @pytest.mark.parametrize("args,expect", [

@@ -7,13 +7,16 @@ tiles are computed (the sparse top-k variant its results section compares agains
  * the selection lists and counts are index work: bit-exact against the oracle;
  * the attention over the selected tiles: within the same tolerance as the dense path, against
    the oracle's attention restricted to the same tile mask on the oracle's own int8 codes;
- * with every tile listed, the sparse kernel reproduces the dense kernel bit for bit.
+ * with every tile listed, the sparse kernel reproduces the dense kernel bit for bit;
+ * a query block whose list is empty has no key: its rows come out as zeros;
+ * at full size (llama8b_32k top-16, long128k top-64, the bench's sparse modes) the lists are
+   compared in full and a seeded sample of output rows against the oracle.
 """
 import numpy as np
 import pytest
 import torch
 
-from bit_quantized_attention_smoothing_b200.workloads import WORKLOADS, make_inputs
+from bit_quantized_attention_smoothing_b200.workloads import WORKLOADS, make_inputs, sample_rows
 from conftest import check_output, np16
 
 pytestmark = pytest.mark.gpu
@@ -120,3 +123,51 @@ def test_block_select_ties_bit_exact(lib, oracle, causal, pattern):
         torch.cuda.synchronize()
         rl, rc = oracle.block_select(np16(q), np16(k), w.B, w.H, w.Hkv, w.N, w.d, causal, topk)
         _lists_equal(gl, gc, rl, rc)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_empty_lists_give_zero_rows(lib, causal):
+    """Query blocks whose kv_count is 0 (lists a caller built; the selection never writes one)
+    have no key to attend to: the kernel writes their rows as zeros and reports no error; the
+    other blocks are unaffected (equal to the dense kernel, since they list every tile)."""
+    w = WORKLOADS["prefill4k"].with_(B=1, H=2, Hkv=1, N=1000, causal=causal)
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    q_i8, q_s, k_i8, k_s, _ = lib.qattn_smooth_quant(q, k)
+    kl, kc = lib.qattn_block_select(q, k, 10 ** 6, causal=causal)
+    kc[:, 1] = 0        # rows 256 .. 511 of both heads
+    dense = lib.qattn_attn_quantized(q_i8, q_s, k_i8, k_s, v, causal=causal)
+    sparse = lib.qattn_attn_quantized_sparse(q_i8, q_s, k_i8, k_s, v, kl, kc, causal=causal)
+    torch.cuda.synchronize()
+    assert lib.qattn_check_device_status() == 0
+    assert torch.count_nonzero(sparse[:, :, 256:512]) == 0
+    assert torch.equal(sparse[:, :, :256], dense[:, :, :256])
+    assert torch.equal(sparse[:, :, 512:], dense[:, :, 512:])
+
+
+@pytest.mark.parametrize("name,topk", [("llama8b_32k", 16), ("long128k", 64)])
+def test_full_size_sparse(lib, oracle, name, topk):
+    """The bench's block-sparse modes at full size: every list and count bit-exact against the
+    oracle's selection, then the one-call sparse forward on a seeded sample of rows per head (the
+    first and last rows of the sequence and random ones) against the oracle's attention restricted
+    to the same tiles."""
+    w = WORKLOADS[name]
+    q, k, v = make_inputs(w, device="cuda")
+    gl, gc = lib.qattn_block_select(q, k, topk, causal=w.causal)
+    torch.cuda.synchronize()
+    qh, kh, vh = np16(q), np16(k), np16(v)
+    rl, rc = oracle.block_select(qh, kh, w.B, w.H, w.Hkv, w.N, w.d, w.causal, topk)
+    _lists_equal(gl, gc, rl, rc)
+    del gl, gc
+    out = lib.qattn_forward_sparse(q, k, v, topk, causal=w.causal)
+    assert lib.qattn_check_device_status() == 0
+    rows = tuple(t.numpy() for t in sample_rows(w, 8, edge_first=8, edge_last=8))
+    flat = out.reshape(-1, w.d)
+    got = flat[torch.as_tensor(rows[0] * w.N + rows[1], device=out.device)].float().cpu().numpy()
+    del out, flat, q, k, v
+    sq = oracle.smooth_quant(qh, kh, w.B, w.H, w.Hkv, w.N, w.d)
+    ref = oracle.attention_quantized_sparse(sq["q_i8"], sq["q_scale"], sq["k_i8"], sq["k_scale"],
+                                            vh, w.B, w.H, w.Hkv, w.N, w.d, w.causal,
+                                            oracle.tile_mask(rl, rc, w.N), rows=rows)
+    ok, msg = check_output(got, ref)
+    print(name, f"top{topk}", msg)
+    assert ok, msg

@@ -1,16 +1,18 @@
 """GPU parity: the CUDA path through the C ABI against the CPU oracle on the same seeded inputs.
 
 * smoothing + quantization (int8 codes, block scales, channel means): bit-exact;
-* int32 score tiles from the tcgen05 kind::i8 path: bit-exact;
-* forward output: mean-abs <= 2e-4 and max-abs <= 2e-3 against the oracle's unrounded float64
-  output (the oracle rounds nothing after the int32 product; the GPU rounds P to fp16, accumulates
-  in fp32, uses a hardware exp2 and rounds O to fp16); where |O| >= 4 the fp16 output grid's own
-  half-spacing (1.95e-3) is added to the 2e-3 budget (tests/conftest.py, check_output).
+* int32 score tiles, as the attention kernel itself loads them from tensor memory (its DUMP
+  instantiation, causal and non-causal): bit-exact;
+* forward output: max-abs <= 2e-3 and mean-abs <= 2e-4 against the oracle's unrounded float64
+  output, flat (tests/conftest.py, check_output; the oracle rounds nothing after the int32
+  product, the GPU rounds P to fp16, accumulates in fp32, uses a hardware exp2 and rounds O to
+  fp16).
 
 Small cases compare every output element and cover ragged N (partial Q tile, partial K block,
 odd tile counts), N=1, GQA, causal and non-causal, d=64 and d=128.  The five named workloads run at
-full size with the bench's launch configuration, comparing every int8 code and scale and a seeded
-sample of output rows (first and last rows of every head plus random rows).
+full size with the bench's launch configuration, comparing every int8 code and scale, every
+output row of tiny, prefill4k and wide64 and a seeded sample of rows of llama8b_32k and long128k
+(first and last rows of every head plus random rows).
 """
 import numpy as np
 import pytest
@@ -42,8 +44,9 @@ SMALL = [
 ]
 SMALL_IDS = [f"{n}-" + "-".join(f"{k}{v}" for k, v in o.items()) for n, o in SMALL]
 
-# rows sampled per head at full size (plus the first 128 and last 128 rows of every head)
-FULL_SAMPLES = {"tiny": None, "prefill4k": 32, "llama8b_32k": 32, "long128k": 4, "wide64": 32}
+# rows sampled per head at full size (plus the first 128 and last 128 rows of every head); None:
+# every row (the oracle's matmul form for the larger ones)
+FULL_SAMPLES = {"tiny": None, "prefill4k": None, "llama8b_32k": 32, "long128k": 4, "wide64": None}
 
 
 def _inputs(w, device="cuda"):
@@ -79,17 +82,23 @@ def test_smooth_quant_bit_exact_small(lib, oracle, name, over):
 
 @pytest.mark.parametrize("name,over", SMALL, ids=SMALL_IDS)
 def test_qk_int32_tiles_bit_exact_small(lib, oracle, name, over):
+    """The int32 scores the attention kernel's softmax threads load from tensor memory (non-causal
+    kernel: every tile; causal kernel: the tiles it computes, the others untouched)."""
     w = WORKLOADS[name].with_(**over)
     q, k, _ = _inputs(w, "cpu")
     (q_i8, _, k_i8, _), ref = _check_quant(lib, oracle, w, q, k)
     nt = -(-w.N // 128)
+    lower = np.kron(np.tril(np.ones((nt, nt), dtype=bool)), np.ones((128, 128), dtype=bool))
     for b, h in {(0, 0), (w.B - 1, w.H - 1)}:
-        s = lib.qattn_debug_qk_int32(q_i8, k_i8, b, h, 0, nt, 0, nt).cpu().numpy()
         # rows/columns beyond N are products with zero-filled rows
         full = np.zeros((nt * 128, nt * 128), dtype=np.int32)
         full[: w.N, : w.N] = oracle.qk_int32(ref["q_i8"], ref["k_i8"], w.B, w.H, w.Hkv, w.N, w.d,
                                              b, h, 0, w.N, 0, w.N)
+        s = lib.qattn_debug_qk_int32(q_i8, k_i8, b, h, 0, nt, 0, nt, causal=False).cpu().numpy()
         assert np.array_equal(s, full)
+        s = lib.qattn_debug_qk_int32(q_i8, k_i8, b, h, 0, nt, 0, nt, causal=True).cpu().numpy()
+        assert np.array_equal(s, np.where(lower, full, 0))
+    assert lib.qattn_check_device_status() == 0
 
 
 @pytest.mark.parametrize("name,over", SMALL, ids=SMALL_IDS)
@@ -114,6 +123,20 @@ def test_attention_on_oracle_codes(lib, oracle, name, over):
                                    causal=w.causal)
     ref = oracle.attention_quantized(ref_sq["q_i8"], ref_sq["q_scale"], ref_sq["k_i8"],
                                      ref_sq["k_scale"], np16(v), w.B, w.H, w.Hkv, w.N, w.d, w.causal)
+    ok, msg = check_output(out.float().cpu().numpy().reshape(-1, w.d), ref)
+    assert ok, msg
+
+
+@pytest.mark.parametrize("name,over", SMALL, ids=SMALL_IDS)
+def test_fused_q_forward_against_oracle(lib, oracle, name, over):
+    """qattn_smooth_k + qattn_attn_fused_q (Q quantized inside the attention kernel) against the
+    oracle's whole path, every output element."""
+    w = WORKLOADS[name].with_(**over)
+    q, k, v = _inputs(w)
+    k_i8, k_s, _ = lib.qattn_smooth_k(k)
+    out = lib.qattn_attn_fused_q(q, k_i8, k_s, v, causal=w.causal)
+    assert lib.qattn_check_device_status() == 0
+    ref, _ = oracle.forward(np16(q), np16(k), np16(v), w.B, w.H, w.Hkv, w.N, w.d, w.causal)
     ok, msg = check_output(out.float().cpu().numpy().reshape(-1, w.d), ref)
     assert ok, msg
 
@@ -219,29 +242,42 @@ def test_gpu_rejects_bad_arguments(lib):
 
 @pytest.mark.parametrize("name", ORDER)
 def test_full_size_workload(lib, oracle, name):
-    """Full-size workload, same launch as the benchmark: every code and scale bit-exact, a seeded
-    sample of output rows within tolerance, plus int32 score tiles on the first/last tiles."""
+    """Full-size workload, same launch as the benchmark: every code and scale bit-exact, int32
+    score tiles of the product kernel (causal as the workload) on the first, last, a middle and the
+    whole last row of key tiles, and the output rows (all rows, or a seeded sample) within
+    tolerance."""
     w = WORKLOADS[name]
     q, k, v = make_inputs(w, device="cuda")
     (q_i8, _, k_i8, _), ref_sq = _check_quant(lib, oracle, w, q, k)
     nt = -(-w.N // 128)
-    for qt, kt in {(0, 0), (nt - 1, nt - 1), (nt - 1, 0), (nt // 2, nt // 3)}:
-        s = lib.qattn_debug_qk_int32(q_i8, k_i8, w.B - 1, w.H - 1, qt, 1, kt, 1).cpu().numpy()
+    b, h = w.B - 1, w.H - 1
+    for qt, kt, nk in {(0, 0, 1), (nt - 1, nt - 1, 1), (nt // 2, nt // 3, 1), (nt - 1, 0, nt)}:
+        s = lib.qattn_debug_qk_int32(q_i8, k_i8, b, h, qt, 1, kt, nk, causal=w.causal).cpu().numpy()
         r = oracle.qk_int32(ref_sq["q_i8"], ref_sq["k_i8"], w.B, w.H, w.Hkv, w.N, w.d,
-                            w.B - 1, w.H - 1, qt * 128, 128, kt * 128, 128)
-        assert np.array_equal(s, r)
+                            b, h, qt * 128, min(128, w.N - qt * 128), kt * 128, min(nk * 128, w.N - kt * 128))
+        assert np.array_equal(s[: r.shape[0], : r.shape[1]], r)
     del q_i8, k_i8
     out = lib.qattn_forward(q, k, v, causal=w.causal)
     assert lib.qattn_check_device_status() == 0
     per = FULL_SAMPLES[name]
     if per is None:
-        rows = oracle.all_rows(w.B, w.H, w.N)
+        got = out.float().cpu().numpy().reshape(-1, w.d)
+        del out
+        if w.B * w.H * w.N <= 4096:
+            ref = oracle.attention_quantized(ref_sq["q_i8"], ref_sq["q_scale"], ref_sq["k_i8"],
+                                             ref_sq["k_scale"], np16(v), w.B, w.H, w.Hkv, w.N,
+                                             w.d, w.causal)
+        else:
+            ref = oracle.attention_quantized_all(ref_sq["q_i8"], ref_sq["q_scale"], ref_sq["k_i8"],
+                                                 ref_sq["k_scale"], np16(v), w.B, w.H, w.Hkv, w.N,
+                                                 w.d, w.causal)
     else:
         rows = tuple(t.numpy() for t in sample_rows(w, per, edge_first=128, edge_last=128 if per > 4 else 8))
-    ref = oracle.attention_quantized(ref_sq["q_i8"], ref_sq["q_scale"], ref_sq["k_i8"],
-                                     ref_sq["k_scale"], np16(v), w.B, w.H, w.Hkv, w.N, w.d,
-                                     w.causal, rows=rows)
-    ok, msg = check_output(_rows_of(out, w, rows), ref)
+        got = _rows_of(out, w, rows)
+        ref = oracle.attention_quantized(ref_sq["q_i8"], ref_sq["q_scale"], ref_sq["k_i8"],
+                                         ref_sq["k_scale"], np16(v), w.B, w.H, w.Hkv, w.N, w.d,
+                                         w.causal, rows=rows)
+    ok, msg = check_output(got, ref)
     print(name, msg)
     assert ok, msg
 

@@ -287,6 +287,50 @@ def test_quantized_attention_exact_on_dyadic_inputs(oracle, causal):
     np.testing.assert_allclose(out.reshape(B, H, N, d), ref, rtol=0, atol=1e-12)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_matmul_form_exact_on_dyadic_inputs(oracle, causal):
+    """The oracle's matmul form of the quantized attention (attention_quantized_all, used to
+    compare every row of the larger workloads) on the dyadic inputs above: float64 SDPA to 1e-12,
+    which pins its block indexing and dequantization independently of the C loops."""
+    rng = np.random.default_rng(9)
+    B, H, Hkv, N, d = 1, 2, 1, 256, 16
+    q = np.zeros((B, H, N, d))
+    for h in range(H):
+        for blk, e in enumerate([-6, -4]):
+            x = rng.integers(-126, 127, (128, d)).astype(np.float64)
+            x[0, 0] = 127
+            q[0, h, blk * 128:(blk + 1) * 128] = x * 2.0 ** (e - h)
+    k = np.zeros((B, Hkv, N, d))
+    for blk, e in enumerate([-7, -5, -6, -8]):
+        x = rng.integers(-126, 127, (32, d)).astype(np.float64)
+        x[0, 0] = 127
+        k[0, 0, blk * 64:(blk + 1) * 64] = np.concatenate([x, -x]) * 2.0 ** e
+    v = rng.standard_normal((B, Hkv, N, d))
+    q, k, v = q.astype(np.float16), k.astype(np.float16), v.astype(np.float16)
+    sq = oracle.smooth_quant(q, k, B, H, Hkv, N, d)
+    out = oracle.attention_quantized_all(sq["q_i8"], sq["q_scale"], sq["k_i8"], sq["k_scale"], v,
+                                         B, H, Hkv, N, d, causal, chunk=100)
+    np.testing.assert_allclose(out.reshape(B, H, N, d), _sdpa64(q, k, v, H, Hkv, causal), rtol=0,
+                               atol=1e-12)
+
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny", {}), ("tiny", {"N": 129, "causal": True}), ("prefill4k", {"B": 2, "H": 4, "Hkv": 2, "N": 700}),
+    ("wide64", {"B": 1, "H": 3, "Hkv": 1, "N": 1100}), ("long128k", {"H": 2, "Hkv": 1, "N": 900}),
+])
+def test_matmul_form_equals_row_loops(oracle, name, over):
+    """The matmul form and the C row loops are two writings of one definition; they may differ
+    only in the order of the float64 sums (chunks of 300 rows cross the 128-row Q blocks)."""
+    w = WORKLOADS[name].with_(**over)
+    q, k, v = (_np16(t) for t in make_inputs(w))
+    sq = oracle.smooth_quant(q, k, w.B, w.H, w.Hkv, w.N, w.d)
+    args = (sq["q_i8"], sq["q_scale"], sq["k_i8"], sq["k_scale"], v, w.B, w.H, w.Hkv, w.N, w.d,
+            w.causal)
+    a = oracle.attention_quantized(*args)
+    b = oracle.attention_quantized_all(*args, chunk=300)
+    assert np.abs(a - b).max() <= 1e-12 * max(1.0, np.abs(a).max())
+
+
 def test_causal_first_row_is_v0(oracle):
     w = WORKLOADS["tiny"].with_(causal=True, N=200)
     q, k, v = (_np16(t) for t in make_inputs(w))
