@@ -122,7 +122,7 @@ __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, 
       : "f"(a0), "f"(a1), "f"(b), "f"(c));
 }
 
-// (d0, d1) = (a0 + b0, a1 + b1) and (a0 * b0 + c0, a1 * b1 + c1) as packed sm_100 fp32x2 ops.
+// (d0, d1) = (a0 + b0, a1 + b1) as one packed sm_100 fp32x2 add.
 __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
   asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
       "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
@@ -130,43 +130,8 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, 
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
-__device__ __forceinline__ void ffma2v(float& d0, float& d1, float a0, float a1, float b0, float b1,
-                                       float c0, float c1) {
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
-}
 
-// 2^f on [-1/2, 1/2]: degree-4 minimax polynomial (relative error 2.6e-6), coefficients from
-// gen_exp2_poly.py (Chebyshev start, Remez exchange).
-constexpr float kExpC0 = 0.9999992847442627f;
-constexpr float kExpC1 = 0.6931217908859253f;
-constexpr float kExpC2 = 0.240247443318367f;
-constexpr float kExpC3 = 0.05591785907745361f;
-constexpr float kExpC4 = 0.009570102207362652f;
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: x + M rounds x to an integer
-
-// 2^y for two values on the FMA pipe instead of MUFU: n = round(y) through the 1.5 * 2^23 add,
-// f = y - n (exact), 2^y = p(f) * 2^n with the power of two added to the exponent bits.  y is
-// clamped at -125 so the exponent stays normal; the results only feed fp16 P, where anything
-// below 2^-24 is zero anyway.
-__device__ __forceinline__ void exp2_poly2(float y0, float y1, float& r0, float& r1) {
-  y0 = fmaxf(y0, -125.0f);
-  y1 = fmaxf(y1, -125.0f);
-  float t0, t1, n0, n1, f0, f1, p0, p1;
-  fadd2(t0, t1, y0, y1, kRoundMagic, kRoundMagic);
-  fadd2(n0, n1, t0, t1, -kRoundMagic, -kRoundMagic);
-  ffma2v(f0, f1, n0, n1, -1.0f, -1.0f, y0, y1);
-  ffma2v(p0, p1, f0, f1, kExpC4, kExpC4, kExpC3, kExpC3);
-  ffma2v(p0, p1, p0, p1, f0, f1, kExpC2, kExpC2);
-  ffma2v(p0, p1, p0, p1, f0, f1, kExpC1, kExpC1);
-  ffma2v(p0, p1, p0, p1, f0, f1, kExpC0, kExpC0);
-  // the low 9 bits of t's pattern hold n (two's complement), so t << 23 is n << 23
-  r0 = __uint_as_float((__float_as_uint(t0) << 23) + __float_as_uint(p0));
-  r1 = __uint_as_float((__float_as_uint(t1) << 23) + __float_as_uint(p1));
-}
 
 __device__ __forceinline__ float scaled_max(float m, float c) {
   return m == -INFINITY ? -INFINITY : m * c;
@@ -178,21 +143,14 @@ __device__ __forceinline__ float scaled_max(float m, float c) {
 __device__ __forceinline__ float score_biased(uint32_t s) { return __uint_as_float(s + 0x4B400000u); }
 static_assert(127 * 127 * 128 < (1 << 22), "biased score conversion range");
 
-// Score-register groups i (0-15) for which kExp2EmulateMask has bit i set go through exp2_poly2
-// on the FMA pipe; the rest use MUFU ex2.  Measured on B200 (llama8b_32k): moving 1/8, 1/4 or 3/8
-// of the exponentials to the FMA pipe made the kernel 3 %, 7 % and 13 % slower, so none is moved.
-constexpr uint32_t kExp2EmulateMask = 0x0000;
-__device__ __forceinline__ constexpr bool emulated_pair(int i) { return (kExp2EmulateMask >> i) & 1; }
-
 // One 128-key step of the softmax for the thread's score row: int32 -> float (exact, see
-// score_biased),
-// masked keys (MASK; key offset above lim) -> -inf, row maximum per 64-key K scale block, lazy
+// score_biased), masked keys (MASK; key offset above lim) -> -inf, row maximum per 64-key K scale block, lazy
 // update of the running max m (alpha = rescale factor, need = O must be rescaled), then
 // P = 2^(x * c - m + offset) packed as fp16 pairs (even key in the low half) and stored over the
 // row's first 64 TMEM columns, and the row sum of the fp16-rounded P.  Once the first 64 keys'
 // P are stored, the warp arrives on mx_bar (the other Q tile's softmax waits for it).  MASK is a
 // compile-time switch so the unmasked steps carry no per-element tests.
-template <bool MASK>
+template <int D, bool MASK>
 __device__ __forceinline__ void softmax_row(uint32_t (&sr)[4][32], int lim, float c0, float c1,
                                             bool first, float& m, float& l, float& alpha,
                                             bool& need, uint32_t s_tm, uint64_t* mx_bar) {
@@ -232,17 +190,12 @@ __device__ __forceinline__ void softmax_row(uint32_t (&sr)[4][32], int lim, floa
     for (int q = 0; q < 2; ++q) {
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
-        const int i = (2 * hf + q) * 16 + (e >> 1);  // pair index 0..63
         float x0, x1, y0, y1, p0, p1;
         fadd2(x0, x1, __uint_as_float(sr[2 * hf + q][e]), __uint_as_float(sr[2 * hf + q][e + 1]),
               -kRoundMagic, -kRoundMagic);
         ffma2(y0, y1, x0, x1, c, g);
-        if (emulated_pair(i & 15)) {
-          exp2_poly2(y0, y1, p0, p1);
-        } else {
-          p0 = ex2_approx(y0);
-          p1 = ex2_approx(y1);
-        }
+        p0 = ex2_approx(y0);
+        p1 = ex2_approx(y1);
         if (MASK) {
           // -inf * 0 would be NaN for a zero-scale block: select instead
           if (x0 == -INFINITY) p0 = 0.0f;
@@ -364,7 +317,15 @@ __device__ __forceinline__ void setmaxnreg_dec56() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
 }
 
-// Score-tile dump of the DUMP instantiation: the CTAs of query head bh, pairs pair0 .. (one per
+// Instantiations of the attention kernel.  kOutF16 is the product (fp16 output); kDumpS is the
+// same kernel, which also writes the int32 score tiles it reads (the exactness check of Q K^T);
+// kOutF32 writes O / l as fp32 instead of rounding it to fp16 (the fp16 output is exactly its
+// round-to-nearest).
+constexpr int kOutF16 = 0;
+constexpr int kDumpS = 1;
+constexpr int kOutF32 = 2;
+
+// Score-tile dump of the kDumpS instantiation: the CTAs of query head bh, pairs pair0 .. (one per
 // block), store the raw int32 scores each softmax thread loads from tensor memory for query tiles
 // qt0 .. qt0+nqt-1 and key tiles kt0 .. kt0+nkt-1 into s_out [nqt*128][ld] (row-major).
 struct ScoreDump {
@@ -375,16 +336,18 @@ struct ScoreDump {
 // QF16: Q arrives as fp16 (q16) and the softmax warps quantize their own Q tile into shared
 // memory before the first QK^T (per-tile amax, scale = amax / 127, the same rounding as
 // quantize_kernel); otherwise int8 Q and its scales come from the smoothing + quantization pass
-// (tm_q, q_scale).  DUMP: the same kernel, which also writes the int32 score tiles it reads (the
-// exactness check of Q K^T); only its block-to-work mapping differs (see ScoreDump).
-template <int D, bool CAUSAL, bool QF16, bool DUMP = false>
+// (tm_q, q_scale).  MODE: kOutF16, kDumpS (only its block-to-work mapping differs, see
+// ScoreDump) or kOutF32 (out points to fp32).
+template <int D, bool CAUSAL, bool QF16, int MODE = kOutF16>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scale,
                     const uint16_t* __restrict__ q16, const int* __restrict__ kv_list,
                     const int* __restrict__ kv_count,
-                    const float* __restrict__ k_scale, __half* __restrict__ out, int B, int H,
+                    const float* __restrict__ k_scale, void* __restrict__ out_any, int B, int H,
                     int Hkv, int N, float scale_log2, ScoreDump dump) {
+  constexpr bool DUMP = MODE == kDumpS;
+  __half* out = static_cast<__half*>(out_any);
   using Cfg = AttnCfg<D>;
   constexpr int ST = Cfg::kStages;
   constexpr int kTmaWarp = kSoftmaxThreads / 32;  // warp 8
@@ -640,8 +603,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const bool masked = __any_sync(0xFFFFFFFFu, lim < kBN - 1);
         float alpha;
         bool need;
-        if (masked) softmax_row<true>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, &bars->mx_done[wt][warp & 3]);
-        else softmax_row<false>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, &bars->mx_done[wt][warp & 3]);
+        if (masked) softmax_row<D, true>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, &bars->mx_done[wt][warp & 3]);
+        else softmax_row<D, false>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, &bars->mx_done[wt][warp & 3]);
         if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
           // O holds PV up to tile j-1 (complete: QK(j) was issued after PV(j-1)), and PV(j)
           // waits for this warp's arrive below.
@@ -671,7 +634,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           uint32_t o[32];
           tmem_ld32(o_tm + cc * 32, o);
           tmem_ld_wait(o);
-          if (qrow < N) {
+          if (MODE == kOutF32 && qrow < N) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out_any) +
+                                                    (static_cast<size_t>(bh) * N + qrow) * D + cc * 32);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(o[4 * v + 0]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
+                                   __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
+          } else if (qrow < N) {
             uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -690,9 +660,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // empty, and its rows are written as zeros
       const int qrow = (wt == 0 ? tq0 : tq1) * kBM + row;
       if ((wt == 0 || has1) && qrow < N) {
-        uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * N + qrow) * D);
+        constexpr int kBytes = MODE == kOutF32 ? 4 : 2;
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(out_any) +
+                                              (static_cast<size_t>(bh) * N + qrow) * D * kBytes);
 #pragma unroll
-        for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0, 0, 0, 0);
+        for (int v = 0; v < D * kBytes / 16; ++v) dst[v] = make_uint4(0, 0, 0, 0);
       }
     }
   }

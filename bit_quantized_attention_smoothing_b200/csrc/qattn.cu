@@ -192,9 +192,10 @@ qattn_status run_smooth_quant(const void* q, const void* k, int B, int H, int Hk
   return launch_status();
 }
 
-// q is int8 (with q_scale) or, for QF16, the fp16 Q that the kernel quantizes itself.  DUMP:
-// the score-dumping instantiation, one CTA per Q-tile pair dump->pair0 .. of head dump->bh.
-template <int D, bool CAUSAL, bool QF16, bool DUMP = false>
+// q is int8 (with q_scale) or, for QF16, the fp16 Q that the kernel quantizes itself.  MODE
+// kDumpS: the score-dumping instantiation, one CTA per Q-tile pair dump->pair0 .. of head
+// dump->bh; kOutF32: out is fp32.
+template <int D, bool CAUSAL, bool QF16, int MODE = kOutF16>
 qattn_status run_attn(const void* q, const float* q_scale, const int8_t* k_i8,
                       const float* k_scale, const void* v, void* out, int B, int H, int Hkv,
                       int N, cudaStream_t st, const int* kv_list = nullptr,
@@ -207,7 +208,8 @@ qattn_status run_attn(const void* q, const float* q_scale, const int8_t* k_i8,
       !make_v_map(&tv, v, D, N, static_cast<long long>(B) * Hkv))
     return QATTN_ERR_CUDA;
   using Cfg = AttnCfg<D>;
-  auto kern = attn_fwd_kernel<D, CAUSAL, QF16, DUMP>;
+  constexpr bool DUMP = MODE == kDumpS;
+  auto kern = attn_fwd_kernel<D, CAUSAL, QF16, MODE>;
   // The kernel moves registers between its warpgroups with setmaxnreg; the split adds up only if
   // the launch allocates exactly kAttnLaunchRegs per thread, so never launch it otherwise.
   static int regs_checked = 0;
@@ -226,20 +228,20 @@ qattn_status run_attn(const void* q, const float* q_scale, const int8_t* k_i8,
   const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   kern<<<static_cast<unsigned>(grid), kAttnThreads, Cfg::kSmemBytes, st>>>(
       tq, tk, tv, q_scale, QF16 ? static_cast<const uint16_t*>(q) : nullptr, kv_list, kv_count, k_scale,
-      static_cast<__half*>(out), B, H, Hkv, N, scale_log2, dump ? *dump : ScoreDump{});
+      out, B, H, Hkv, N, scale_log2, dump ? *dump : ScoreDump{});
   return launch_status();
 }
 
-template <bool QF16>
+template <bool QF16, int MODE = kOutF16>
 qattn_status dispatch_attn(const void* q, const float* q_scale, const int8_t* k_i8,
                            const float* k_scale, const void* v, void* out, int B, int H, int Hkv,
                            int N, int d, int causal, cudaStream_t st, const int* kv_list = nullptr,
                            const int* kv_count = nullptr) {
   if (d == 128)
-    return causal ? run_attn<128, true, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, kv_list, kv_count)
-                  : run_attn<128, false, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, kv_list, kv_count);
-  return causal ? run_attn<64, true, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, kv_list, kv_count)
-                : run_attn<64, false, QF16>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, kv_list, kv_count);
+    return causal ? run_attn<128, true, QF16, MODE>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, kv_list, kv_count)
+                  : run_attn<128, false, QF16, MODE>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, kv_list, kv_count);
+  return causal ? run_attn<64, true, QF16, MODE>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, kv_list, kv_count)
+                : run_attn<64, false, QF16, MODE>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, kv_list, kv_count);
 }
 
 // Block selection workspace: query-block means, key-tile means, scores (binary64).
@@ -505,6 +507,19 @@ qattn_status qattn_attn_quantized(const int8_t* q_i8, const float* q_scale, cons
   if ((s = device_ok()) != QATTN_OK) return s;
   return dispatch_attn<false>(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, d, causal,
                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+qattn_status qattn_attn_quantized_f32(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                                      const float* k_scale, const void* v, float* out, int B,
+                                      int H, int Hkv, int N, int d, int causal,
+                                      qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q_i8, q_scale, k_i8, k_scale, v, out);
+  if (s != QATTN_OK) return s;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  return dispatch_attn<false, kOutF32>(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, d,
+                                       causal, reinterpret_cast<cudaStream_t>(stream));
 }
 
 qattn_status qattn_smooth_k(const void* k, int B, int Hkv, int N, int d, int8_t* k_i8,
@@ -819,11 +834,11 @@ qattn_status qattn_debug_qk_int32(const int8_t* q_i8, const int8_t* k_i8, int32_
   if (s == QATTN_OK) {
 #define QATTN_DUMP_ARGS q_i8, qs, k_i8, ks, w, w + vb, B, H, Hkv, N, st, nullptr, nullptr, &dump, pairs
     if (d == 128)
-      s = causal ? run_attn<128, true, false, true>(QATTN_DUMP_ARGS)
-                 : run_attn<128, false, false, true>(QATTN_DUMP_ARGS);
+      s = causal ? run_attn<128, true, false, kDumpS>(QATTN_DUMP_ARGS)
+                 : run_attn<128, false, false, kDumpS>(QATTN_DUMP_ARGS);
     else
-      s = causal ? run_attn<64, true, false, true>(QATTN_DUMP_ARGS)
-                 : run_attn<64, false, false, true>(QATTN_DUMP_ARGS);
+      s = causal ? run_attn<64, true, false, kDumpS>(QATTN_DUMP_ARGS)
+                 : run_attn<64, false, false, kDumpS>(QATTN_DUMP_ARGS);
 #undef QATTN_DUMP_ARGS
   }
   if (cudaFreeAsync(ws, st) != cudaSuccess && s == QATTN_OK) s = QATTN_ERR_CUDA;

@@ -8,8 +8,10 @@
 //  * mean = (float)((double)sum / (N * 2^24)) with correctly rounded operations;
 //  * K' = (float)K - mean, amax, scale = amax / 127 are single correctly rounded binary32 ops;
 //  * code = rint(x / scale): computed as rint(x * (1/scale)), which equals rint(x / scale) unless
-//    x / scale lies within 2^-13 of a half-integer (the two quotients differ by less than 2^-16
-//    for |x / scale| <= 128); those rare elements take the correctly rounded division.
+//    x / scale lies within 2^-13 of a half-integer: for |x / scale| <= 127 the product carries two
+//    roundings of relative size <= 2^-24 each (< 2^-16 absolute) and the correctly rounded
+//    quotient one more (< 2^-17), so the two differ by less than 2^-15; those rare elements take
+//    the correctly rounded division.
 // Build without fast-math so that division, reciprocal and conversions round to nearest-even
 // and subnormals are kept.
 #pragma once

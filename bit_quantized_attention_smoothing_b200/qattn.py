@@ -27,7 +27,7 @@ KBLOCK = 64
 EXPORTS = [
     "qattn_status_string", "qattn_version", "qattn_smooth_quant_workspace", "qattn_smooth_quant",
     "qattn_smooth_quant_noalloc",
-    "qattn_attn_quantized", "qattn_smooth_k", "qattn_attn_fused_q",
+    "qattn_attn_quantized", "qattn_attn_quantized_f32", "qattn_smooth_k", "qattn_attn_fused_q",
     "qattn_block_select_workspace", "qattn_block_select", "qattn_attn_quantized_sparse",
     "qattn_forward_sparse",
     "qattn_forward_workspace", "qattn_forward_ws", "qattn_forward",
@@ -71,6 +71,8 @@ def _lib():
         L.qattn_smooth_quant_noalloc.restype = i
         L.qattn_attn_quantized.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, P]
         L.qattn_attn_quantized.restype = i
+        L.qattn_attn_quantized_f32.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, P]
+        L.qattn_attn_quantized_f32.restype = i
         L.qattn_smooth_k.argtypes = [P, i, i, i, i, P, P, P, P, sz, P]
         L.qattn_smooth_k.restype = i
         L.qattn_attn_fused_q.argtypes = [P, P, P, P, P, i, i, i, i, i, i, P]
@@ -196,6 +198,17 @@ def qattn_attn_quantized(q_i8, q_scale, k_i8, k_scale, v, out=None, causal=False
     st = _lib().qattn_attn_quantized(_p(q_i8), _p(q_scale), _p(k_i8), _p(k_scale), _p(v), _p(out),
                                      B, H, Hkv, N, d, int(bool(causal)), _stream(stream))
     _check("qattn_attn_quantized", st)
+    return out
+
+
+def qattn_attn_quantized_f32(q_i8, q_scale, k_i8, k_scale, v, out=None, causal=False, stream=None):
+    """qattn_attn_quantized with an fp32 output (the fp16 output is exactly its nearest fp16)."""
+    B, H, Hkv, N, d = _dims(q_i8, k_i8)
+    out = torch.empty(B, H, N, d, dtype=torch.float32, device=v.device) if out is None else out
+    st = _lib().qattn_attn_quantized_f32(_p(q_i8), _p(q_scale), _p(k_i8), _p(k_scale), _p(v),
+                                         _p(out), B, H, Hkv, N, d, int(bool(causal)),
+                                         _stream(stream))
+    _check("qattn_attn_quantized_f32", st)
     return out
 
 

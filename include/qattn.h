@@ -109,6 +109,16 @@ qattn_status qattn_attn_quantized(const int8_t* q_i8, const float* q_scale, cons
                                   const float* k_scale, const void* v, void* out, int B, int H,
                                   int Hkv, int N, int d, int causal, qattn_stream_t stream);
 
+/* qattn_attn_quantized with the output O = sum_j P_j V_j / l in fp32 (out: device float
+ * [B][H][N][d]) instead of fp16: the same kernel and arithmetic up to its last step, so
+ * qattn_attn_quantized's fp16 output is exactly this output rounded to the nearest fp16.  For
+ * callers that keep the attention in fp32, and for checking the attention's value apart from the
+ * rounding of the fp16 output type.  Errors as qattn_attn_quantized. */
+qattn_status qattn_attn_quantized_f32(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                                      const float* k_scale, const void* v, float* out, int B,
+                                      int H, int Hkv, int N, int d, int causal,
+                                      qattn_stream_t stream);
+
 /* ------------------------------------------------------------------------------------------
  * Block-sparse attention.  The page "ThriftAttention: Selective Mixed Precision for
  * Long-Context FP4 Attention" (technical summary, method, heuristic block selection) rates each
