@@ -122,15 +122,16 @@ qattn_status launch_attn_nvfp4(const CUtensorMap* maps, const uint8_t* q_sf, con
                                const float* v_g, const void* q16, const float* k_mean,
                                const int* kv_list, const int* kv_count, void* out, int B, int H,
                                int Hkv, int N, int Np, cudaStream_t st) {
-  // 140 KB of shared memory keeps one CTA (and its 512 tensor-memory columns) per SM.
-  const int smem = 140 * 1024;
-  static_assert(Fp4AttnCfg<D>::kSmemUsed <= 140 * 1024, "shared memory");
+  // One CTA per SM (its 512 tensor-memory columns); at d = 128 the double-buffered FP4 and fp16
+  // K/V tiles take ~211 KB of shared memory.
+  const int smem = Fp4AttnCfg<D>::kSmemUsed;
+  static_assert(Fp4AttnCfg<D>::kSmemUsed <= 227 * 1024, "shared memory");
   auto kern = attn_nvfp4_kernel<D, CAUSAL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return QATTN_ERR_CUDA;
   const dim3 grid((N + 127) / 128, B * H);
   const float sl2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-  kern<<<grid, 128, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], q_sf, k_sf,
+  kern<<<grid, kFp4Threads, smem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], q_sf, k_sf,
                                 vt_sf, q_g, k_g, v_g, static_cast<const uint16_t*>(q16), k_mean,
                                 kv_list, kv_count, static_cast<__half*>(out), H, Hkv, N, Np, sl2);
   return launch_status();
@@ -858,6 +859,8 @@ qattn_status qattn_attn_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales, c
   if (kv_list != nullptr && (s = check_ptrs(q, k, v, k_mean, kv_list, kv_count)) != QATTN_OK)
     return s;
   if (static_cast<long long>(B) * H > 65535) return QATTN_ERR_UNSUPPORTED;
+  // promotion lists index at most 1024 key tiles (N <= 131072, the selection's limit)
+  if (kv_list != nullptr && (N + 127) / 128 > Fp4AttnCfg<128>::kMaxTiles) return QATTN_ERR_UNSUPPORTED;
   if ((s = device_ok()) != QATTN_OK) return s;
   return dispatch_attn_nvfp4(q_codes, q_scales, q_g, k_codes, k_scales, k_g, vt_codes, vt_scales,
                              v_g, q, k, v, k_mean, kv_list, kv_count, out, B, H, Hkv, N, d, causal,

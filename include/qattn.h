@@ -268,8 +268,9 @@ qattn_status qattn_quant_nvfp4(const void* x, const float* mean, int S, int R, i
  * k_mean) over B*Hkv slices, vt_* along the rows (transposed, Np = N rounded up to 128) over B*Hkv
  * slices.  With kv_list == NULL every tile runs in FP4 and q, k, v, k_mean, kv_count are not read;
  * otherwise q [B][H][N][d], k and v [B][Hkv][N][d] are the fp16 inputs, k_mean float [B*Hkv][d],
- * kv_list / kv_count as qattn_block_select writes them.  Same checks and errors as
- * qattn_attn_quantized; B * H <= 65535. */
+ * kv_list / kv_count as qattn_block_select writes them (a count above the row's ceil(N/128)
+ * entries is read as that many).  Same checks and errors as qattn_attn_quantized; B * H <= 65535;
+ * with kv_list, N <= 131072 (else QATTN_ERR_UNSUPPORTED). */
 qattn_status qattn_attn_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales, const float* q_g,
                               const uint8_t* k_codes, const uint8_t* k_scales, const float* k_g,
                               const uint8_t* vt_codes, const uint8_t* vt_scales, const float* v_g,
