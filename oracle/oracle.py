@@ -87,6 +87,15 @@ def lib():
         L.oracle_attention_nvfp4.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P,
                                              i, i, i, i, i, i, i, P, P, ctypes.c_long, P, P]
         L.oracle_attention_nvfp4.restype = i
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_decode.restype = ctypes.c_double
+        L.oracle_quant_v_fp8.argtypes = [P, i, i, i, P, P]
+        L.oracle_quant_v_fp8.restype = i
+        L.oracle_attention_pv8.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, P, P,
+                                           ctypes.c_long, P, P]
+        L.oracle_attention_pv8.restype = i
         _lib = L
     return _lib
 
@@ -432,3 +441,60 @@ def attention_nvfp4(qn, kn, vn, B, H, Hkv, N, d, causal, rows=None, promote=None
     if rc != 0:
         raise ValueError("oracle_attention_nvfp4: bad argument")
     return out, slack
+
+
+# ---- adaptive quantization: the FP8 (E4M3) P V variant (the C file states the readings) ----
+
+def e4m3_encode(x: float) -> int:
+    return int(lib().oracle_e4m3_encode(float(x)))
+
+
+def e4m3_decode(code: int) -> float:
+    return lib().oracle_e4m3_decode(int(code))
+
+
+def e4m3_decode_array(codes) -> np.ndarray:
+    """Values of an array of E4M3 bytes (float64), by the oracle's decoder."""
+    table = np.array([e4m3_decode(c) for c in range(256)], dtype=np.float64)
+    return table[np.asarray(codes, dtype=np.uint8)]
+
+
+def quant_v_fp8(v):
+    """E4M3 quantization of fp16 v [S, R, C] per slice, transposed: (codes uint8 [S, C, Rp],
+    scale float32 [S]), Rp = R rounded up to 128."""
+    v = _bits16(v)
+    S, R, C = v.shape
+    Rp = -(-R // 128) * 128
+    codes = np.zeros((S, C, Rp), dtype=np.uint8)
+    scale = np.zeros(S, dtype=np.float32)
+    assert lib().oracle_quant_v_fp8(_ptr(v), S, R, C, _ptr(codes), _ptr(scale)) == 0
+    return codes, scale
+
+
+def attention_pv8(q_i8, q_scale, k_i8, k_scale, vt8, v_scale, B, H, Hkv, N, d, causal,
+                  rows=None):
+    """Rows of the attention with INT8 Q K^T and E4M3 P V (float64 [nrows, d]) and the per-row
+    slack for E4M3 decisions near a tie.  vt8, v_scale as quant_v_fp8 returns them over the
+    B*Hkv slices."""
+    row_bh, row_i = all_rows(B, H, N) if rows is None else rows
+    row_bh = np.ascontiguousarray(row_bh, dtype=np.int64)
+    row_i = np.ascontiguousarray(row_i, dtype=np.int64)
+    vt8 = np.ascontiguousarray(vt8, dtype=np.uint8)
+    Np = vt8.shape[-1]
+    out = np.zeros((row_bh.size, d), dtype=np.float64)
+    slack = np.zeros(row_bh.size, dtype=np.float64)
+    assert lib().oracle_attention_pv8(
+        _ptr(np.ascontiguousarray(q_i8, dtype=np.int8)), _ptr(np.ascontiguousarray(q_scale, dtype=np.float32)),
+        _ptr(np.ascontiguousarray(k_i8, dtype=np.int8)), _ptr(np.ascontiguousarray(k_scale, dtype=np.float32)),
+        _ptr(vt8), _ptr(np.ascontiguousarray(v_scale, dtype=np.float32)), B, H, Hkv, N, Np, d,
+        1 if causal else 0, _ptr(row_bh), _ptr(row_i), row_bh.size, _ptr(out), _ptr(slack)) == 0
+    return out, slack
+
+
+def forward_pv8(q, k, v, B, H, Hkv, N, d, causal, rows=None):
+    """The FP8 P V variant's whole path: smoothing + INT8 quantization of Q and K, E4M3 V, then
+    the attention rows; returns (out, slack)."""
+    sq = smooth_quant(q, k, B, H, Hkv, N, d)
+    vt8, vs = quant_v_fp8(_bits16(v).reshape(B * Hkv, N, d))
+    return attention_pv8(sq["q_i8"], sq["q_scale"], sq["k_i8"], sq["k_scale"], vt8, vs, B, H,
+                         Hkv, N, d, causal, rows=rows)

@@ -778,3 +778,158 @@ int oracle_attention_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales, cons
     free(acc);
     return 0;
 }
+
+/* ------------------------------------------------------------------------------------------------
+ * Adaptive quantization (SageAttention summary page, aibr.jp/archives/102657: the dialogue and
+ * sec. 2-4 -- the quantization strength is chosen per layer or head, so that the important parts
+ * keep more precision while the others run faster; +11.7 % speed without metric loss).  The page
+ * names no variants.  The coarser variant here keeps the INT8 Q K^T and runs P V in FP8 E4M3
+ * (twice the FP16 tensor rate on Blackwell) instead of FP16; the choice between the two is made
+ * per (batch, kv head) by calibration.  Readings:
+ *   - V in E4M3 per (batch, kv head) slice: amax = max |v|, sV = amax / 448 (binary32 division;
+ *     448 is the largest E4M3 value), code = E4M3(v / sV) with binary32 division, nearest-even,
+ *     saturating at 448; amax == 0 gives sV = 0 and codes 0; a zero code is +0 (0x00) whatever
+ *     the sign of the input.  Stored transposed ([slice][channel][Np] bytes, Np = N rounded up to
+ *     128, zero padding), the K-major operand of the P V product.
+ *   - P in E4M3 follows FlashAttention's online softmax over key tiles of 128 (page sec. 4):
+ *     per tile the maximum t of the scaled scores of the tile's visible keys, m' = max(m, t); if
+ *     m' > m the accumulated O and l are scaled by 2^(m - m') and m = m'; then per key
+ *     p = 2^(y), y = S_int * c + (8 - m) (one binary32 fused multiply-add; c = (sQ * sK) * sl2 in
+ *     binary32, sl2 = binary32(log2(e) / sqrt(d))), so that p <= 2^8 < 448; p^ = E4M3(p);
+ *     l += p^; O += p^ v^ with v^ the E4M3 code values; out = O * sV / l.  The scaled maximum of
+ *     a 64-key scale block is (max S_int over its visible keys) * c, one binary32 product.
+ *   - The GPU computes 2^(y) with MUFU ex2 (binary32, a few ulp), so an E4M3 decision taken
+ *     within a relative 2^-16 of a rounding tie may go the other way there: for each output row
+ *     the oracle returns a slack, the sum over such decisions of one E4M3 step times
+ *     (max |v^| sV + max |out|) / l.
+ * ---------------------------------------------------------------------------------------------- */
+
+/* E4M3 byte of x (sign bit 7, then the unsigned byte of |x|), nearest-even, saturating at 448;
+ * a zero magnitude is +0. */
+uint8_t oracle_e4m3_encode(float x) {
+    uint8_t mag = oracle_ue4m3_encode(fabsf(x));
+    if (mag == 0) return 0;
+    return (x < 0.0f) ? (uint8_t)(mag | 0x80) : mag;
+}
+
+double oracle_e4m3_decode(uint8_t code) {
+    double v = oracle_ue4m3_decode((uint8_t)(code & 0x7F));
+    return (code & 0x80) ? -v : v;
+}
+
+/* v: fp16 [S][R][C]; codes [S][C][Rp] (Rp = R rounded up to 128, rows R .. Rp-1 zero);
+ * scale [S].  Returns 0, or -1 on a bad argument. */
+int oracle_quant_v_fp8(const uint16_t* v, int S, int R, int C, uint8_t* codes, float* scale) {
+    if (S < 1 || R < 1 || C < 1) return -1;
+    const long Rp = (R + 127) / 128 * 128;
+    for (long s = 0; s < S; ++s) {
+        float amax = 0.0f;
+        for (long r = 0; r < R; ++r)
+            for (int c = 0; c < C; ++c) {
+                float a = fabsf((float)oracle_f16_to_f64(v[(s * R + r) * C + c]));
+                if (a > amax) amax = a;
+            }
+        const float sv = amax / 448.0f;
+        scale[s] = sv;
+        for (int c = 0; c < C; ++c)
+            for (long r = 0; r < Rp; ++r) {
+                uint8_t code = 0;
+                if (r < R && amax > 0.0f)
+                    code = oracle_e4m3_encode((float)oracle_f16_to_f64(v[(s * R + r) * C + c]) / sv);
+                codes[(s * C + c) * Rp + r] = code;
+            }
+    }
+    return 0;
+}
+
+/* E4M3 code of p >= 0 and whether a relative perturbation of 2^-16 could change it; *step is
+ * the distance between the two codes that perturbation can give. */
+static uint8_t e4m3_with_risk(float p, double* step) {
+    const double d = ldexp(1.0, -16);
+    const uint8_t lo = oracle_ue4m3_encode((float)(p * (1.0 - d)));
+    const uint8_t hi = oracle_ue4m3_encode((float)(p * (1.0 + d)));
+    *step = (lo != hi) ? oracle_ue4m3_decode(hi) - oracle_ue4m3_decode(lo) : 0.0;
+    return oracle_ue4m3_encode(p);
+}
+
+/* Attention with INT8 Q K^T (as oracle_attention_quantized) and FP8 P V, row by row in the online
+ * order above.  q_i8 [B*H][N][d], q_scale [B*H][ceil(N/128)], k_i8 [B*Hkv][N][d],
+ * k_scale [B*Hkv][ceil(N/64)], vt8 [B*Hkv][d][Np], v_scale [B*Hkv].  Rows (row_bh[r], row_i[r]);
+ * out [nrows][d], slack [nrows].  Returns 0, or -1 on a bad argument. */
+int oracle_attention_pv8(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                         const float* k_scale, const uint8_t* vt8, const float* v_scale, int B,
+                         int H, int Hkv, int N, int Np, int d, int causal, const long* row_bh,
+                         const long* row_i, long nrows, double* out, double* slack) {
+    if (B < 1 || H < 1 || Hkv < 1 || N < 1 || H % Hkv || Np < N || Np % 128) return -1;
+    const float sl2 = (float)(1.4426950408889634 / sqrt((double)d));
+    const int nqb = (N + ORACLE_QBLOCK - 1) / ORACLE_QBLOCK, nkb = (N + ORACLE_KBLOCK - 1) / ORACLE_KBLOCK;
+    double* acc = (double*)malloc(sizeof(double) * d);
+    int32_t s[128];
+    double ph[128], step[128];
+    for (long r = 0; r < nrows; ++r) {
+        const long bh = row_bh[r], i = row_i[r];
+        const long b = bh / H, h = bh % H, bg = b * Hkv + h / (H / Hkv);
+        const int8_t* qrow = q_i8 + (bh * N + i) * (long)d;
+        const float sq = q_scale[bh * nqb + i / ORACLE_QBLOCK];
+        const long last = causal ? i : N - 1;
+        float m = -INFINITY;
+        double l = 0.0, rv = 0.0, rp = 0.0, vmax = 0.0;
+        for (int c = 0; c < d; ++c) acc[c] = 0.0;
+        for (int c = 0; c < d; ++c)
+            for (long j = 0; j <= last; ++j) {
+                double a = fabs(oracle_e4m3_decode(vt8[(bg * d + c) * (long)Np + j]));
+                if (a > vmax) vmax = a;
+            }
+        for (long t0 = 0; t0 <= last; t0 += 128) {
+            const int n = (int)((last - t0 + 1) < 128 ? (last - t0 + 1) : 128);   /* visible keys */
+            float cb[2], t = -INFINITY;
+            for (int blk = 0; blk < 2; ++blk) {
+                const long kb = (t0 + 64 * blk) / ORACLE_KBLOCK;
+                cb[blk] = kb < nkb ? (sq * k_scale[bg * nkb + kb]) * sl2 : 0.0f;
+                int32_t mx = 0;
+                int any = 0;
+                for (int j = 64 * blk; j < 64 * blk + 64 && j < n; ++j) {
+                    int32_t a = 0;
+                    const int8_t* krow = k_i8 + (bg * N + t0 + j) * (long)d;
+                    for (int c = 0; c < d; ++c) a += (int32_t)qrow[c] * (int32_t)krow[c];
+                    s[j] = a;
+                    if (!any || a > mx) mx = a;
+                    any = 1;
+                }
+                if (any) {
+                    const float tb = (float)mx * cb[blk];
+                    if (tb > t) t = tb;
+                }
+            }
+            if (t > m) {
+                const double alpha = (m == -INFINITY) ? 0.0 : exp2((double)m - (double)t);
+                l *= alpha;
+                rv *= alpha;
+                rp *= alpha;
+                for (int c = 0; c < d; ++c) acc[c] *= alpha;
+                m = t;
+            }
+            const float g = 8.0f - m;
+            for (int j = 0; j < n; ++j) {
+                const float y = fmaf((float)s[j], cb[j / 64], g);
+                const float p = (float)exp2((double)y);
+                ph[j] = oracle_ue4m3_decode(e4m3_with_risk(p, &step[j]));
+            }
+            for (int j = 0; j < n; ++j) {
+                l += ph[j];
+                for (int c = 0; c < d; ++c)
+                    acc[c] += ph[j] * oracle_e4m3_decode(vt8[(bg * d + c) * (long)Np + t0 + j]);
+                rv += step[j] * vmax;
+                rp += step[j];
+            }
+        }
+        double omax = 0.0;
+        for (int c = 0; c < d; ++c) {
+            out[r * d + c] = acc[c] * (double)v_scale[bg] / l;
+            if (fabs(out[r * d + c]) > omax) omax = fabs(out[r * d + c]);
+        }
+        slack[r] = (rv * (double)v_scale[bg] + rp * omax) / l;
+    }
+    free(acc);
+    return 0;
+}
