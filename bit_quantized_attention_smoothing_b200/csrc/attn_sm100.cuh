@@ -50,6 +50,17 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: O is rescaled only whe
 // 131072 keys per row, P normalised to 1 loses enough weight in fp16 subnormals to cost ~4e-3 of
 // output accuracy; the offset cancels in O / l.
 constexpr float kPOffset = 7.0f;
+// The FP8 P V variant (adaptive quantization): the running maximum moves only when it grows by
+// more than kRescaleThreshold8, and P = 2^(x - m + kPOffset8) <= 2^(4 + 4) = 256, inside E4M3's
+// 448 (keys down to ~2^-10 of the running maximum stay normal E4M3 numbers).
+constexpr float kRescaleThreshold8 = 4.0f;
+constexpr float kPOffset8 = 4.0f;
+
+// P V variants of the attention kernel: FP16 P and V (the product), FP8 E4M3 P and V, or the
+// variant chosen per (batch, kv head) group by a table (adaptive quantization).
+constexpr int kPvF16 = 0;
+constexpr int kPvF8 = 1;
+constexpr int kPvTable = 2;
 
 template <int D>
 struct AttnCfg {
@@ -69,6 +80,9 @@ struct AttnCfg {
   static constexpr uint32_t kSboQK = 8 * D;
   // V: MN-major fp16 operand, 64-column (128-byte) swizzled boxes of 128 rows.
   static constexpr uint32_t kVBox = kBN * 128;  // bytes of one 64-column box
+  // FP8 variant: V^T tile of D channel rows x 128 keys (E4M3 bytes, 128-byte swizzle), the K-major
+  // B operand of P V; it uses the first half of a V stage.
+  static constexpr int kV8Tile = D * kBN;
 };
 
 struct __align__(16) AttnBars {
@@ -150,7 +164,10 @@ static_assert(127 * 127 * 128 < (1 << 22), "biased score conversion range");
 // row's first 64 TMEM columns, and the row sum of the fp16-rounded P.  Once the first 64 keys'
 // P are stored, the warp arrives on mx_bar (the other Q tile's softmax waits for it).  MASK is a
 // compile-time switch so the unmasked steps carry no per-element tests.
-template <int D, bool MASK>
+// PV8 (the FP8 P V variant): the running max moves when it grows by more than 4, P =
+// 2^(x * c - m + 4) is rounded to E4M3, four keys per tensor-memory column (the lowest key in the
+// lowest byte) over the row's first 32 columns, and the row sum takes the E4M3 values.
+template <int D, bool MASK, bool PV8>
 __device__ __forceinline__ void softmax_row(uint32_t (&sr)[4][32], int lim, float c0, float c1,
                                             bool first, float& m, float& l, float& alpha,
                                             bool& need, uint32_t s_tm, uint64_t* mx_bar) {
@@ -173,45 +190,80 @@ __device__ __forceinline__ void softmax_row(uint32_t (&sr)[4][32], int lim, floa
   const float t = fmaxf(scaled_max(fmaxf(mx0, mx1) - kRoundMagic, c0),
                        scaled_max(fmaxf(mx2, mx3) - kRoundMagic, c1));
   const float mn = fmaxf(m, t);
-  need = mn > m + kRescaleThreshold;
+  need = mn > m + (PV8 ? kRescaleThreshold8 : kRescaleThreshold);
   alpha = 1.0f;
   if (need) {
     alpha = first ? 0.0f : ex2_approx(m - mn);
     m = mn;
     l *= alpha;
   }
-  const float g = kPOffset - m;
+  const float g = (PV8 ? kPOffset8 : kPOffset) - m;
   float acc0 = 0.0f, acc1 = 0.0f;
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {
     const float c = hf == 0 ? c0 : c1;
-    uint32_t pk[32];
+    if constexpr (PV8) {
+      uint32_t pk8[16];
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
+      for (int q = 0; q < 2; ++q) {
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        float x0, x1, y0, y1, p0, p1;
-        fadd2(x0, x1, __uint_as_float(sr[2 * hf + q][e]), __uint_as_float(sr[2 * hf + q][e + 1]),
-              -kRoundMagic, -kRoundMagic);
-        ffma2(y0, y1, x0, x1, c, g);
-        p0 = ex2_approx(y0);
-        p1 = ex2_approx(y1);
-        if (MASK) {
-          // -inf * 0 would be NaN for a zero-scale block: select instead
-          if (x0 == -INFINITY) p0 = 0.0f;
-          if (x1 == -INFINITY) p1 = 0.0f;
+        for (int e = 0; e < 32; e += 4) {
+          uint32_t* w = &sr[2 * hf + q][e];
+          float x0, x1, x2, x3, y0, y1, y2, y3;
+          fadd2(x0, x1, __uint_as_float(w[0]), __uint_as_float(w[1]), -kRoundMagic, -kRoundMagic);
+          fadd2(x2, x3, __uint_as_float(w[2]), __uint_as_float(w[3]), -kRoundMagic, -kRoundMagic);
+          ffma2(y0, y1, x0, x1, c, g);
+          ffma2(y2, y3, x2, x3, c, g);
+          float p0 = ex2_approx(y0), p1 = ex2_approx(y1), p2 = ex2_approx(y2), p3 = ex2_approx(y3);
+          if (MASK) {
+            if (x0 == -INFINITY) p0 = 0.0f;
+            if (x1 == -INFINITY) p1 = 0.0f;
+            if (x2 == -INFINITY) p2 = 0.0f;
+            if (x3 == -INFINITY) p3 = 0.0f;
+          }
+          uint16_t lo, hi;
+          asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(p1), "f"(p0));
+          asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(p3), "f"(p2));
+          pk8[q * 8 + (e >> 2)] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+          // the row sum takes the E4M3 values the P V product uses (exact in fp16)
+          uint32_t h01, h23;
+          asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h01) : "h"(lo));
+          asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h23) : "h"(hi));
+          acc0 = add_half2_f32(acc0, h01);
+          acc1 = add_half2_f32(acc1, h23);
         }
-        const uint32_t h2 = pack_half2(p0, p1);
-        pk[q * 16 + (e >> 1)] = h2;
-        // the row sum takes the fp16-rounded P that the P V product uses, so that O / l is a
-        // weighted mean of V with exactly those weights
-        if (e & 2) acc1 = add_half2_f32(acc1, h2);
-        else acc0 = add_half2_f32(acc0, h2);
       }
+      // keys 64 * hf .. 64 * hf + 63 -> P columns 16 * hf .. 16 * hf + 15
+      tmem_st32x16(s_tm + hf * 16, pk8);
+    } else {
+      uint32_t pk[32];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float x0, x1, y0, y1, p0, p1;
+          fadd2(x0, x1, __uint_as_float(sr[2 * hf + q][e]), __uint_as_float(sr[2 * hf + q][e + 1]),
+                -kRoundMagic, -kRoundMagic);
+          ffma2(y0, y1, x0, x1, c, g);
+          p0 = ex2_approx(y0);
+          p1 = ex2_approx(y1);
+          if (MASK) {
+            // -inf * 0 would be NaN for a zero-scale block: select instead
+            if (x0 == -INFINITY) p0 = 0.0f;
+            if (x1 == -INFINITY) p1 = 0.0f;
+          }
+          const uint32_t h2 = pack_half2(p0, p1);
+          pk[q * 16 + (e >> 1)] = h2;
+          // the row sum takes the fp16-rounded P that the P V product uses, so that O / l is a
+          // weighted mean of V with exactly those weights
+          if (e & 2) acc1 = add_half2_f32(acc1, h2);
+          else acc0 = add_half2_f32(acc0, h2);
+        }
+      }
+      // keys 64 * hf .. 64 * hf + 63 -> P columns 32 * hf .. 32 * hf + 31; all scores are in
+      // registers by now, so these columns are free
+      tmem_st32(s_tm + hf * 32, pk);
     }
-    // keys 64 * hf .. 64 * hf + 63 -> P columns 32 * hf .. 32 * hf + 31; all scores are in
-    // registers by now, so these columns are free
-    tmem_st32(s_tm + hf * 32, pk);
     if (hf == 0) {
       // half of the row's exponentials done: the other Q tile's softmax may start its step
       __syncwarp();
@@ -337,14 +389,18 @@ struct ScoreDump {
 // memory before the first QK^T (per-tile amax, scale = amax / 127, the same rounding as
 // quantize_kernel); otherwise int8 Q and its scales come from the smoothing + quantization pass
 // (tm_q, q_scale).  MODE: kOutF16, kDumpS (only its block-to-work mapping differs, see
-// ScoreDump) or kOutF32 (out points to fp32).
-template <int D, bool CAUSAL, bool QF16, int MODE = kOutF16>
+// ScoreDump) or kOutF32 (out points to fp32).  PVK: kPvF16 (P and V in fp16), kPvF8 (P and V in
+// E4M3: tm_v8 maps V^T in E4M3, v_scale its per-(batch, kv head) scale) or kPvTable (pv_variant[bg]
+// chooses per group, 1 = E4M3).
+template <int D, bool CAUSAL, bool QF16, int MODE = kOutF16, int PVK = kPvF16>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scale,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_v8,
+                    const float* __restrict__ q_scale,
                     const uint16_t* __restrict__ q16, const int* __restrict__ kv_list,
                     const int* __restrict__ kv_count,
-                    const float* __restrict__ k_scale, void* __restrict__ out_any, int B, int H,
+                    const float* __restrict__ k_scale, const float* __restrict__ v_scale,
+                    const uint8_t* __restrict__ pv_variant, void* __restrict__ out_any, int B, int H,
                     int Hkv, int N, float scale_log2, ScoreDump dump) {
   constexpr bool DUMP = MODE == kDumpS;
   __half* out = static_cast<__half*>(out_any);
@@ -380,6 +436,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int h = bh % H;
   const int g = h / (H / Hkv);
   const int bg = b * Hkv + g;
+  // the P V variant of this CTA's (batch, kv head) group
+  const bool pv8 = PVK == kPvF8 || (PVK == kPvTable && __ldg(pv_variant + bg) != 0);
   const int tq0 = 2 * pair, tq1 = 2 * pair + 1;
   const bool has1 = tq1 < nqt;
   // Block-sparse: the CTA streams only the key tiles listed for its 256 query rows (ascending;
@@ -440,13 +498,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int s = j % ST;
         const uint32_t u = static_cast<uint32_t>(j / ST);
         if (!mbar_wait(&bars->kv_empty[s], (u & 1u) ^ 1u, abort)) break;
-        mbar_arrive_expect_tx(&bars->kv_full[s], Cfg::kKTile + Cfg::kVTile);
+        mbar_arrive_expect_tx(&bars->kv_full[s], Cfg::kKTile + (pv8 ? Cfg::kV8Tile : Cfg::kVTile));
         const int kt = ktile(j);
         tma_load_3d(smem + Cfg::kOffK + s * Cfg::kKTile, &tm_k, &bars->kv_full[s], 0, kt * kBN, bg);
         uint8_t* vdst = smem + Cfg::kOffV + s * Cfg::kVTile;
+        if (pv8) {
+          tma_load_3d(vdst, &tm_v8, &bars->kv_full[s], kt * kBN, 0, bg);
+        } else {
 #pragma unroll
-        for (int x = 0; x < D / 64; ++x)
-          tma_load_3d(vdst + x * Cfg::kVBox, &tm_v, &bars->kv_full[s], x * 64, kt * kBN, bg);
+          for (int x = 0; x < D / 64; ++x)
+            tma_load_3d(vdst + x * Cfg::kVBox, &tm_v, &bars->kv_full[s], x * 64, kt * kBN, bg);
+        }
       }
     } else if (warp == kMmaWarp) {
       // ---------------------------------------------------------------- MMA issuer
@@ -463,6 +525,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t dq0 = smem_desc(smem_u32(smem + Cfg::kOffQ), 16, Cfg::kSboQK, Cfg::kSwQK);
       const uint64_t dk0 = smem_desc(smem_u32(smem + Cfg::kOffK), 16, Cfg::kSboQK, Cfg::kSwQK);
       const uint64_t dv0 = smem_desc(smem_u32(smem + Cfg::kOffV), Cfg::kVBox, 1024, kSwizzle128B);
+      // FP8 variant: V^T rows of 128 keys (128 bytes), 8-row swizzle atoms, K = 32 keys per MMA
+      constexpr uint32_t idv8 = idesc_f8_f32(kBM, D);
+      const uint64_t dv80 = smem_desc(smem_u32(smem + Cfg::kOffV), 16, 1024, kSwizzle128B);
       // a CTA whose lists hold no key tile (n_kv == 0: block-sparse lists with zero entries) has
       // nothing to multiply; its softmax warps write zero rows
       bool ok = n_kv > 0 &&
@@ -493,10 +558,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (!ok) continue;
           tc_fence_after();
           const uint32_t ts = tmem + w * 128, to = tmem + 256 + w * D;
-          if (j == 0) mma_f16_ts_warp(to, ts, dv, idv, 0u);
-          else mma_f16_ts_warp(to, ts, dv, idv, 1u);
+          if (pv8) {
+            const uint64_t dv8 = dv80 + static_cast<uint64_t>((s * Cfg::kVTile) >> 4);
+            mma_f8_ts_warp(to, ts, dv8, idv8, j == 0 ? 0u : 1u);
 #pragma unroll
-          for (int kk = 1; kk < kBN / 16; ++kk) mma_f16_ts_warp(to, ts + kk * 8, dv + kk * 128, idv, 1u);
+            for (int kk = 1; kk < kBN / 32; ++kk) mma_f8_ts_warp(to, ts + kk * 8, dv8 + 2 * kk, idv8, 1u);
+          } else {
+            if (j == 0) mma_f16_ts_warp(to, ts, dv, idv, 0u);
+            else mma_f16_ts_warp(to, ts, dv, idv, 1u);
+#pragma unroll
+            for (int kk = 1; kk < kBN / 16; ++kk) mma_f16_ts_warp(to, ts + kk * 8, dv + kk * 128, idv, 1u);
+          }
           mma_commit_warp(&bars->pv_done[w]);
           if (j + 1 < nw) {
             if (!next_ready) {
@@ -603,8 +675,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const bool masked = __any_sync(0xFFFFFFFFu, lim < kBN - 1);
         float alpha;
         bool need;
-        if (masked) softmax_row<D, true>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, &bars->mx_done[wt][warp & 3]);
-        else softmax_row<D, false>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, &bars->mx_done[wt][warp & 3]);
+        uint64_t* gate = &bars->mx_done[wt][warp & 3];
+        if (pv8) {
+          if (masked) softmax_row<D, true, true>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, gate);
+          else softmax_row<D, false, true>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, gate);
+        } else {
+          if (masked) softmax_row<D, true, false>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, gate);
+          else softmax_row<D, false, false>(sr, lim, c0, c1, j == 0, m, l, alpha, need, s_tm, gate);
+        }
         if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
           // O holds PV up to tile j-1 (complete: QK(j) was issued after PV(j-1)), and PV(j)
           // waits for this warp's arrive below.
@@ -627,7 +705,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ok = __all_sync(0xFFFFFFFFu, ok);
       tc_fence_after();
       if (ok) {
-        const float inv_l = 1.0f / l;
+        // the FP8 variant's O is in units of V's E4M3 codes: times its scale
+        const float inv_l = (pv8 ? __ldg(v_scale + bg) : 1.0f) / l;
         __half* orow = out + (static_cast<size_t>(bh) * N + qrow) * D;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {

@@ -17,6 +17,7 @@
 #include "block_sparse.cuh"
 #include "nvfp4.cuh"
 #include "fp4_sm100.cuh"
+#include "adaptive.cuh"
 
 namespace {
 
@@ -143,6 +144,12 @@ bool make_v_map(CUtensorMap* m, const void* base, int d, int N, long long outer)
                   CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// E4M3 V^T [outer][d][Np] bytes: tiles of d channel rows x 128 keys, 128-byte swizzle.
+bool make_v8_map(CUtensorMap* m, const void* base, int d, int Np, long long outer) {
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Np, d, outer, 128, d,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 // ---------------------------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------------------------
@@ -196,21 +203,36 @@ qattn_status run_smooth_quant(const void* q, const void* k, int B, int H, int Hk
 // q is int8 (with q_scale) or, for QF16, the fp16 Q that the kernel quantizes itself.  MODE
 // kDumpS: the score-dumping instantiation, one CTA per Q-tile pair dump->pair0 .. of head
 // dump->bh; kOutF32: out is fp32.
-template <int D, bool CAUSAL, bool QF16, int MODE = kOutF16>
+// The E4M3 operands of the FP8 P V variant (PVK kPvF8 or kPvTable): V^T codes, per-group scales and,
+// for kPvTable, the per-group variant table.
+struct Pv8Args {
+  const uint8_t* vt8 = nullptr;
+  const float* v_scale = nullptr;
+  const uint8_t* variant = nullptr;
+};
+
+template <int D, bool CAUSAL, bool QF16, int MODE = kOutF16, int PVK = kPvF16>
 qattn_status run_attn(const void* q, const float* q_scale, const int8_t* k_i8,
                       const float* k_scale, const void* v, void* out, int B, int H, int Hkv,
                       int N, cudaStream_t st, const int* kv_list = nullptr,
                       const int* kv_count = nullptr, const ScoreDump* dump = nullptr,
-                      int dump_pairs = 0) {
-  CUtensorMap tq, tk, tv;
+                      int dump_pairs = 0, Pv8Args pv = Pv8Args()) {
+  CUtensorMap tq, tk, tv, tv8;
   std::memset(&tq, 0, sizeof(tq));  // unused by the QF16 kernel
   if ((!QF16 && !make_i8_map(&tq, q, D, N, static_cast<long long>(B) * H)) ||
       !make_i8_map(&tk, k_i8, D, N, static_cast<long long>(B) * Hkv) ||
-      !make_v_map(&tv, v, D, N, static_cast<long long>(B) * Hkv))
+      (v != nullptr && !make_v_map(&tv, v, D, N, static_cast<long long>(B) * Hkv)))
     return QATTN_ERR_CUDA;
+  if (PVK != kPvF16) {
+    if (!make_v8_map(&tv8, pv.vt8, D, (N + 127) / 128 * 128, static_cast<long long>(B) * Hkv))
+      return QATTN_ERR_CUDA;
+    if (v == nullptr) tv = tv8;  // every group on the FP8 path: the fp16 map is never read
+  } else {
+    tv8 = tv;  // never read
+  }
   using Cfg = AttnCfg<D>;
   constexpr bool DUMP = MODE == kDumpS;
-  auto kern = attn_fwd_kernel<D, CAUSAL, QF16, MODE>;
+  auto kern = attn_fwd_kernel<D, CAUSAL, QF16, MODE, PVK>;
   // The kernel moves registers between its warpgroups with setmaxnreg; the split adds up only if
   // the launch allocates exactly kAttnLaunchRegs per thread, so never launch it otherwise.
   static int regs_checked = 0;
@@ -228,8 +250,8 @@ qattn_status run_attn(const void* q, const float* q_scale, const int8_t* k_i8,
   if (grid > 0x7FFFFFFFLL) return QATTN_ERR_UNSUPPORTED;
   const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   kern<<<static_cast<unsigned>(grid), kAttnThreads, Cfg::kSmemBytes, st>>>(
-      tq, tk, tv, q_scale, QF16 ? static_cast<const uint16_t*>(q) : nullptr, kv_list, kv_count, k_scale,
-      out, B, H, Hkv, N, scale_log2, dump ? *dump : ScoreDump{});
+      tq, tk, tv, tv8, q_scale, QF16 ? static_cast<const uint16_t*>(q) : nullptr, kv_list, kv_count,
+      k_scale, pv.v_scale, pv.variant, out, B, H, Hkv, N, scale_log2, dump ? *dump : ScoreDump{});
   return launch_status();
 }
 
@@ -243,6 +265,43 @@ qattn_status dispatch_attn(const void* q, const float* q_scale, const int8_t* k_
                   : run_attn<128, false, QF16, MODE>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, kv_list, kv_count);
   return causal ? run_attn<64, true, QF16, MODE>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, kv_list, kv_count)
                 : run_attn<64, false, QF16, MODE>(q, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, kv_list, kv_count);
+}
+
+// The attention on int8 Q and K with the FP8 P V variant for every group (PVK kPvF8) or per group
+// (kPvTable; v is the fp16 V for the groups on the FP16 path).
+template <int PVK>
+qattn_status dispatch_attn_pv8(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                               const float* k_scale, const void* v, Pv8Args pv, void* out, int B,
+                               int H, int Hkv, int N, int d, int causal, cudaStream_t st) {
+#define QATTN_PV_ARGS q_i8, q_scale, k_i8, k_scale, v, out, B, H, Hkv, N, st, nullptr, nullptr, nullptr, 0, pv
+  if (d == 128)
+    return causal ? run_attn<128, true, false, kOutF16, PVK>(QATTN_PV_ARGS)
+                  : run_attn<128, false, false, kOutF16, PVK>(QATTN_PV_ARGS);
+  return causal ? run_attn<64, true, false, kOutF16, PVK>(QATTN_PV_ARGS)
+                : run_attn<64, false, false, kOutF16, PVK>(QATTN_PV_ARGS);
+#undef QATTN_PV_ARGS
+}
+
+// E4M3 V: slice maxima, scales, transposed codes (arguments already checked).
+qattn_status dispatch_quant_v_fp8(const void* v, int S, int R, int C, uint8_t* vt8, float* scale,
+                                  cudaStream_t st) {
+  const uint16_t* vh = static_cast<const uint16_t*>(v);
+  if (cudaMemsetAsync(scale, 0, sizeof(float) * static_cast<size_t>(S), st) != cudaSuccess)
+    return QATTN_ERR_CUDA;
+  const long long nvec = static_cast<long long>(R) * C / 8;
+  long long gx = (nvec + 1023) / 1024;
+  const long long cap = (148LL * 16 + S - 1) / S;
+  if (gx > cap) gx = cap;
+  if (gx < 1) gx = 1;
+  nvfp4_amax_kernel<<<dim3(static_cast<unsigned>(gx), S), 256, 0, st>>>(
+      vh, nullptr, R, C, reinterpret_cast<unsigned*>(scale));
+  if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
+  v_fp8_scale_kernel<<<(S + 255) / 256, 256, 0, st>>>(scale, S);
+  if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
+  const int Rp = (R + 127) / 128 * 128;
+  const dim3 grid(Rp / kV8Tile, (C + kV8Tile - 1) / kV8Tile, S);
+  v_fp8_quant_kernel<<<grid, 256, 0, st>>>(vh, R, C, Rp, scale, vt8);
+  return launch_status();
 }
 
 // Block selection workspace: query-block means, key-tile means, scores (binary64).
@@ -995,6 +1054,152 @@ qattn_status qattn_quant_nvfp4(const void* x, const float* mean, int S, int R, i
   if ((s = device_ok()) != QATTN_OK) return s;
   return dispatch_quant_nvfp4(x, mean, S, R, C, along_rows, codes, scales, gscale,
                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+qattn_status qattn_quant_v_fp8(const void* v, int B, int Hkv, int N, int d, uint8_t* vt8,
+                              float* v_scale, qattn_stream_t stream) {
+  qattn_status s = check_shape(B, Hkv, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(v, vt8, v_scale);
+  if (s != QATTN_OK) return s;
+  if (static_cast<long long>(B) * Hkv > 65535) return QATTN_ERR_UNSUPPORTED;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  return dispatch_quant_v_fp8(v, B * Hkv, N, d, vt8, v_scale, reinterpret_cast<cudaStream_t>(stream));
+}
+
+qattn_status qattn_attn_quantized_pv8(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                                      const float* k_scale, const uint8_t* vt8,
+                                      const float* v_scale, void* out, int B, int H, int Hkv,
+                                      int N, int d, int causal, qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q_i8, q_scale, k_i8, k_scale, vt8, v_scale, out);
+  if (s != QATTN_OK) return s;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  Pv8Args pv;
+  pv.vt8 = vt8;
+  pv.v_scale = v_scale;
+  return dispatch_attn_pv8<kPvF8>(q_i8, q_scale, k_i8, k_scale, nullptr, pv, out, B, H, Hkv, N, d,
+                                  causal, reinterpret_cast<cudaStream_t>(stream));
+}
+
+namespace {
+
+// Workspace of the adaptive entry points: the INT8 path's operands, E4M3 V^T and its scales.
+struct AdaptiveLayout {
+  QuantLayout q;
+  size_t vt8, vscale, total;
+};
+
+AdaptiveLayout adaptive_layout(int B, int H, int Hkv, int N, int d) {
+  AdaptiveLayout L;
+  L.q = forward_layout(B, H, Hkv, N, d);
+  const size_t Np = (static_cast<size_t>(N) + 127) / 128 * 128;
+  L.vt8 = L.q.total;
+  L.vscale = align_up(L.vt8 + static_cast<size_t>(B) * Hkv * d * Np);
+  L.total = align_up(L.vscale + sizeof(float) * B * Hkv);
+  return L;
+}
+
+// Smoothing + INT8 quantization of Q and K and E4M3 V into workspace w.
+qattn_status adaptive_operands(const void* q, const void* k, const void* v, int B, int H, int Hkv,
+                               int N, int d, const AdaptiveLayout& L, uint8_t* w, cudaStream_t st) {
+  qattn_status s = dispatch_smooth_quant(
+      q, k, B, H, Hkv, N, d, reinterpret_cast<int8_t*>(w + L.q.q_i8),
+      reinterpret_cast<float*>(w + L.q.q_scale), reinterpret_cast<int8_t*>(w + L.q.k_i8),
+      reinterpret_cast<float*>(w + L.q.k_scale), nullptr, reinterpret_cast<long long*>(w + L.q.sums),
+      st);
+  if (s != QATTN_OK) return s;
+  return dispatch_quant_v_fp8(v, B * Hkv, N, d, w + L.vt8, reinterpret_cast<float*>(w + L.vscale), st);
+}
+
+}  // namespace
+
+qattn_status qattn_forward_adaptive(const void* q, const void* k, const void* v, void* out, int B,
+                                    int H, int Hkv, int N, int d, int causal,
+                                    const uint8_t* variant, qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q, k, v, out);
+  if (s != QATTN_OK) return s;
+  if (variant == nullptr) return QATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * Hkv > 65535) return QATTN_ERR_UNSUPPORTED;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const AdaptiveLayout L = adaptive_layout(B, H, Hkv, N, d);
+  void* ws = nullptr;
+  if ((s = pool_alloc(&ws, L.total, st)) != QATTN_OK) return s;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  s = adaptive_operands(q, k, v, B, H, Hkv, N, d, L, w, st);
+  if (s == QATTN_OK) {
+    Pv8Args pv;
+    pv.vt8 = w + L.vt8;
+    pv.v_scale = reinterpret_cast<const float*>(w + L.vscale);
+    pv.variant = variant;
+    s = dispatch_attn_pv8<kPvTable>(reinterpret_cast<const int8_t*>(w + L.q.q_i8),
+                                    reinterpret_cast<const float*>(w + L.q.q_scale),
+                                    reinterpret_cast<const int8_t*>(w + L.q.k_i8),
+                                    reinterpret_cast<const float*>(w + L.q.k_scale), v, pv, out, B,
+                                    H, Hkv, N, d, causal, st);
+  }
+  if (cudaFreeAsync(ws, st) != cudaSuccess && s == QATTN_OK) s = QATTN_ERR_CUDA;
+  return s;
+}
+
+qattn_status qattn_adaptive_calibrate(const void* q, const void* k, const void* v, int B, int H,
+                                      int Hkv, int N, int d, int causal, float tau,
+                                      uint8_t* variant, float* cosine, qattn_stream_t stream) {
+  qattn_status s = check_shape(B, H, Hkv, N, d);
+  if (s != QATTN_OK) return s;
+  s = check_ptrs(q, k, v, variant);
+  if (s != QATTN_OK) return s;
+  if (!(tau >= -1.0f && tau <= 2.0f)) return QATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * Hkv > 65535) return QATTN_ERR_UNSUPPORTED;
+  if ((s = device_ok()) != QATTN_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const AdaptiveLayout L = adaptive_layout(B, H, Hkv, N, d);
+  const size_t ob = align_up(sizeof(uint16_t) * static_cast<size_t>(B) * H * N * d);
+  const size_t G = static_cast<size_t>(B) * Hkv;
+  const size_t off_a = L.total, off_b = off_a + ob, off_acc = off_b + ob;
+  const size_t total = align_up(off_acc + sizeof(double) * 3 * G);
+  void* ws = nullptr;
+  if ((s = pool_alloc(&ws, total, st)) != QATTN_OK) return s;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  double* acc = reinterpret_cast<double*>(w + off_acc);
+  s = adaptive_operands(q, k, v, B, H, Hkv, N, d, L, w, st);
+  const int8_t* q_i8 = reinterpret_cast<const int8_t*>(w + L.q.q_i8);
+  const int8_t* k_i8 = reinterpret_cast<const int8_t*>(w + L.q.k_i8);
+  const float* q_s = reinterpret_cast<const float*>(w + L.q.q_scale);
+  const float* k_s = reinterpret_cast<const float*>(w + L.q.k_scale);
+  // both variants on the calibration input, then the cosine of their outputs per group
+  if (s == QATTN_OK)
+    s = dispatch_attn<false>(q_i8, q_s, k_i8, k_s, v, w + off_a, B, H, Hkv, N, d, causal, st);
+  if (s == QATTN_OK) {
+    Pv8Args pv;
+    pv.vt8 = w + L.vt8;
+    pv.v_scale = reinterpret_cast<const float*>(w + L.vscale);
+    s = dispatch_attn_pv8<kPvF8>(q_i8, q_s, k_i8, k_s, nullptr, pv, w + off_b, B, H, Hkv, N, d,
+                                 causal, st);
+  }
+  if (s == QATTN_OK && cudaMemsetAsync(acc, 0, sizeof(double) * 3 * G, st) != cudaSuccess)
+    s = QATTN_ERR_CUDA;
+  if (s == QATTN_OK) {
+    const long long per = static_cast<long long>(H / Hkv) * N * d;
+    long long gx = per / (256 * 64);
+    const long long cap = (148LL * 8 + static_cast<long long>(G) - 1) / static_cast<long long>(G);
+    if (gx > cap) gx = cap;
+    if (gx < 1) gx = 1;
+    group_cosine_parts_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(G)), 256, 0, st>>>(
+        reinterpret_cast<const __half*>(w + off_a), reinterpret_cast<const __half*>(w + off_b), per, acc);
+    s = launch_status();
+  }
+  if (s == QATTN_OK) {
+    choose_variant_kernel<<<static_cast<unsigned>((G + 255) / 256), 256, 0, st>>>(
+        acc, static_cast<int>(G), tau, variant, cosine);
+    s = launch_status();
+  }
+  if (cudaFreeAsync(ws, st) != cudaSuccess && s == QATTN_OK) s = QATTN_ERR_CUDA;
+  return s;
 }
 
 qattn_status qattn_check_device_status(qattn_stream_t stream) {

@@ -32,7 +32,9 @@ EXPORTS = [
     "qattn_forward_sparse",
     "qattn_forward_workspace", "qattn_forward_ws", "qattn_forward",
     "qattn_forward_host", "qattn_debug_qk_int32", "qattn_debug_wait_timeout",
-    "qattn_quant_nvfp4", "qattn_attn_nvfp4", "qattn_forward_nvfp4", "qattn_debug_qk_nvfp4", "qattn_check_device_status",
+    "qattn_quant_nvfp4", "qattn_attn_nvfp4", "qattn_forward_nvfp4", "qattn_debug_qk_nvfp4",
+    "qattn_quant_v_fp8", "qattn_attn_quantized_pv8", "qattn_adaptive_calibrate",
+    "qattn_forward_adaptive", "qattn_check_device_status",
 ]
 
 
@@ -106,6 +108,14 @@ def _lib():
         L.qattn_forward_nvfp4.restype = i
         L.qattn_debug_qk_nvfp4.argtypes = [P, P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, i, P]
         L.qattn_debug_qk_nvfp4.restype = i
+        L.qattn_quant_v_fp8.argtypes = [P, i, i, i, i, P, P, P]
+        L.qattn_quant_v_fp8.restype = i
+        L.qattn_attn_quantized_pv8.argtypes = [P, P, P, P, P, P, P, i, i, i, i, i, i, P]
+        L.qattn_attn_quantized_pv8.restype = i
+        L.qattn_adaptive_calibrate.argtypes = [P, P, P, i, i, i, i, i, i, ctypes.c_float, P, P, P]
+        L.qattn_adaptive_calibrate.restype = i
+        L.qattn_forward_adaptive.argtypes = [P, P, P, P, i, i, i, i, i, i, P, P]
+        L.qattn_forward_adaptive.restype = i
         L.qattn_check_device_status.argtypes = [P]
         L.qattn_check_device_status.restype = i
         _L = L
@@ -403,6 +413,55 @@ def qattn_debug_qk_nvfp4(q_nvfp4, k_nvfp4, B, H, Hkv, N, d, b, h, qt0, nqt, kt0,
                                      B, H, Hkv, N, d, b, h, qt0, nqt, kt0, nkt, _stream(stream))
     _check("qattn_debug_qk_nvfp4", st)
     return s_out
+
+
+def qattn_quant_v_fp8(v, stream=None):
+    """E4M3 V of the FP8 P V variant: v fp16 [B, Hkv, N, d] -> (vt8 uint8 [B*Hkv, d, Np],
+    v_scale float32 [B*Hkv]), Np = N rounded up to 128."""
+    B, Hkv, N, d = v.shape
+    Np = -(-N // 128) * 128
+    vt8 = torch.empty(B * Hkv, d, Np, dtype=torch.uint8, device=v.device)
+    vs = torch.empty(B * Hkv, dtype=torch.float32, device=v.device)
+    _check("qattn_quant_v_fp8", _lib().qattn_quant_v_fp8(_p(v), B, Hkv, N, d, _p(vt8), _p(vs),
+                                                          _stream(stream)))
+    return vt8, vs
+
+
+def qattn_attn_quantized_pv8(q_i8, q_scale, k_i8, k_scale, vt8, v_scale, out=None, causal=False,
+                             stream=None):
+    """Attention on int8 Q, K with P V in FP8 E4M3 (vt8, v_scale from qattn_quant_v_fp8)."""
+    B, H, Hkv, N, d = _dims(q_i8, k_i8)
+    out = torch.empty(B, H, N, d, dtype=torch.float16, device=q_i8.device) if out is None else out
+    st = _lib().qattn_attn_quantized_pv8(_p(q_i8), _p(q_scale), _p(k_i8), _p(k_scale), _p(vt8),
+                                         _p(v_scale), _p(out), B, H, Hkv, N, d,
+                                         int(bool(causal)), _stream(stream))
+    _check("qattn_attn_quantized_pv8", st)
+    return out
+
+
+def qattn_adaptive_calibrate(q, k, v, tau, causal=False, variant=None, cosine=None, stream=None):
+    """Per (batch, kv head) group: cosine of the FP8-P V output against the FP16-P V output on
+    this input, and variant = cosine >= tau.  Returns (variant uint8 [B*Hkv], cosine float32
+    [B*Hkv])."""
+    B, H, Hkv, N, d = _dims(q, k)
+    dev = q.device
+    variant = torch.empty(B * Hkv, dtype=torch.uint8, device=dev) if variant is None else variant
+    cosine = torch.empty(B * Hkv, dtype=torch.float32, device=dev) if cosine is None else cosine
+    st = _lib().qattn_adaptive_calibrate(_p(q), _p(k), _p(v), B, H, Hkv, N, d, int(bool(causal)),
+                                         float(tau), _p(variant), _p(cosine), _stream(stream))
+    _check("qattn_adaptive_calibrate", st)
+    return variant, cosine
+
+
+def qattn_forward_adaptive(q, k, v, variant, out=None, causal=False, stream=None):
+    """The forward with each (batch, kv head) group on the variant variant[b * Hkv + g] names
+    (0: FP16 P V, 1: FP8 P V); fp16 in, fp16 out."""
+    B, H, Hkv, N, d = _dims(q, k)
+    out = torch.empty_like(q) if out is None else out
+    st = _lib().qattn_forward_adaptive(_p(q), _p(k), _p(v), _p(out), B, H, Hkv, N, d,
+                                       int(bool(causal)), _p(variant), _stream(stream))
+    _check("qattn_forward_adaptive", st)
+    return out
 
 
 def qattn_debug_wait_timeout(limit_cycles: int, stream=None) -> int:

@@ -290,6 +290,55 @@ qattn_status qattn_forward_nvfp4(const void* q, const void* k, const void* v, vo
                                  qattn_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Adaptive quantization (SageAttention summary page, aibr.jp/archives/102657: dialogue and
+ * sec. 2-4 -- the quantization strength is chosen per layer or head, keeping precision where it
+ * matters and speed elsewhere; +11.7 % speed without metric loss on the page).  The page names no
+ * variants.  Here the choice is per (batch, kv head) group between the INT8 path above (FP16
+ * P V) and a coarser variant that keeps INT8 Q K^T and runs P V in FP8 E4M3 on the tensor cores
+ * (twice the FP16 rate).  FP8 variant: V is E4M3 per group (sV = max |v| / 448, code =
+ * E4M3(v / sV), nearest-even, saturating, transposed); P = 2^(x - m + 4) against the running
+ * maximum m, which moves (rescaling O and l) when the tile maximum exceeds it by more than 4, so
+ * P <= 256; P rounded to E4M3; l sums those values; out = O sV / l in fp16.
+ * ------------------------------------------------------------------------------------------ */
+
+/* E4M3 V for the FP8 variant: v fp16 [B][Hkv][N][d] -> vt8 [B*Hkv][d][Np] bytes (Np = N rounded
+ * up to 128; rows N .. Np-1 zero; a zero code is +0) and v_scale float [B*Hkv] (sV of each
+ * group).  Every binary32 step rounds once; codes and scales are a deterministic function of v.
+ * Errors as qattn_smooth_k; B * Hkv <= 65535. */
+qattn_status qattn_quant_v_fp8(const void* v, int B, int Hkv, int N, int d, uint8_t* vt8,
+                               float* v_scale, qattn_stream_t stream);
+
+/* qattn_attn_quantized with P V in FP8 (every group): q_i8 / q_scale / k_i8 / k_scale as
+ * qattn_smooth_quant writes them, vt8 / v_scale as qattn_quant_v_fp8 writes them; fp16 out
+ * [B][H][N][d].  P V runs as tcgen05.mma kind::f8f6f4 (E4M3 P from tensor memory, E4M3 V^T from
+ * shared memory, f32 accumulator).  Errors as qattn_attn_quantized. */
+qattn_status qattn_attn_quantized_pv8(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                                      const float* k_scale, const uint8_t* vt8,
+                                      const float* v_scale, void* out, int B, int H, int Hkv,
+                                      int N, int d, int causal, qattn_stream_t stream);
+
+/* Calibration of the adaptive choice on the given (calibration) input: both variants' outputs
+ * (FP16 P V and FP8 P V, on the same INT8 Q and K), then per (batch, kv head) group the cosine
+ * similarity of the two over the group's rows (its H / Hkv query heads, all N rows, d channels;
+ * binary64 sums); variant[g] = 1 (FP8 P V) when that cosine >= tau, else 0 (FP16 P V).
+ * variant: device uint8 [B*Hkv]; cosine: device float [B*Hkv] or NULL.  Workspace (operands and
+ * both outputs) from the library's per-device pool.  Errors: tau outside [-1, 2] or a NULL
+ * variant QATTN_ERR_INVALID_ARG; otherwise as qattn_forward; B * Hkv <= 65535. */
+qattn_status qattn_adaptive_calibrate(const void* q, const void* k, const void* v, int B, int H,
+                                      int Hkv, int N, int d, int causal, float tau,
+                                      uint8_t* variant, float* cosine, qattn_stream_t stream);
+
+/* The forward with the per-group choice: smoothing + INT8 quantization of Q and K, E4M3 V, then
+ * one attention launch in which each group runs the variant variant[b * Hkv + g] names (0: FP16
+ * P V, the result qattn_forward gives; 1: FP8 P V, the result qattn_attn_quantized_pv8 gives), bit
+ * for bit.  variant: device uint8 [B*Hkv] (e.g. from qattn_adaptive_calibrate).  Workspace from
+ * the library's pool.  Errors as qattn_forward; a NULL variant QATTN_ERR_INVALID_ARG;
+ * B * Hkv <= 65535. */
+qattn_status qattn_forward_adaptive(const void* q, const void* k, const void* v, void* out, int B,
+                                    int H, int Hkv, int N, int d, int causal,
+                                    const uint8_t* variant, qattn_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------
  * Checks.
  * ------------------------------------------------------------------------------------------ */
 

@@ -791,11 +791,12 @@ int oracle_attention_nvfp4(const uint8_t* q_codes, const uint8_t* q_scales, cons
  *     saturating at 448; amax == 0 gives sV = 0 and codes 0; a zero code is +0 (0x00) whatever
  *     the sign of the input.  Stored transposed ([slice][channel][Np] bytes, Np = N rounded up to
  *     128, zero padding), the K-major operand of the P V product.
- *   - P in E4M3 follows FlashAttention's online softmax over key tiles of 128 (page sec. 4):
- *     per tile the maximum t of the scaled scores of the tile's visible keys, m' = max(m, t); if
- *     m' > m the accumulated O and l are scaled by 2^(m - m') and m = m'; then per key
- *     p = 2^(y), y = S_int * c + (8 - m) (one binary32 fused multiply-add; c = (sQ * sK) * sl2 in
- *     binary32, sl2 = binary32(log2(e) / sqrt(d))), so that p <= 2^8 < 448; p^ = E4M3(p);
+ *   - P in E4M3 follows FlashAttention's online softmax over key tiles of 128 (page sec. 4),
+ *     with the running maximum moved only when it grows by more than 4 (log2 units): per tile
+ *     the maximum t of the scaled scores of the tile's visible keys; if t > m + 4 (or on the first
+ *     tile) the accumulated O and l are scaled by 2^(m - t) and m = t; then per key p = 2^(y),
+ *     y = S_int * c + (4 - m) (one binary32 fused multiply-add; c = (sQ * sK) * sl2 in binary32,
+ *     sl2 = binary32(log2(e) / sqrt(d))), so that p <= 2^(4 + 4) = 256 < 448; p^ = E4M3(p);
  *     l += p^; O += p^ v^ with v^ the E4M3 code values; out = O * sV / l.  The scaled maximum of
  *     a 64-key scale block is (max S_int over its visible keys) * c, one binary32 product.
  *   - The GPU computes 2^(y) with MUFU ex2 (binary32, a few ulp), so an E4M3 decision taken
@@ -901,7 +902,7 @@ int oracle_attention_pv8(const int8_t* q_i8, const float* q_scale, const int8_t*
                     if (tb > t) t = tb;
                 }
             }
-            if (t > m) {
+            if (t > m + 4.0f) {
                 const double alpha = (m == -INFINITY) ? 0.0 : exp2((double)m - (double)t);
                 l *= alpha;
                 rv *= alpha;
@@ -909,7 +910,7 @@ int oracle_attention_pv8(const int8_t* q_i8, const float* q_scale, const int8_t*
                 for (int c = 0; c < d; ++c) acc[c] *= alpha;
                 m = t;
             }
-            const float g = 8.0f - m;
+            const float g = 4.0f - m;
             for (int j = 0; j < n; ++j) {
                 const float y = fmaf((float)s[j], cb[j / 64], g);
                 const float p = (float)exp2((double)y);

@@ -211,3 +211,21 @@ def test_binding_argument_counts_match_the_header():
         params = params.strip()
         n = 0 if params in ("", "void") else params.count(",") + 1
         assert len(getattr(L, name).argtypes) == n, name
+
+
+def test_adaptive_argument_checks():
+    L = Q.load()
+    # null pointers, a bad threshold, a missing variant table, d
+    assert L.qattn_quant_v_fp8(None, 1, 2, 256, 128, P(16), P(32), None) == 1
+    assert L.qattn_quant_v_fp8(P(16), 1, 2, 256, 96, P(16), P(32), None) == 2
+    assert L.qattn_quant_v_fp8(P(16), 1, 2, 256, 128, P(20), P(32), None) == 3
+    assert L.qattn_attn_quantized_pv8(P(16), P(32), P(48), P(64), None, P(80), P(96), 1, 4, 2,
+                                      256, 128, 1, None) == 1
+    assert L.qattn_adaptive_calibrate(P(16), P(32), P(48), 1, 4, 2, 256, 128, 1, 3.0, P(64),
+                                      None, None) == 1
+    assert L.qattn_adaptive_calibrate(P(16), P(32), P(48), 1, 4, 2, 256, 128, 1, 0.99, None,
+                                      None, None) == 1
+    assert L.qattn_forward_adaptive(P(16), P(32), P(48), P(64), 1, 4, 2, 256, 128, 1, None,
+                                    None) == 1
+    assert L.qattn_forward_adaptive(P(16), P(32), P(48), P(64), 1, 4, 3, 256, 128, 1, P(80),
+                                    None) == 1
