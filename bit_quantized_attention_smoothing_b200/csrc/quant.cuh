@@ -24,6 +24,7 @@ namespace qattn {
 constexpr int kQBlock = 128;  // Q quantization block: 128 consecutive rows of one head
 constexpr int kKBlock = 64;   // K quantization block: 64 consecutive rows of one kv head
 constexpr int kSumRowsPerCta = 512;
+constexpr float kRoundBias = 12582912.0f;  // 1.5 * 2^23
 
 __device__ __forceinline__ float half_bits_to_float(uint32_t bits16) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(bits16)));
@@ -149,18 +150,23 @@ __device__ __forceinline__ void quantize_block_cta(const uint16_t* __restrict__ 
       x[2 * e] = half_bits_to_float(w[e] & 0xFFFFu) - m[2 * e];
       x[2 * e + 1] = half_bits_to_float(w[e] >> 16) - m[2 * e + 1];
     }
-    int r[8];
+    // rint(y) by adding 1.5 * 2^23 (the sum rounds to nearest-even, leaving rint(y) in two's
+    // complement in the low mantissa bits for |y| < 2^22; |y| <= 127 here), on the FMA pipe
+    // instead of a rounding and a float-to-int conversion per value
+    uint32_t t[8];
     bool near_tie = false;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const float y = x[e] * rcp;
-      const float ry = rintf(y);
+      const float y = __fmul_rn(x[e], rcp);
+      const float tb = __fadd_rn(y, kRoundBias);
+      const float ry = __fadd_rn(tb, -kRoundBias);
       near_tie |= fabsf(y - ry) > 0.4998779296875f;  // within 2^-13 of a half-integer
-      r[e] = static_cast<int>(ry);
+      t[e] = __float_as_uint(tb);
     }
+    // the low byte of each biased sum is the int8 code
     uint2 out;
-    out.x = __byte_perm(__byte_perm(r[0], r[1], 0x0040), __byte_perm(r[2], r[3], 0x0040), 0x5410);
-    out.y = __byte_perm(__byte_perm(r[4], r[5], 0x0040), __byte_perm(r[6], r[7], 0x0040), 0x5410);
+    out.x = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+    out.y = __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410);
     if (__any_sync(0xFFFFFFFFu, near_tie) && near_tie) {
       float q[8];
 #pragma unroll
