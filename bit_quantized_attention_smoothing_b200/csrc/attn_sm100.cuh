@@ -278,11 +278,11 @@ __device__ __forceinline__ void softmax_row(uint32_t (&sr)[4][32], int lim, floa
 // past N), the tile's amax (|x| and max on packed fp16 pairs, exact) through a warp shuffle and
 // a warpgroup barrier, scale = amax / 127 and codes rint(x * (1 / scale)) -- with the correctly
 // rounded quotient x / scale instead where a value lies within 2^-13 of a half-integer, which is
-// quantize_kernel's rule, so codes and scales are bit-identical to it (an 8-value chunk holding
-// such a value is recomputed on its own) -- written into the K-major swizzled layout the TMA
-// would produce (128-byte rows with 128-byte swizzle at d = 128, 64-byte rows with 64-byte
-// swizzle at d = 64).  |x| <= amax keeps every code within [-127, 127].  Returns the scale (0 for
-// an all-zero tile).
+// the pre-pass's rule (quantize_block_cta), so codes and scales are bit-identical to it (an
+// 8-value chunk holding such a value is recomputed on its own) -- written into the K-major
+// swizzled layout the TMA would produce (128-byte rows with 128-byte swizzle at d = 128, 64-byte
+// rows with 64-byte swizzle at d = 64).  |x| <= amax keeps every code within [-127, 127].
+// Returns the scale (0 for an all-zero tile).
 template <int D>
 __device__ __forceinline__ float quantize_q_tile(const uint16_t* __restrict__ q_head, int r0,
                                                  int N, int tid, int wt, uint8_t* tile,
@@ -387,7 +387,7 @@ struct ScoreDump {
 
 // QF16: Q arrives as fp16 (q16) and the softmax warps quantize their own Q tile into shared
 // memory before the first QK^T (per-tile amax, scale = amax / 127, the same rounding as
-// quantize_kernel); otherwise int8 Q and its scales come from the smoothing + quantization pass
+// the pre-pass); otherwise int8 Q and its scales come from the smoothing + quantization pass
 // (tm_q, q_scale).  MODE: kOutF16, kDumpS (only its block-to-work mapping differs, see
 // ScoreDump) or kOutF32 (out points to fp32).  PVK: kPvF16 (P and V in fp16), kPvF8 (P and V in
 // E4M3: tm_v8 maps V^T in E4M3, v_scale its per-(batch, kv head) scale) or kPvTable (pv_variant[bg]

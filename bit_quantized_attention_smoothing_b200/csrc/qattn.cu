@@ -178,25 +178,33 @@ QuantLayout forward_layout(int B, int H, int Hkv, int N, int d) {
   return L;
 }
 
-// Channel sums, then one quantization launch over the Q blocks (unless q is null: the fused
-// forward quantizes Q inside the attention kernel) and the K blocks.
+// Two launches.  With q: Q's quantization together with the K channel sums (the K-sum CTAs last,
+// so that K is still in L2), then the K quantization.  Without q (the fused forward quantizes Q
+// inside the attention kernel): the channel sums, then the K quantization.
 template <int D>
 qattn_status run_smooth_quant(const void* q, const void* k, int B, int H, int Hkv, int N,
                               int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale,
                               float* k_mean, long long* sums, cudaStream_t st) {
   const int nqb = (N + kQBlock - 1) / kQBlock;
   const int nkb = (N + kKBlock - 1) / kKBlock;
+  const int nchunk = (N + kSumRowsPerCta - 1) / kSumRowsPerCta;
+  const long long nq = q ? static_cast<long long>(B) * H * nqb : 0;
+  const long long nsum = static_cast<long long>(B) * Hkv * nchunk;
+  const long long nk = static_cast<long long>(B) * Hkv * nkb;
+  if (nq + nsum > 0x7FFFFFFFLL || nk > 0x7FFFFFFFLL) return QATTN_ERR_UNSUPPORTED;
   if (cudaMemsetAsync(sums, 0, sizeof(long long) * B * Hkv * D, st) != cudaSuccess)
     return QATTN_ERR_CUDA;
-  dim3 g1(B * Hkv, (N + kSumRowsPerCta - 1) / kSumRowsPerCta);
-  k_channel_sums_kernel<D><<<g1, 256, 0, st>>>(static_cast<const uint16_t*>(k), N, sums);
+  if (q) {
+    q_quant_k_sums_kernel<D><<<static_cast<unsigned>(nq + nsum), 256, 0, st>>>(
+        static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), N, nqb, nq, nchunk, q_i8,
+        q_scale, sums);
+  } else {
+    dim3 g1(B * Hkv, nchunk);
+    k_channel_sums_kernel<D><<<g1, 256, 0, st>>>(static_cast<const uint16_t*>(k), N, sums);
+  }
   if (launch_status() != QATTN_OK) return QATTN_ERR_CUDA;
-  const long long nq = q ? static_cast<long long>(B) * H * nqb : 0;
-  const long long nk = static_cast<long long>(B) * Hkv * nkb;
-  if (nq + nk > 0x7FFFFFFFLL) return QATTN_ERR_UNSUPPORTED;
-  quantize_kernel<D><<<static_cast<unsigned>(nq + nk), 256, 0, st>>>(
-      static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), N, nqb, nkb, nq, sums,
-      q_i8, q_scale, k_i8, k_scale, k_mean);
+  k_quantize_kernel<D><<<static_cast<unsigned>(nk), 256, 0, st>>>(
+      static_cast<const uint16_t*>(k), N, nkb, sums, k_i8, k_scale, k_mean);
   return launch_status();
 }
 

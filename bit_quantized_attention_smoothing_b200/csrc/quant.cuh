@@ -31,20 +31,19 @@ __device__ __forceinline__ float half_bits_to_float(uint32_t bits16) {
 }
 
 // ---------------------------------------------------------------------------------------------
-// K channel sums: sums[bg * D + c] += sum over this CTA's rows of K[bg, n, c] * 2^24 (exact).
-// grid (B*Hkv, ceil(N / kSumRowsPerCta)), 256 threads.  sums must be zeroed beforehand.
+// K channel sums: sums[bg * D + c] += sum over rows kSumRowsPerCta * chunk .. of K[bg, n, c] * 2^24
+// (exact), one 256-thread CTA.  sums must be zeroed beforehand.
 // ---------------------------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(256) k_channel_sums_kernel(const uint16_t* __restrict__ k, int N,
-                                                             long long* __restrict__ sums) {
+__device__ __forceinline__ void k_channel_sums_cta(const uint16_t* __restrict__ k, int N, int bg,
+                                                   int chunk, long long* __restrict__ sums) {
   constexpr int VPR = D / 8;            // 16-byte vectors per row
   constexpr int RPI = 256 / VPR;        // rows per iteration of the CTA
   __shared__ long long red[RPI][D];
-  const int bg = blockIdx.x;
   const int tid = threadIdx.x;
   const int cg = tid % VPR;
   const int r_in = tid / VPR;
-  const int n0 = blockIdx.y * kSumRowsPerCta;
+  const int n0 = chunk * kSumRowsPerCta;
   const int n1 = min(N, n0 + kSumRowsPerCta);
   const uint4* base = reinterpret_cast<const uint4*>(k + static_cast<size_t>(bg) * N * D);
   long long acc[8];
@@ -69,6 +68,13 @@ __global__ void __launch_bounds__(256) k_channel_sums_kernel(const uint16_t* __r
     atomicAdd(reinterpret_cast<unsigned long long*>(sums + static_cast<size_t>(bg) * D + c),
               static_cast<unsigned long long>(s));
   }
+}
+
+// grid (B*Hkv, ceil(N / kSumRowsPerCta)), 256 threads.
+template <int D>
+__global__ void __launch_bounds__(256) k_channel_sums_kernel(const uint16_t* __restrict__ k, int N,
+                                                             long long* __restrict__ sums) {
+  k_channel_sums_cta<D>(k, N, blockIdx.x, blockIdx.y, sums);
 }
 
 // rint(x / s) for x, s > 0 as described in the file header.
@@ -178,17 +184,44 @@ __device__ __forceinline__ void quantize_block_cta(const uint16_t* __restrict__ 
   }
 }
 
+// The second pre-pass launch: K' = K - mean and its per-64-row INT8 quantization, one CTA per K
+// block (mean from the exact channel sums, written to k_mean by each kv group's first block when
+// k_mean is not null).
 template <int D>
-__global__ void __launch_bounds__(256) quantize_kernel(
-    const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, int N, int nqb, int nkb,
-    long long nq, const long long* __restrict__ sums, int8_t* __restrict__ q_i8,
-    float* __restrict__ q_scale, int8_t* __restrict__ k_i8, float* __restrict__ k_scale,
-    float* __restrict__ k_mean) {
+__global__ void __launch_bounds__(256) k_quantize_kernel(
+    const uint16_t* __restrict__ k, int N, int nkb, const long long* __restrict__ sums,
+    int8_t* __restrict__ k_i8, float* __restrict__ k_scale, float* __restrict__ k_mean) {
   __shared__ float mean_s[D];
   __shared__ float red[8];
-  // K blocks first: the channel-sum pass has just read K, so its second read mostly hits L2
-  const long long nk = static_cast<long long>(gridDim.x) - nq;
-  const long long blk = blockIdx.x < nk ? nq + blockIdx.x : blockIdx.x - nk;
+  const long long kblk = blockIdx.x;
+  const long long bg = kblk / nkb;
+  const int kb = static_cast<int>(kblk % nkb);
+  if (threadIdx.x < D) {
+    const long long s = sums[bg * D + threadIdx.x];
+    const double den = static_cast<double>(N) * 16777216.0;
+    const float mu = __double2float_rn(__ddiv_rn(__ll2double_rn(s), den));
+    mean_s[threadIdx.x] = mu;
+    if (kb == 0 && k_mean != nullptr) k_mean[bg * D + threadIdx.x] = mu;
+  }
+  __syncthreads();
+  const int r0 = kb * kKBlock;
+  const int rows = min(kKBlock, N - r0);
+  const size_t off = (static_cast<size_t>(bg) * N + r0) * D;
+  quantize_block_cta<D, kKBlock>(k + off, rows, mean_s, k_i8 + off, k_scale + kblk, red);
+}
+
+// The first of the forward's two pre-pass launches: Q's quantization (which needs no K mean) and
+// the K channel sums in one grid of nq + nsum CTAs.  CTAs 0 .. nq-1 quantize Q blocks (as
+// quantize_kernel does); the last nsum sum K rows (chunk = index % nchunk of kv group index /
+// nchunk), so that K has just passed through L2 when the second launch (quantize_kernel over the
+// K blocks alone) reads it again.
+template <int D>
+__global__ void __launch_bounds__(256) q_quant_k_sums_kernel(
+    const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, int N, int nqb, long long nq,
+    int nchunk, int8_t* __restrict__ q_i8, float* __restrict__ q_scale,
+    long long* __restrict__ sums) {
+  __shared__ float red[8];
+  const long long blk = blockIdx.x;
   if (blk < nq) {
     const long long bh = blk / nqb;
     const int qb = static_cast<int>(blk % nqb);
@@ -197,21 +230,8 @@ __global__ void __launch_bounds__(256) quantize_kernel(
     const size_t off = (static_cast<size_t>(bh) * N + r0) * D;
     quantize_block_cta<D, kQBlock>(q + off, rows, nullptr, q_i8 + off, q_scale + blk, red);
   } else {
-    const long long kblk = blk - nq;
-    const long long bg = kblk / nkb;
-    const int kb = static_cast<int>(kblk % nkb);
-    if (threadIdx.x < D) {
-      const long long s = sums[bg * D + threadIdx.x];
-      const double den = static_cast<double>(N) * 16777216.0;
-      const float mu = __double2float_rn(__ddiv_rn(__ll2double_rn(s), den));
-      mean_s[threadIdx.x] = mu;
-      if (kb == 0 && k_mean != nullptr) k_mean[bg * D + threadIdx.x] = mu;
-    }
-    __syncthreads();
-    const int r0 = kb * kKBlock;
-    const int rows = min(kKBlock, N - r0);
-    const size_t off = (static_cast<size_t>(bg) * N + r0) * D;
-    quantize_block_cta<D, kKBlock>(k + off, rows, mean_s, k_i8 + off, k_scale + kblk, red);
+    const long long i = blk - nq;
+    k_channel_sums_cta<D>(k, N, static_cast<int>(i / nchunk), static_cast<int>(i % nchunk), sums);
   }
 }
 
