@@ -14,8 +14,10 @@
 // instruction reads them in this arrangement: row r = r0 + 32 r1 (r0 < 32, r1 < 4) of the operand
 // has its four scale bytes of one 64-element K step (blocks 4 kc .. 4 kc + 3, the lowest block in
 // the lowest byte) in the 32-bit column (base + r1) of lane r0, and the same 32 lanes are repeated
-// in each of the four 32-lane sub-partitions.  Each warp writes its own sub-partition's copy with
-// tcgen05.st, so no shared-memory staging is needed for the scales.
+// in each of the four 32-lane sub-partitions.  Q's, K's and V's scales are written by each warp
+// into its own sub-partition with tcgen05.st; P's, whose rows belong to all sub-partitions, are
+// staged in shared memory in that order ([K step][r0][r1] words) and copied into all four
+// sub-partitions at once by the issuing warp (tcgen05.cp .32x128b.warpx4).
 #pragma once
 
 #include <cstdint>
@@ -212,8 +214,8 @@ namespace qattn {
 //   K scales, arrive on s_free; exchange the row maximum; wait P V(j - 1) and fold it into the
 //   outputs (O = O corr + acc f); compute P (FP4: two-level codes and scales, codes into the
 //   swizzled shared-memory operand; FP16: pairs into tensor memory over the consumed scores),
-//   write tile j's V scales; after a barrier among the softmax warps write their share of P's
-//   block scales into every sub-partition and arrive on p_full.
+//   write tile j's V scales and stage P's block scales in shared memory, arrive on p_full; the
+//   issuing warp copies P's scales into tensor memory ahead of P V(j).
 // Exponentials and reciprocals are MUFU ex2 / rcp, code and scale quotients products with those
 // reciprocals; they differ from the correctly rounded operations only within a relative 2^-20 of a
 // rounding tie.  Every wait is bounded; the softmax warps agree on each step's outcome at their
@@ -240,9 +242,11 @@ struct Fp4AttnCfg {
   static constexpr int kOffQ16 = kOffP + kP;
   static constexpr int kOffK16 = kOffQ16 + kT16;      // two fp16 K tiles
   static constexpr int kOffV16 = kOffK16 + 2 * kT16;  // two fp16 V tiles
-  static constexpr int kOffSfp = kOffV16 + 2 * kT16;  // uint32 [2][128]: P scale words by K step
-  static constexpr int kOffRed = kOffSfp + 1024;      // float [4][128]: row parts' maxima, sums
-  static constexpr int kOffMask = kOffRed + 2048;     // uint32 [32]: promoted key tiles, bit t
+  static constexpr int kOffSfp = kOffV16 + 2 * kT16;  // uint32 [2][32][4]: P scale words, K step,
+                                                      // row % 32, row / 32 (tcgen05.cp source)
+  static constexpr int kOffRed = kOffSfp + 1024;      // float [2][4][128]: row parts' maxima by
+                                                      // step parity; sums
+  static constexpr int kOffMask = kOffRed + 4096;     // uint32 [32]: promoted key tiles, bit t
   static constexpr int kOffBar = kOffMask + 128;
   static constexpr int kSmemUsed = kOffBar + 128 + 1024;  // + alignment slack
   static constexpr uint32_t kSwQK = D == 128 ? kSwizzle64B : kSwizzle32B;
@@ -370,6 +374,20 @@ __device__ __forceinline__ void mma_nvf4_ss_warp(uint32_t d_tmem, uint64_t adesc
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
+
+// tcgen05.cp of 32 rows x 128 bits from shared memory (descriptor sdesc: no swizzle, rows 16 bytes
+// apart, 8-row groups 128 bytes apart) into the four columns at taddr of lanes 0-31 of every
+// 32-lane sub-partition; one lane, picked by elect.sync, issues it.  It executes in order with the
+// tensor-core operations the same lane issues after it.
+__device__ __forceinline__ void tmem_cp32x128_warpx4_warp(uint32_t taddr, uint64_t sdesc) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr),
+      "l"(sdesc)
+      : "memory");
+}
+
 __device__ __forceinline__ void mma_f16_ss_warp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                                 uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -589,7 +607,17 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
     // -------------------------------------------------------------------------- issuing warp
     // The whole warp runs this loop on warp-uniform values; lane 0 issues the TMA loads and one
     // elected lane each tensor-core instruction.
-    int n_kl[2] = {0, 0}, n_kw[2] = {0, 0}, n_vl[2] = {0, 0}, n_vw[2] = {0, 0};
+    // loads issued and waited per K / V buffer (two scalars each: an array indexed by the buffer
+    // number would live in local memory)
+    struct Count2 {
+      int v0, v1;
+      __device__ int operator[](int b) const { return b ? v1 : v0; }
+      __device__ void inc(int b) {
+        if (b) ++v1;
+        else ++v0;
+      }
+    };
+    Count2 n_kl{0, 0}, n_kw{0, 0}, n_vl{0, 0}, n_vw{0, 0};
     bool q_waited = false, q16_waited = false;
     auto load_k = [&](int t) {
       const int bb = t & 1;
@@ -605,7 +633,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
         }
       }
       __syncwarp();
-      ++n_kl[bb];
+      n_kl.inc(bb);
     };
     auto load_v = [&](int t) {
       const int bb = t & 1;
@@ -621,7 +649,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
         }
       }
       __syncwarp();
-      ++n_vl[bb];
+      n_vl.inc(bb);
     };
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort));
@@ -634,7 +662,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
       if (!pr && !q_waited) q_waited = wait_all(q_full, 0);
       if (!(pr ? q16_waited : q_waited)) return false;
       if (!wait_all(k_full + bb, static_cast<uint32_t>(n_kw[bb]) & 1u)) return false;
-      ++n_kw[bb];
+      n_kw.inc(bb);
       tc_fence_after();
       const uint32_t ds = tmem + Cfg::kColS + 128 * bb;
       if (pr) {
@@ -663,7 +691,7 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
     auto issue_pv = [&](int t) -> bool {
       const int bb = t & 1;
       if (!wait_all(v_full + bb, static_cast<uint32_t>(n_vw[bb]) & 1u)) return false;
-      ++n_vw[bb];
+      n_vw.inc(bb);
       tc_fence_after();
       if (promoted(t)) {
         constexpr uint32_t id = idesc_f16_f32_bmn(128, D);
@@ -673,6 +701,10 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
         for (int kk = 0; kk < 8; ++kk)
           mma_f16_ts_warp(tmem + Cfg::kColO, ap + 8 * kk, dv + 128 * kk, id, kk > 0 ? 1u : 0u);
       } else {
+        // P's block scales, staged by the softmax warps, into every sub-partition
+#pragma unroll
+        for (int kc = 0; kc < 2; ++kc)
+          tmem_cp32x128_warpx4_warp(tmem + Cfg::kColSfp + 4 * kc, smem_desc(smem_u32(sfp) + kc * 512, 128, 128, 0));
         constexpr uint32_t id = idesc_nvf4(128, D);
 #pragma unroll
         for (int kc = 0; kc < 2; ++kc) {
@@ -851,11 +883,14 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
 #pragma unroll
         for (int k = 0; k < 32; k += 2) smax = fmax3(smax, __uint_as_float(s[k]), __uint_as_float(s[k + 1]));
       }
-      red[pt * 128 + rl] = smax;
+      // by step parity: a part writes this buffer again two steps on, after the next step's
+      // barrier, which every part reaches only after its reads below
+      float* rm = red + 512 * (j & 1);
+      rm[pt * 128 + rl] = smax;
       ok = named_bar_and(1, kFp4Softmax, ok && wok);
       if (!ok) break;
       tc_fence_after();
-      const float row_smax = fmaxf(fmaxf(red[rl], red[128 + rl]), fmaxf(red[256 + rl], red[384 + rl]));
+      const float row_smax = fmaxf(fmaxf(rm[rl], rm[128 + rl]), fmaxf(rm[256 + rl], rm[384 + rl]));
       // (4) running maximum
       const float t = prom ? (row_smax - cq) * sl2 : row_smax * gqk;
       const float m_new = fmaxf(m, t);
@@ -893,19 +928,14 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
       if (!prom) {
         // 16 bytes (keys 32 pt .. 32 pt + 31) into the 64-byte-swizzled row of the P operand
         st_shared_v4(prow + ((static_cast<uint32_t>(pt) ^ swz) << 4), cw[0], cw[1], cw[2], cw[3]);
-        // the two scale bytes: half (pt & 1) of row rl's word for K step pt >> 1
-        reinterpret_cast<uint16_t*>(sfp)[((pt >> 1) * 128 + rl) * 2 + (pt & 1)] = static_cast<uint16_t>(sw);
+        // the two scale bytes: half (pt & 1) of row rl's word for K step pt >> 1, at word
+        // (pt >> 1, rl % 32, rl / 32) of the staging area the issuing warp copies from
+        reinterpret_cast<uint16_t*>(sfp)[((pt >> 1) * 128 + (rl & 31) * 4 + (rl >> 5)) * 2 + (pt & 1)] =
+            static_cast<uint16_t>(sw);
         fence_proxy_async_smem();
         store_v_words(vw);
       }
       l = l * corr + lsum;
-      named_bar_sync(2, kFp4Softmax);
-      // (7) P's block scales: row r0 + 32 r1 in column r1 of lane r0, in every sub-partition; part
-      // pt writes K step pt >> 1, row groups 2 (pt & 1) and 2 (pt & 1) + 1
-      if (!prom) {
-        const uint32_t* w = sfp + (pt >> 1) * 128 + lane + 64 * (pt & 1);
-        tmem_st32x2(lane_base + Cfg::kColSfp + 4 * (pt >> 1) + 2 * (pt & 1), w[0], w[32]);
-      }
       tmem_st_wait();
       tc_fence_before();
       arrive(p_full);
