@@ -430,7 +430,8 @@ def workload_line(w, r, steps, world, p8, p16, peak_src):
             "peak": round(mixed_peak, 1),
             "unit": "TFLOP/s",
             "frac": round(achieved / mixed_peak, 4),
-            "traffic": profiled_traffic(w.name),
+            # the committed capture is of the dense launch; a block-sparse launch moves less
+            "traffic": None if r["sparse"] else profiled_traffic(w.name),
             "peak_source": ("mixed INT8/FP16 ceiling 2/(1/P8+1/P16), since half the metric's "
                             "operations run at each rate; " + peak_src),
             "frac_of_int8_peak": round(achieved / p8, 4),
