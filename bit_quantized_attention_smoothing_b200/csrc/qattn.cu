@@ -796,17 +796,39 @@ qattn_status qattn_forward_host(const void* q_host, const void* k_host, const vo
   uint8_t* b8 = static_cast<uint8_t*>(buf);
   // Every (batch, kv head) group -- its kv head and the H / Hkv query heads reading it -- is an
   // independent forward (the smoothing mean is per group), and group f = b * Hkv + g owns
-  // contiguous bytes of q, k, v and out.  The groups are cut into up to kHostChunks chunks; chunk
-  // c's upload (s_in), forward (the caller's stream) and download (s_out) are ordered by events,
-  // so one chunk's copies overlap another chunk's kernels.
+  // contiguous bytes of q, k, v and out (its query heads too).  The groups are cut into up to
+  // kHostChunks chunks; chunk c's upload (s_in), forward (the caller's stream) and download (s_out)
+  // are ordered by events, so one chunk's copies overlap another chunk's kernels.  When the chunks
+  // are single groups of two or more query heads, the first and the last group run as two pieces
+  // of half their query heads each (the first piece uploads the group's K and V): the first
+  // forward starts after a smaller upload and the last download is smaller, at the price of one
+  // more smoothing pass of those groups' K.
   const int G = B * Hkv, r = H / Hkv;
   const int nch = G < kHostChunks ? G : kHostChunks;
   const int per = (G + nch - 1) / nch;
-  const size_t q_grp = sizeof(uint16_t) * static_cast<size_t>(r) * N * d;
-  const size_t k_grp = sizeof(uint16_t) * static_cast<size_t>(N) * d;
-  cudaEvent_t ev[2 * kHostChunks + 2] = {};
+  const size_t q_head = sizeof(uint16_t) * static_cast<size_t>(N) * d;
+  const size_t q_grp = q_head * r;
+  const size_t k_grp = q_head;
+  struct Piece {
+    int f0, nf, h0, nh;  // groups f0 .. f0 + nf - 1, query heads h0 .. h0 + nh - 1 of each
+    bool kv;             // this piece uploads the groups' K and V
+  };
+  Piece pcs[kHostChunks + 2];
+  int np = 0;
+  const bool split = per == 1 && r >= 2;
+  for (int c = 0; c < nch; ++c) {
+    const int f0 = c * per, nf = (f0 + per <= G ? per : G - f0);
+    if (nf <= 0) break;
+    if (split && (c == 0 || c == nch - 1)) {
+      pcs[np++] = Piece{f0, 1, 0, r / 2, true};
+      pcs[np++] = Piece{f0, 1, r / 2, r - r / 2, false};
+    } else {
+      pcs[np++] = Piece{f0, nf, 0, r, true};
+    }
+  }
+  cudaEvent_t ev[2 * (kHostChunks + 2) + 2] = {};
   int nev = 0;
-  for (int i = 0; i < 2 * nch + 2 && s == QATTN_OK; ++i, ++nev)
+  for (int i = 0; i < 2 * np + 2 && s == QATTN_OK; ++i, ++nev)
     if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) s = QATTN_ERR_CUDA;
   const char* qh = static_cast<const char*>(q_host);
   const char* kh = static_cast<const char*>(k_host);
@@ -814,42 +836,47 @@ qattn_status qattn_forward_host(const void* q_host, const void* k_host, const vo
   char* oh = static_cast<char*>(out_host);
   // s_in and s_out start after the work already queued on the caller's stream (the pool
   // allocation above and anything before this call)
-  if (s == QATTN_OK && (cudaEventRecord(ev[2 * nch], st) != cudaSuccess ||
-                        cudaStreamWaitEvent(s_in, ev[2 * nch], 0) != cudaSuccess ||
-                        cudaStreamWaitEvent(s_out, ev[2 * nch], 0) != cudaSuccess))
+  if (s == QATTN_OK && (cudaEventRecord(ev[2 * np], st) != cudaSuccess ||
+                        cudaStreamWaitEvent(s_in, ev[2 * np], 0) != cudaSuccess ||
+                        cudaStreamWaitEvent(s_out, ev[2 * np], 0) != cudaSuccess))
     s = QATTN_ERR_CUDA;
-  for (int c = 0; c < nch && s == QATTN_OK; ++c) {
-    const int f0 = c * per, nf = (f0 + per <= G ? per : G - f0);
-    if (nf <= 0) break;
-    if (cudaMemcpyAsync(b8 + f0 * q_grp, qh + f0 * q_grp, nf * q_grp, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
-        cudaMemcpyAsync(b8 + off_k + f0 * k_grp, kh + f0 * k_grp, nf * k_grp, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
-        cudaMemcpyAsync(b8 + off_v + f0 * k_grp, vh + f0 * k_grp, nf * k_grp, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+  // q and out bytes of a piece: its query heads are contiguous within each of its groups, and a
+  // piece of several groups takes all their heads, so the piece's bytes are one contiguous run
+  auto q_off = [&](const Piece& p) { return p.f0 * q_grp + p.h0 * q_head; };
+  auto q_len = [&](const Piece& p) { return p.nf * static_cast<size_t>(p.nh) * q_head; };
+  for (int c = 0; c < np && s == QATTN_OK; ++c) {
+    const Piece& p = pcs[c];
+    if (cudaMemcpyAsync(b8 + q_off(p), qh + q_off(p), q_len(p), cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        (p.kv && (cudaMemcpyAsync(b8 + off_k + p.f0 * k_grp, kh + p.f0 * k_grp, p.nf * k_grp,
+                                  cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+                  cudaMemcpyAsync(b8 + off_v + p.f0 * k_grp, vh + p.f0 * k_grp, p.nf * k_grp,
+                                  cudaMemcpyHostToDevice, s_in) != cudaSuccess)) ||
         cudaEventRecord(ev[c], s_in) != cudaSuccess)
       s = QATTN_ERR_CUDA;
   }
-  for (int c = 0; c < nch && s == QATTN_OK; ++c) {
-    const int f0 = c * per, nf = (f0 + per <= G ? per : G - f0);
-    if (nf <= 0) break;
+  for (int c = 0; c < np && s == QATTN_OK; ++c) {
+    const Piece& p = pcs[c];
+    // a piece's K and V arrived with it or with an earlier piece (s_in runs in order)
     if (cudaStreamWaitEvent(st, ev[c], 0) != cudaSuccess) {
       s = QATTN_ERR_CUDA;
       break;
     }
-    // the chunk as a forward of nf "batches" of one kv head and r query heads each
-    s = qattn_forward(b8 + f0 * q_grp, b8 + off_k + f0 * k_grp, b8 + off_v + f0 * k_grp,
-                      b8 + off_o + f0 * q_grp, nf, r, 1, N, d, causal, stream);
-    if (s == QATTN_OK && (cudaEventRecord(ev[nch + c], st) != cudaSuccess ||
-                          cudaStreamWaitEvent(s_out, ev[nch + c], 0) != cudaSuccess ||
-                          cudaMemcpyAsync(oh + f0 * q_grp, b8 + off_o + f0 * q_grp, nf * q_grp,
+    // the piece as a forward of nf "batches" of one kv head and nh query heads each
+    s = qattn_forward(b8 + q_off(p), b8 + off_k + p.f0 * k_grp, b8 + off_v + p.f0 * k_grp,
+                      b8 + off_o + q_off(p), p.nf, p.nh, 1, N, d, causal, stream);
+    if (s == QATTN_OK && (cudaEventRecord(ev[np + c], st) != cudaSuccess ||
+                          cudaStreamWaitEvent(s_out, ev[np + c], 0) != cudaSuccess ||
+                          cudaMemcpyAsync(oh + q_off(p), b8 + off_o + q_off(p), q_len(p),
                                           cudaMemcpyDeviceToHost, s_out) != cudaSuccess))
       s = QATTN_ERR_CUDA;
   }
   // the caller's stream takes up both copy streams again before the buffer goes back to the pool
-  if (nev < 2 * nch + 2) {
-    // no event, so nothing was queued on the copy streams
-  } else if (cudaEventRecord(ev[2 * nch + 1], s_out) != cudaSuccess ||
-      cudaStreamWaitEvent(st, ev[2 * nch + 1], 0) != cudaSuccess ||
-      cudaEventRecord(ev[2 * nch], s_in) != cudaSuccess ||
-      cudaStreamWaitEvent(st, ev[2 * nch], 0) != cudaSuccess) {
+  if (nev < 2 * np + 2) {
+    // not every event exists, so nothing was queued on the copy streams
+  } else if (cudaEventRecord(ev[2 * np + 1], s_out) != cudaSuccess ||
+      cudaStreamWaitEvent(st, ev[2 * np + 1], 0) != cudaSuccess ||
+      cudaEventRecord(ev[2 * np], s_in) != cudaSuccess ||
+      cudaStreamWaitEvent(st, ev[2 * np], 0) != cudaSuccess) {
     if (s == QATTN_OK) s = QATTN_ERR_CUDA;
   }
   if (cudaFreeAsync(buf, st) != cudaSuccess && s == QATTN_OK) s = QATTN_ERR_CUDA;

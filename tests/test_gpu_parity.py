@@ -220,12 +220,26 @@ def test_forward_variants_agree(lib):
     assert torch.equal(a.cpu(), c) and torch.equal(a.cpu(), d)
 
 
+HOST_SHAPES = [
+    # 9 groups: uneven chunks of 2, 2, 2, 2, 1 groups
+    {"B": 3, "H": 6, "Hkv": 3, "N": 300},
+    # 8 single-group chunks of 4 query heads: the first and last run as two pieces of 2 heads
+    {"B": 1, "H": 32, "Hkv": 8, "N": 300},
+    # one group of 3 query heads: pieces of 1 and 2 heads; two groups of 2: both split
+    {"B": 1, "H": 3, "Hkv": 1, "N": 520},
+    {"B": 1, "H": 4, "Hkv": 2, "N": 129},
+    # one group of one query head: no split
+    {"B": 1, "H": 1, "Hkv": 1, "N": 700},
+]
+
+
+@pytest.mark.parametrize("shape", HOST_SHAPES, ids=lambda o: "-".join(f"{k}{v}" for k, v in o.items()))
 @pytest.mark.parametrize("pinned", [True, False])
-def test_host_forward_pipeline_chunks(lib, pinned):
+def test_host_forward_pipeline_chunks(lib, pinned, shape):
     """qattn_forward_host cuts the (batch, kv head) groups into chunks whose copies and kernels
-    overlap; 9 groups make uneven chunks (2, 2, 2, 2, 1).  Results must equal the device-buffer
-    forward bit for bit."""
-    w = WORKLOADS["wide64"].with_(B=3, H=6, Hkv=3, N=300, causal=True)
+    overlap, and the first and last single-group chunks into two pieces of half their query heads.
+    Results must equal the device-buffer forward bit for bit."""
+    w = WORKLOADS["wide64"].with_(causal=True, **shape)
     q, k, v = _inputs(w, "cpu")
     a = lib.qattn_forward(q.cuda(), k.cuda(), v.cuda(), causal=True)
     hq, hk, hv = (t.cpu() for t in (q, k, v))
