@@ -1,6 +1,8 @@
 // quant.cuh -- smoothing of K and per-block INT8 quantization of Q and K' (SageAttention summary
-// page, aibr.jp/archives/102657, sec. 3: smooth K, quantize to INT8).  Both kernels are bound by
-// HBM bandwidth: 16-byte coalesced loads, warp-shuffle reductions, one pass over the data each.
+// page, aibr.jp/archives/102657, sec. 3: smooth K, quantize to INT8).  The forward's two launches
+// (Q's quantization with the K channel sums, then K's smoothing and quantization) are bound by
+// HBM bandwidth: 16-byte coalesced loads, warp-shuffle reductions; Q is read once, K twice (the
+// second time mostly from L2).
 //
 // Bit-exactness.  The codes and scales are exact functions of the inputs:
 //  * the channel sums are exact int64 sums of K * 2^24 (every fp16 value is an integer multiple of
@@ -211,10 +213,9 @@ __global__ void __launch_bounds__(256) k_quantize_kernel(
 }
 
 // The first of the forward's two pre-pass launches: Q's quantization (which needs no K mean) and
-// the K channel sums in one grid of nq + nsum CTAs.  CTAs 0 .. nq-1 quantize Q blocks (as
-// quantize_kernel does); the last nsum sum K rows (chunk = index % nchunk of kv group index /
-// nchunk), so that K has just passed through L2 when the second launch (quantize_kernel over the
-// K blocks alone) reads it again.
+// the K channel sums in one grid of nq + nsum CTAs.  CTAs 0 .. nq-1 quantize Q's 128-row blocks;
+// the last nsum sum K rows (chunk index % nchunk of kv group index / nchunk), so that K has just
+// passed through L2 when the second launch (k_quantize_kernel) reads it again.
 template <int D>
 __global__ void __launch_bounds__(256) q_quant_k_sums_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, int N, int nqb, long long nq,
