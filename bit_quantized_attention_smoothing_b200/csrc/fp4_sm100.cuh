@@ -884,10 +884,13 @@ __global__ void __launch_bounds__(kFp4Threads, 1)
         for (int k = 0; k < 32; k += 2) smax = fmax3(smax, __uint_as_float(s[k]), __uint_as_float(s[k + 1]));
       }
       // by step parity: a part writes this buffer again two steps on, after the next step's
-      // barrier, which every part reaches only after its reads below
+      // barrier, which every part reaches only after its reads below.  The barrier joins the four
+      // parts of this lane quadrant (the only readers of its rows' entries; named barrier 5 +
+      // quadrant, 128 threads); a quadrant whose wait gave up leaves here, and the others leave at
+      // their next wait once the issuing warp raises the abort flag.
       float* rm = red + 512 * (j & 1);
       rm[pt * 128 + rl] = smax;
-      ok = named_bar_and(1, kFp4Softmax, ok && wok);
+      ok = named_bar_and(5 + quad, 128, ok && wok);
       if (!ok) break;
       tc_fence_after();
       const float row_smax = fmaxf(fmaxf(rm[rl], rm[128 + rl]), fmaxf(rm[256 + rl], rm[384 + rl]));
