@@ -214,8 +214,9 @@ qattn_status qattn_forward(const void* q, const void* k, const void* v, void* ou
 
 /* Forward on HOST buffers: copies q, k, v to the device, runs the forward, copies the result
  * back to out_host, and returns after the copy has finished (the stream is synchronized).  The
- * (batch, kv head) groups are processed in up to 8 chunks whose uploads, kernels (on `stream`)
- * and downloads overlap through two copy streams the library keeps per device; results are
+ * (batch, kv head) groups are processed in up to 8 chunks (the first and last single-group
+ * chunks as two pieces of half their query heads) whose uploads, kernels (on `stream`) and
+ * downloads overlap through two copy streams the library keeps per device; results are
  * identical to qattn_forward.  Device buffers come from the library's pool.  Page-locked host
  * memory gives asynchronous, overlapped copies; pageable memory works but is slower. */
 qattn_status qattn_forward_host(const void* q_host, const void* k_host, const void* v_host,
