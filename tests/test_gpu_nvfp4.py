@@ -426,6 +426,45 @@ def test_attn_nvfp4_promoted_full_size_sampled_rows(lib, oracle):
     _check_fp4_out(got, ref, slack, "llama8b_32k promoted full")
 
 
+def test_attn_nvfp4_promoted_longest_lists(lib, oracle):
+    """131072 tokens = 1024 key tiles, the most the promotion lists may index (the kernel's tile
+    mask holds 1024 bits): one head, causal, top-8; the last query block's diagonal tiles 1022
+    and 1023 are promoted.  Lists, quantized operands and mean from the GPU path (checked against
+    the oracle), sampled rows at both ends of the sequence against the oracle."""
+    w = WORKLOADS["long128k"].with_(H=1, Hkv=1)
+    assert (w.N + 127) // 128 == 1024
+    topk = 8
+    q, k, v = make_inputs(w, device="cuda")
+    sums = oracle.k_channel_sums(np16(k), 1, 1, w.N, w.d)
+    mean = np.array([oracle.lib().oracle_mean_from_sum(int(s), w.N) for s in sums.ravel()],
+                    dtype=np.float32).reshape(1, w.d)
+    meang = torch.from_numpy(mean).cuda()
+    gq = lib.qattn_quant_nvfp4(q.reshape(1, w.N, w.d))
+    gk = lib.qattn_quant_nvfp4(k.reshape(1, w.N, w.d), meang)
+    gv = lib.qattn_quant_nvfp4(v.reshape(1, w.N, w.d), along_rows=True)
+    gl, gc = lib.qattn_block_select(q, k, topk, causal=True)
+    out = lib.qattn_attn_nvfp4(gq, gk, gv, 1, 1, 1, w.N, w.d, causal=True,
+                               promote=(q, k, v, meang, gl, gc))
+    assert lib.qattn_check_device_status() == 0
+    ol, oc = oracle.block_select(np16(q), np16(k), 1, 1, 1, w.N, w.d, True, topk)
+    _lists_equal(gl, gc, ol, oc)
+    qh, kh, vh = np16(q[0]), np16(k[0]), np16(v[0])
+    qn = oracle.quant_nvfp4(qh.view(np.float16))
+    kn = oracle.quant_nvfp4(kh.view(np.float16), mean=mean)
+    vn = oracle.quant_nvfp4(vh.view(np.float16), along_rows=True)
+    for mine, ref in ((gq, qn), (gk, kn), (gv, vn)):
+        for a, r in zip(mine, ref):
+            assert np.array_equal(a.cpu().numpy(), r)
+    mask = oracle.tile_mask(ol, oc, w.N)
+    assert mask[0, -1, -1] and mask[0, -1, -2]
+    rows_i = np.array([0, 255, 256, 65535, w.N - 257, w.N - 129, w.N - 128, w.N - 1], dtype=np.int64)
+    ref, slack = oracle.attention_nvfp4(qn, kn, vn, 1, 1, 1, w.N, w.d, True,
+                                        rows=(np.zeros_like(rows_i), rows_i), promote=mask,
+                                        q16=qh, k16=kh, v16=vh, k_mean=mean)
+    got = out[0, 0, torch.from_numpy(rows_i).cuda()].float().cpu().numpy()
+    _check_fp4_out(got, ref, slack, "long128k promoted, 1024 tiles")
+
+
 @pytest.mark.parametrize("name,over,topk", [("llama8b_32k", {"H": 4, "Hkv": 2, "N": 700}, 2),
                                             ("tiny", {"N": 300}, -1),
                                             ("wide64", {"B": 2, "H": 2, "Hkv": 1, "N": 400,
